@@ -1,0 +1,361 @@
+/*
+ * oracle.c -- plain fp64 CPU reference for shared-prefix attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file; only the tests, the smoke check and the CPU-baseline leg
+ * of the benchmark do.  It shares no code, header or table with the CUDA
+ * library.
+ *
+ * Every function here is the *definition* of the quantity, written out with
+ * no blocking, fusion or reordering: for each (query row, query head) the
+ * logits of every visible key are formed in fp64, then the softmax-weighted
+ * sum of the value rows and the natural-log log-sum-exp of the logits.
+ * Subtracting the row maximum before exponentiating is the only
+ * rearrangement, and it is exact in real arithmetic.
+ *
+ * Sources (web pages, by title and section):
+ *  - "KV-0 redundancy prefix sharing attention mask design" (PrefixSharing
+ *    PR #50), design summary: the prefix K/V is stored once in a flat,
+ *    deduplicated layout [prefix; s_1; ...; s_N]; visibility comes from a
+ *    block-causal mask; one forward pass is mathematically equivalent to
+ *    running every [prefix; s_i] on its own.  Key changes, section 2: the
+ *    mask for the flat GRPO case and for multi-level tree / chain cases.
+ *  - "Split-KV flash-decode attention for EAGLE target-verify" (sglang PR
+ *    #27382), implementation breakdown item 1: verify queries attend to the
+ *    whole cached prefix plus a small causal draft-draft block.
+ *  - "SM8x sparse-MLA prefill fallback re-reads the shared MLA latent once
+ *    per head" (vLLM issue), environment: one shared 512-wide latent serves
+ *    as both K and V for all 64 heads; every query attends to its own top-k
+ *    index list (index_topk = 2048).
+ *
+ * Readings where the pages are silent (also listed in the design notes):
+ *  - Segments form a tree in flat order, parents before children.  A query
+ *    in segment s sees key k iff k <= q and the segment of k is s or one of
+ *    its ancestors.  Flat GRPO is the depth-2 tree; a chain is a path.
+ *  - GQA maps query head h to KV head h / (Hq / Hkv).
+ *  - LSE is the natural log of the sum of exp(scaled logits).
+ *  - A row with no visible key gets O = 0 and LSE = -inf.
+ *
+ * Inputs are fp32 arrays that hold the exact values the GPU reads (bf16
+ * inputs are widened without rounding); all arithmetic is fp64.
+ * Threads split the list of rows; each (row, head) is computed by one thread
+ * in one pass, so threading changes no arithmetic.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0 /* tests build deliberately broken copies with 1..N */
+#endif
+
+/* ------------------------------------------------------------------ */
+/* segment-tree visibility                                              */
+/* ------------------------------------------------------------------ */
+
+/* Segment index of every flat token.  seg_start is ascending. */
+static void token_segments(const int32_t *seg_start, const int32_t *seg_len,
+                           int nseg, int T, int32_t *tok_seg) {
+    for (int t = 0; t < T; ++t) tok_seg[t] = -1;
+    for (int s = 0; s < nseg; ++s)
+        for (int t = seg_start[s]; t < seg_start[s] + seg_len[s]; ++t)
+            if (t >= 0 && t < T) tok_seg[t] = s;
+}
+
+/* 1 iff segment a is segment s or one of its ancestors. */
+static int ancestor_or_self(const int32_t *parent, int a, int s) {
+    while (s >= 0) {
+        if (s == a) return 1;
+        s = parent[s];
+    }
+    return 0;
+}
+
+static int visible(const int32_t *tok_seg, const int32_t *parent, int q, int k) {
+#if ORACLE_MUTANT == 2
+    if (k >= q) return 0;         /* planted: strict causality drops the diagonal */
+#else
+    if (k > q) return 0;
+#endif
+    int sq = tok_seg[q], sk = tok_seg[k];
+    if (sq < 0 || sk < 0) return 0;
+#if ORACLE_MUTANT == 4
+    return sq == sk;              /* planted: suffixes no longer see the prefix */
+#else
+    return ancestor_or_self(parent, sk, sq);
+#endif
+}
+
+/* Dense visibility rows [row0, row0 + nrows) x [0, T) as bytes. */
+int oracle_visibility(const int32_t *seg_start, const int32_t *seg_len,
+                      const int32_t *parent, int nseg, int T, int row0,
+                      int nrows, uint8_t *out) {
+    int32_t *tok_seg = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1));
+    if (!tok_seg) return -1;
+    token_segments(seg_start, seg_len, nseg, T, tok_seg);
+    for (int r = 0; r < nrows; ++r)
+        for (int k = 0; k < T; ++k)
+            out[(size_t)r * T + k] = (uint8_t)visible(tok_seg, parent, row0 + r, k);
+    free(tok_seg);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* one softmax-attention row: the definition                            */
+/* ------------------------------------------------------------------ */
+
+/* Given the logits z[0..n) of the visible keys and pointers to their value
+ * rows, write O (length d) and return the LSE. */
+static double softmax_row(const double *z, const float *const *vrows, int n,
+                          int d, double *o) {
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    if (n == 0) return -INFINITY;
+    double m = -INFINITY;
+    for (int i = 0; i < n; ++i) if (z[i] > m) m = z[i];
+    double l = 0.0;
+    for (int i = 0; i < n; ++i) l += exp(z[i] - m);
+    for (int i = 0; i < n; ++i) {
+        double p = exp(z[i] - m) / l;
+        for (int c = 0; c < d; ++c) o[c] += p * (double)vrows[i][c];
+    }
+#if ORACLE_MUTANT == 5
+    return log(l);                /* planted: LSE forgets the row maximum */
+#else
+    return m + log(l);
+#endif
+}
+
+static double dot(const float *a, const float *b, int d) {
+    double s = 0.0;
+    for (int c = 0; c < d; ++c) s += (double)a[c] * (double)b[c];
+    return s;
+}
+
+static double apply_scale(double qk, double scale) {
+#if ORACLE_MUTANT == 1
+    (void)scale;
+    return qk;                    /* planted: the softmax scale is dropped */
+#else
+    return scale * qk;
+#endif
+}
+
+static int kv_head_of(int h, int Hq, int Hkv) {
+#if ORACLE_MUTANT == 3
+    (void)Hq;
+    return h % Hkv;               /* planted: interleaved instead of contiguous GQA */
+#else
+    return h / (Hq / Hkv);
+#endif
+}
+
+/* ------------------------------------------------------------------ */
+/* threading helper: rows are split into contiguous ranges               */
+/* ------------------------------------------------------------------ */
+
+typedef void (*row_fn)(void *ctx, int r, double *zbuf, const float **vbuf, double *obuf);
+
+typedef struct {
+    row_fn fn;
+    void *ctx;
+    int r0, r1;
+    int zcap, d;
+} worker_arg;
+
+static void *worker(void *p) {
+    worker_arg *w = (worker_arg *)p;
+    double *z = (double *)malloc(sizeof(double) * (size_t)(w->zcap > 0 ? w->zcap : 1));
+    const float **vr = (const float **)malloc(sizeof(float *) * (size_t)(w->zcap > 0 ? w->zcap : 1));
+    double *o = (double *)malloc(sizeof(double) * (size_t)w->d);
+    if (z && vr && o)
+        for (int r = w->r0; r < w->r1; ++r) w->fn(w->ctx, r, z, vr, o);
+    free(z);
+    free((void *)vr);
+    free(o);
+    return NULL;
+}
+
+static void run_rows(row_fn fn, void *ctx, int nrows, int zcap, int d, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > nrows) nthreads = nrows > 0 ? nrows : 1;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    worker_arg *args = (worker_arg *)malloc(sizeof(worker_arg) * (size_t)nthreads);
+    for (int i = 0; i < nthreads; ++i) {
+        args[i].fn = fn;
+        args[i].ctx = ctx;
+        args[i].r0 = (int)((int64_t)nrows * i / nthreads);
+        args[i].r1 = (int)((int64_t)nrows * (i + 1) / nthreads);
+        args[i].zcap = zcap;
+        args[i].d = d;
+        pthread_create(&th[i], NULL, worker, &args[i]);
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+    free(args);
+}
+
+/* ------------------------------------------------------------------ */
+/* prefill over the flat packed layout                                  */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const float *q, *k, *v;
+    int T, Hq, Hkv, d;
+    double scale;
+    const int32_t *tok_seg, *parent;
+    const int32_t *rows;
+    double *o, *lse;
+} prefill_ctx;
+
+static void prefill_row(void *p, int r, double *z, const float **vr, double *o) {
+    prefill_ctx *c = (prefill_ctx *)p;
+    int qi = c->rows[r];
+    for (int h = 0; h < c->Hq; ++h) {
+        int kvh = kv_head_of(h, c->Hq, c->Hkv);
+        const float *qrow = c->q + ((size_t)qi * c->Hq + h) * c->d;
+        int n = 0;
+        for (int kj = 0; kj < c->T; ++kj) {
+            if (!visible(c->tok_seg, c->parent, qi, kj)) continue;
+            const float *krow = c->k + ((size_t)kj * c->Hkv + kvh) * c->d;
+            z[n] = apply_scale(dot(qrow, krow, c->d), c->scale);
+            vr[n] = c->v + ((size_t)kj * c->Hkv + kvh) * c->d;
+            ++n;
+        }
+        double l = softmax_row(z, vr, n, c->d, o);
+        memcpy(c->o + ((size_t)r * c->Hq + h) * c->d, o, sizeof(double) * (size_t)c->d);
+        c->lse[(size_t)r * c->Hq + h] = l;
+    }
+}
+
+/*
+ * q [T, Hq, d], k/v [T, Hkv, d] (fp32 holding the exact input values),
+ * segments (seg_start, seg_len, parent) over the flat token range [0, T),
+ * rows[nrows] = the flat query rows to evaluate.
+ * o [nrows, Hq, d], lse [nrows, Hq] (fp64).
+ */
+int oracle_prefill(const float *q, const float *k, const float *v, int T, int Hq,
+                   int Hkv, int d, double scale, const int32_t *seg_start,
+                   const int32_t *seg_len, const int32_t *parent, int nseg,
+                   const int32_t *rows, int nrows, double *o, double *lse,
+                   int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || T < 0) return -1;
+    int32_t *tok_seg = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1));
+    if (!tok_seg) return -1;
+    token_segments(seg_start, seg_len, nseg, T, tok_seg);
+    prefill_ctx c = {q, k, v, T, Hq, Hkv, d, scale, tok_seg, parent, rows, o, lse};
+    run_rows(prefill_row, &c, nrows, T, d, nthreads);
+    free(tok_seg);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* speculative verify: cached prefix plus a causal draft block          */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const float *qd, *kd, *vd, *kc, *vc;
+    const int64_t *indptr;
+    int Ld, Hq, Hkv, d;
+    double scale;
+    const int32_t *rows;
+    double *o, *lse;
+} verify_ctx;
+
+static void verify_row(void *p, int r, double *z, const float **vr, double *o) {
+    verify_ctx *c = (verify_ctx *)p;
+    int row = c->rows[r]; /* row = b * Ld + j */
+    int b = row / c->Ld, j = row % c->Ld;
+    int64_t p0 = c->indptr[b], p1 = c->indptr[b + 1];
+    for (int h = 0; h < c->Hq; ++h) {
+        int kvh = kv_head_of(h, c->Hq, c->Hkv);
+        const float *qrow = c->qd + ((size_t)row * c->Hq + h) * c->d;
+        int n = 0;
+        for (int64_t t = p0; t < p1; ++t) { /* the whole cached prefix */
+            const float *krow = c->kc + ((size_t)t * c->Hkv + kvh) * c->d;
+            z[n] = apply_scale(dot(qrow, krow, c->d), c->scale);
+            vr[n] = c->vc + ((size_t)t * c->Hkv + kvh) * c->d;
+            ++n;
+        }
+#if ORACLE_MUTANT == 6
+        for (int i = 0; i < c->Ld; ++i) {  /* planted: the draft block is not causal */
+#else
+        for (int i = 0; i <= j; ++i) {     /* drafts 0..j: the causal draft block */
+#endif
+            size_t dr = (size_t)b * c->Ld + i;
+            const float *krow = c->kd + (dr * c->Hkv + kvh) * c->d;
+            z[n] = apply_scale(dot(qrow, krow, c->d), c->scale);
+            vr[n] = c->vd + (dr * c->Hkv + kvh) * c->d;
+            ++n;
+        }
+        double l = softmax_row(z, vr, n, c->d, o);
+        memcpy(c->o + ((size_t)r * c->Hq + h) * c->d, o, sizeof(double) * (size_t)c->d);
+        c->lse[(size_t)r * c->Hq + h] = l;
+    }
+}
+
+/*
+ * q_draft [B*Ld, Hq, d]; k_draft/v_draft [B*Ld, Hkv, d];
+ * k_cache/v_cache [Ntok, Hkv, d]; request b's prefix is cache tokens
+ * [indptr[b], indptr[b+1]).  rows = draft rows b*Ld + j to evaluate.
+ */
+int oracle_verify(const float *qd, const float *kd, const float *vd,
+                  const float *kc, const float *vc, const int64_t *indptr,
+                  int B, int Ld, int Hq, int Hkv, int d, double scale,
+                  const int32_t *rows, int nrows, double *o, double *lse,
+                  int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || B < 0 || Ld <= 0) return -1;
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b)
+        if (indptr[b + 1] - indptr[b] > maxlen) maxlen = indptr[b + 1] - indptr[b];
+    verify_ctx c = {qd, kd, vd, kc, vc, indptr, Ld, Hq, Hkv, d, scale, rows, o, lse};
+    run_rows(verify_row, &c, nrows, (int)maxlen + Ld, d, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* shared-latent sparse attention over per-query index lists            */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const float *q, *lat;
+    const int32_t *idx;
+    int H, dl, topk;
+    double scale;
+    const int32_t *rows;
+    double *o, *lse;
+} sparse_ctx;
+
+static void sparse_row(void *p, int r, double *z, const float **vr, double *o) {
+    sparse_ctx *c = (sparse_ctx *)p;
+    int t = c->rows[r];
+    const int32_t *list = c->idx + (size_t)t * c->topk;
+    for (int h = 0; h < c->H; ++h) {
+        const float *qrow = c->q + ((size_t)t * c->H + h) * c->dl;
+        int n = 0;
+        for (int i = 0; i < c->topk; ++i) {
+            int32_t kj = list[i];
+            if (kj < 0) continue;        /* -1 pads a short list */
+            const float *lrow = c->lat + (size_t)kj * c->dl; /* K = V = latent */
+            z[n] = apply_scale(dot(qrow, lrow, c->dl), c->scale);
+            vr[n] = lrow;
+            ++n;
+        }
+        double l = softmax_row(z, vr, n, c->dl, o);
+        memcpy(c->o + ((size_t)r * c->H + h) * c->dl, o, sizeof(double) * (size_t)c->dl);
+        c->lse[(size_t)r * c->H + h] = l;
+    }
+}
+
+/* q [T, H, dl]; latent [Tk, dl]; idx [T, topk] (-1 = pad). */
+int oracle_sparse_latent(const float *q, const float *lat, const int32_t *idx,
+                         int T, int H, int dl, int topk, double scale,
+                         const int32_t *rows, int nrows, double *o, double *lse,
+                         int nthreads) {
+    (void)T;
+    if (H <= 0 || dl <= 0 || topk < 0) return -1;
+    sparse_ctx c = {q, lat, idx, H, dl, topk, scale, rows, o, lse};
+    run_rows(sparse_row, &c, nrows, topk, dl, nthreads);
+    return 0;
+}

@@ -1,0 +1,269 @@
+"""Seeded synthetic inputs shaped like the workloads on the pages.
+
+This module draws random numbers and lays out shapes; it holds none of the
+attention arithmetic, so both the CUDA path and the fp64 oracle can consume
+what it produces (the same bytes go to both sides).
+
+Workloads (sizes as named; Q/K/V ~ N(0,1) * sigma, rounded once to the
+storage dtype):
+
+* ``tiny``   -- one prefix P=64 plus N=4 suffixes of S=32, 2 heads, d=64, fp32.
+* ``grpo``   -- GRPO rollout group P=2048, N=8, S=512, 16/16 heads, d=128, bf16.
+* ``large``  -- two packed groups of P=8192, N=16, S=1024, 32 query heads on
+  8 KV heads, d=128, bf16.
+* ``verify`` -- 32 requests, 16384-token cached prefix each, 4 draft tokens,
+  32 query / 8 KV heads, d=128, 32 splits, bf16.
+* ``sparse`` -- 16384 queries, 64 heads on one 512-wide latent, 2048 indices
+  per query drawn from its causal past, bf16.
+
+The flat GRPO layout and the tree segments follow "KV-0 redundancy prefix
+sharing attention mask design" (design summary; key changes section 2).
+The verify shape follows "Split-KV flash-decode attention for EAGLE
+target-verify" (motivation: 16k context; test shapes: 4 draft tokens).
+The sparse shape follows "SM8x sparse-MLA prefill fallback re-reads the
+shared MLA latent once per head" (environment: 16384 tokens, 64 heads,
+index_topk 2048, kv_lora_rank 512, no rope part).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+
+# --------------------------------------------------------------------------
+# segment trees
+# --------------------------------------------------------------------------
+
+def grpo_segments(P: int, N: int, S: int, groups: int = 1) -> list[tuple[int, int]]:
+    """(len, parent) per segment in flat order: for each group, the prefix
+    (a root) followed by N suffixes whose parent is that prefix.  A group
+    with P == 0 has no prefix segment: its N suffixes are roots."""
+    segs: list[tuple[int, int]] = []
+    for _ in range(groups):
+        if P > 0:
+            root = len(segs)
+            segs.append((P, -1))
+            segs.extend((S, root) for _ in range(N))
+        else:
+            segs.extend((S, -1) for _ in range(N))
+    return segs
+
+
+def chain_segments(lens: list[int]) -> list[tuple[int, int]]:
+    """A chain: segment i's parent is segment i-1."""
+    return [(n, i - 1) for i, n in enumerate(lens)]
+
+
+def random_tree_segments(gen: torch.Generator, nseg: int, max_len: int,
+                         groups: int = 1) -> list[tuple[int, int]]:
+    """A random forest in flat order (parents precede children)."""
+    segs: list[tuple[int, int]] = []
+    for _ in range(groups):
+        base = len(segs)
+        for i in range(nseg):
+            ln = int(torch.randint(1, max_len + 1, (1,), generator=gen))
+            if i == 0:
+                par = -1
+            else:
+                par = int(torch.randint(-1, i, (1,), generator=gen))
+                par = -1 if par < 0 else base + par
+            segs.append((ln, par))
+    return segs
+
+
+def group_indptr(segments, segs_per_group: list[int]) -> list[int]:
+    out = [0]
+    for n in segs_per_group:
+        out.append(out[-1] + n)
+    return out
+
+
+# --------------------------------------------------------------------------
+# workloads
+# --------------------------------------------------------------------------
+
+@dataclass
+class PrefillWorkload:
+    name: str
+    P: int
+    N: int
+    S: int
+    Hq: int
+    Hkv: int
+    d: int
+    groups: int = 1
+    dtype: torch.dtype = torch.bfloat16
+    sigma: float = 0.5
+    seed: int = 2
+
+    @property
+    def group_len(self) -> int:
+        return self.P + self.N * self.S
+
+    @property
+    def T(self) -> int:
+        return self.groups * self.group_len
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def segments(self):
+        return grpo_segments(self.P, self.N, self.S, self.groups)
+
+    def seg_indptr(self) -> list[int]:
+        per = (self.N + 1) if self.P > 0 else self.N
+        return [g * per for g in range(self.groups + 1)]
+
+    def cu_seqlens(self) -> list[int]:
+        return [g * self.group_len for g in range(self.groups + 1)]
+
+    def visible_pairs_per_head(self) -> int:
+        """Exact visible (q, k) pairs per query head (closed form for the
+        flat GRPO tree): causal prefix plus, per suffix, the whole prefix and
+        its own causal triangle."""
+        P, N, S = self.P, self.N, self.S
+        per_group = P * (P + 1) // 2 + N * (S * P + S * (S + 1) // 2)
+        return self.groups * per_group
+
+    def flops(self) -> float:
+        """4 * d * Hq * visible pairs (QK^T and PV, 2 flops per MAC)."""
+        return 4.0 * self.d * self.Hq * self.visible_pairs_per_head()
+
+    def make(self, device="cpu", seed: int | None = None):
+        g = torch.Generator(device=device)
+        g.manual_seed(self.seed if seed is None else seed)
+        T = self.T
+
+        def draw(shape):
+            x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+            return (x * self.sigma).to(self.dtype)
+
+        q = draw((T, self.Hq, self.d))
+        k = draw((T, self.Hkv, self.d))
+        v = draw((T, self.Hkv, self.d))
+        return q, k, v
+
+
+@dataclass
+class VerifyWorkload:
+    name: str
+    B: int
+    L: int
+    Ld: int
+    Hq: int
+    Hkv: int
+    d: int
+    nsplit: int
+    dtype: torch.dtype = torch.bfloat16
+    sigma: float = 0.5
+    seed: int = 4
+    prefix_lens: list[int] | None = None   # ragged prefixes (default: all L)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def lens(self) -> list[int]:
+        return list(self.prefix_lens) if self.prefix_lens is not None else [self.L] * self.B
+
+    def kv_indptr(self) -> list[int]:
+        out = [0]
+        for n in self.lens():
+            out.append(out[-1] + n)
+        return out
+
+    def prefix_kv_bytes(self) -> int:
+        """Prefix K and V bytes read once: sum(L_b) * Hkv * d * 2 tensors * elem."""
+        elem = torch.tensor([], dtype=self.dtype).element_size()
+        return sum(self.lens()) * self.Hkv * self.d * 2 * elem
+
+    def make(self, device="cpu", seed: int | None = None):
+        g = torch.Generator(device=device)
+        g.manual_seed(self.seed if seed is None else seed)
+        ntok = sum(self.lens())
+        BL = self.B * self.Ld
+
+        def draw(shape):
+            x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+            return (x * self.sigma).to(self.dtype)
+
+        q = draw((BL, self.Hq, self.d))
+        kd = draw((BL, self.Hkv, self.d))
+        vd = draw((BL, self.Hkv, self.d))
+        kc = draw((ntok, self.Hkv, self.d))
+        vc = draw((ntok, self.Hkv, self.d))
+        return q, kd, vd, kc, vc
+
+
+@dataclass
+class SparseLatentWorkload:
+    name: str
+    T: int
+    H: int
+    dl: int
+    topk: int
+    dtype: torch.dtype = torch.bfloat16
+    sigma: float = 0.5
+    seed: int = 5
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.dl)
+
+    def pairs(self) -> int:
+        return sum(min(t + 1, self.topk) for t in range(self.T))
+
+    def flops(self) -> float:
+        return 4.0 * self.dl * self.H * self.pairs()
+
+    def make_indices(self, g: torch.Generator, device="cpu") -> torch.Tensor:
+        """[T, topk] int32.  Row t < topk lists 0..t then -1 padding (dense
+        causal); row t >= topk lists topk distinct positions drawn uniformly
+        without replacement from [0, t], sorted ascending."""
+        T, K = self.T, self.topk
+        idx = torch.full((T, K), -1, dtype=torch.int32, device=device)
+        dense = min(T, K)
+        ar = torch.arange(K, device=device, dtype=torch.int32)
+        tri = torch.where(ar[None, :] <= torch.arange(dense, device=device,
+                                                       dtype=torch.int32)[:, None],
+                          ar[None, :], torch.full_like(ar[None, :], -1))
+        idx[:dense] = tri
+        block = 256
+        for r0 in range(K, T, block):
+            r1 = min(T, r0 + block)
+            width = r1  # positions 0 .. r1-1 cover every row's causal past
+            u = torch.rand((r1 - r0, width), generator=g, device=device)
+            pos = torch.arange(width, device=device)
+            rows = torch.arange(r0, r1, device=device)
+            u = torch.where(pos[None, :] <= rows[:, None], u, torch.full_like(u, -1.0))
+            pick = torch.topk(u, K, dim=1).indices
+            idx[r0:r1] = torch.sort(pick, dim=1).values.to(torch.int32)
+        return idx
+
+    def make(self, device="cpu", seed: int | None = None):
+        g = torch.Generator(device=device)
+        g.manual_seed(self.seed if seed is None else seed)
+
+        def draw(shape):
+            x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+            return (x * self.sigma).to(self.dtype)
+
+        q = draw((self.T, self.H, self.dl))
+        lat = draw((self.T, self.dl))
+        idx = self.make_indices(g, device)
+        return q, lat, idx
+
+
+TINY = PrefillWorkload("tiny P=64 N=4 S=32 H=2 d=64 fp32", P=64, N=4, S=32, Hq=2, Hkv=2,
+                       d=64, dtype=torch.float32, sigma=1.0, seed=1)
+GRPO = PrefillWorkload("grpo P=2048 N=8 S=512 H=16/16 d=128 bf16", P=2048, N=8, S=512,
+                       Hq=16, Hkv=16, d=128, seed=2)
+LARGE = PrefillWorkload("large 2x(P=8192 N=16 S=1024) H=32/8 d=128 bf16", P=8192, N=16,
+                        S=1024, Hq=32, Hkv=8, d=128, groups=2, seed=3)
+VERIFY = VerifyWorkload("verify B=32 L=16384 drafts=4 H=32/8 d=128 splits=32 bf16", B=32,
+                        L=16384, Ld=4, Hq=32, Hkv=8, d=128, nsplit=32, seed=4)
+SPARSE = SparseLatentWorkload("sparse T=16384 H=64 dl=512 topk=2048 bf16", T=16384, H=64,
+                              dl=512, topk=2048, seed=5)
