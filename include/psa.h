@@ -1,0 +1,240 @@
+/*
+ * psa.h -- C ABI of libpsa: shared-prefix attention over a flat,
+ * deduplicated packed layout, for NVIDIA B200 (sm_100a).
+ *
+ * Page references are by title and section:
+ *   [PS]  "KV-0 redundancy prefix sharing attention mask design"
+ *         (PrefixSharing PR #50)
+ *   [SKV] "Split-KV flash-decode attention for EAGLE target-verify"
+ *         (sglang PR #27382)
+ *   [MLA] "SM8x sparse-MLA prefill fallback re-reads the shared MLA latent
+ *         once per head" (vLLM issue write-up)
+ *
+ * Conventions shared by every call:
+ *   - Every function returns an int status (psa_status).  Nothing throws
+ *     across this boundary.
+ *   - Pointers named dev_* or documented as "device" are CUDA device
+ *     pointers; all other pointers are host memory.  All buffers are owned
+ *     by the caller; the library allocates and frees nothing and never
+ *     synchronises the host with the device.
+ *   - GPU work is enqueued on the caller's stream (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream) and returns before it runs.
+ *   - Tensors are dense, row-major and token-major, as documented per call.
+ *     Every device pointer must be 16-byte aligned.
+ *   - dev_status (nullable) is a device int32 the caller zeroes; a kernel
+ *     that gives up on a bounded wait writes PSA_ERR_TIMEOUT there instead
+ *     of hanging.  Read it with psa_read_status after the stream drains.
+ *   - Arithmetic: bf16 inputs, fp32 accumulation, bf16 output; LSE is fp32
+ *     natural-log of the sum of exp(scale * q.k) over visible keys.
+ *   - GQA: query head h reads KV head h / (Hq / Hkv).
+ */
+#ifndef PSA_H
+#define PSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+#if defined(__GNUC__)
+#pragma GCC visibility push(default) /* the ABI stays visible under -fvisibility=hidden */
+#endif
+
+#define PSA_VERSION 1
+
+typedef enum psa_status {
+    PSA_OK = 0,
+    PSA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned, inconsistent shapes */
+    PSA_ERR_UNSUPPORTED = 2,  /* a feature outside what the kernels implement */
+    PSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than *_workspace_size */
+    PSA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+    PSA_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up (via dev_status) */
+    PSA_ERR_CAPACITY = 6      /* a host output array is too small; *nout holds the need */
+} psa_status;
+
+typedef enum psa_dtype {
+    PSA_BF16 = 0,
+    PSA_F32 = 1
+} psa_dtype;
+
+/* Library version (PSA_VERSION) and a static string for a status code. */
+int psa_version(void);
+const char *psa_status_string(int status);
+
+/* ------------------------------------------------------------------------
+ * Mask spec (host only)                                      [PS] key changes s.2
+ * --------------------------------------------------------------------- */
+
+/* One segment of the flat layout: `len` tokens; `parent` is the global
+ * index of the parent segment or -1 for a root.  Segments are listed in
+ * flat order, parents before children; consecutive segments are adjacent
+ * in the flat token range. */
+typedef struct psa_segment {
+    int32_t len;
+    int32_t parent;
+} psa_segment;
+
+/* A visibility rectangle over flat token indices: queries [q0, q1) see keys
+ * [k0, k1); if causal, only where q - q0 >= k - k0 (top-left aligned). */
+typedef struct psa_rect {
+    int32_t q0, q1, k0, k1;
+    int32_t causal;
+} psa_rect;
+
+/* Segments of the flat GRPO layout [PS] design summary: one prefix of P
+ * tokens stored once, then N suffixes of S tokens, each child of the
+ * prefix.  P == 0 gives N independent roots.  Writes N+1 (or N) segments.
+ * Returns PSA_ERR_CAPACITY (with *nout set) if cap is too small. */
+int psa_spec_flat(int32_t P, int32_t N, int32_t S, psa_segment *out, int32_t cap,
+                  int32_t *nout);
+
+/* Rectangle spec from a segment forest [PS] design summary ("a rectangle
+ * spec rather than a full mask") and key changes s.2 (flat GRPO and
+ * multi-level tree / chain cases).  Each segment sees every ancestor
+ * segment fully and itself causally, so the rectangles are disjoint and
+ * together cover exactly the visible (q, k) pairs.  No dense mask is ever
+ * formed.  segs: nseg segments (flat order, all groups back to back).
+ * Returns PSA_ERR_INVALID_ARG for a parent that does not precede its child
+ * or a non-positive length; PSA_ERR_CAPACITY if cap < the rect count. */
+int psa_build_spec(const psa_segment *segs, int32_t nseg, psa_rect *out, int32_t cap,
+                   int32_t *nout);
+
+/* Tile schedule for psa_prefill_fwd (host int32 array).  Q tiles of tile_m
+ * rows and KV tiles of tile_n keys are cut per group (cu_seqlens, host,
+ * ngroups+1 entries); for every Q tile it lists only the KV tiles with at
+ * least one visible pair, flagging each as fully visible or partial, and
+ * for partial tiles it copies the rectangles that cut them.  Q tiles are
+ * ordered longest-first (most KV tiles first).
+ *
+ * Layout (int32):  [0] magic 0x50534131  [1] n_items  [2] n_kv  [3] n_rect
+ *   [4] tile_m  [5] tile_n  [6] total tokens  [7] max KV tiles per item
+ *   items   at 8:                  {q0, q_len, kv_begin, kv_count} x n_items
+ *   kv      at 8 + 4*n_items:      {k0, k_len, rect_begin, rect_count} x n_kv
+ *                                  (rect_count == 0: every pair visible)
+ *   rects   at 8 + 4*(n_items+n_kv): {q0, q1, k0, k1, causal} x n_rect
+ * Returns PSA_ERR_CAPACITY (with *nout = needed length) if cap is short. */
+int psa_build_schedule(const psa_rect *rects, int32_t nrect, const int32_t *cu_seqlens,
+                       int32_t ngroups, int32_t tile_m, int32_t tile_n, int32_t *out,
+                       int64_t cap, int64_t *nout);
+
+/* The tile sizes psa_prefill_fwd expects in its schedule (tile_m, tile_n). */
+int psa_prefill_tiles(int32_t head_dim, int32_t *tile_m, int32_t *tile_n);
+
+/* ------------------------------------------------------------------------
+ * Prefill over the packed layout          [PS] design summary, key changes
+ * --------------------------------------------------------------------- */
+
+/* Workspace bytes psa_prefill_fwd needs (PSA_F32 inputs are converted to
+ * bf16 into it; the tile scheduler keeps its counter there). */
+size_t psa_prefill_workspace_size(int dtype, int32_t T, int32_t Hq, int32_t Hkv,
+                                  int32_t head_dim);
+
+/* One forward pass of softmax attention over the flat layout with the
+ * visibility described by dev_schedule (device copy of a
+ * psa_build_schedule result, sched_len int32).
+ *   q   device [T, Hq, d]      dtype (PSA_BF16 or PSA_F32)
+ *   k,v device [T, Hkv, d]     dtype
+ *   o   device [T, Hq, d]      dtype (written)
+ *   lse device [T, Hq] fp32    (written; nullable)
+ * d in {64, 128}; Hq % Hkv == 0.  Rows with no visible key (none occur for
+ * a valid spec) are written as O = 0, LSE = -inf.
+ * workspace: device, >= psa_prefill_workspace_size bytes, 256-B aligned. */
+int psa_prefill_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                    int dtype, int32_t T, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                    float scale, const int32_t *dev_schedule, int64_t sched_len,
+                    void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Speculative verify: split-KV over the cached prefix, then an LSE combine
+ * that folds in the causal draft block.   [SKV] implementation item 1
+ * --------------------------------------------------------------------- */
+
+/* Features of the general extend-attention call that the split-KV path
+ * does not implement ([SKV] key code: can_handle).  Pass NULL for the
+ * supported case; any non-default field makes psa_verify_fwd return
+ * PSA_ERR_UNSUPPORTED (there is no fallback path). */
+typedef struct psa_verify_features {
+    int32_t has_custom_mask;     /* tree drafts (topk > 1) carry a custom mask */
+    int32_t is_causal;           /* must be 1 */
+    int32_t sliding_window;      /* must be <= 0 */
+    int32_t has_sinks;           /* must be 0 */
+    float logit_cap;             /* must be 0 */
+    int32_t xai_temperature_len; /* must be <= 0 */
+    int32_t ragged_extend;       /* per-request draft counts differ: must be 0 */
+} psa_verify_features;
+
+/* Split count chosen when nsplit == 0: enough (request, split) units to
+ * fill the GPU, each covering a whole number of key tiles. */
+int32_t psa_verify_auto_splits(int32_t B, int64_t max_prefix_len, int32_t Hkv,
+                               int32_t head_dim);
+
+/* Workspace bytes for the split partials: nsplit * B*Ld*Hq * (d + 1) fp32,
+ * plus alignment padding.  Size it for the largest batch you will run and
+ * reuse it ([SKV] review: key scratch by the maximum batch, not by the
+ * current one). */
+size_t psa_verify_workspace_size(int32_t B, int32_t Ld, int32_t Hq, int32_t head_dim,
+                                 int32_t nsplit);
+
+/*
+ *   q_draft          device [B*Ld, Hq, d] bf16   draft-token queries, request-major
+ *   k_draft, v_draft device [B*Ld, Hkv, d] bf16  draft-token keys/values
+ *   k_cache, v_cache device [Ntok, Hkv, d] bf16  cached prefix, one contiguous
+ *                                                token range per request
+ *   n_cache_tokens   host value Ntok (rows of k_cache / v_cache)
+ *   dev_kv_indptr    device int32 [B+1]         request b's prefix is cache tokens
+ *                                                [indptr[b], indptr[b+1])
+ *   max_prefix_len   host value >= every prefix length (no device sync is made)
+ *   kv_indices       must be NULL (paged caches are not implemented:
+ *                    PSA_ERR_UNSUPPORTED)
+ *   o                device [B*Ld, Hq, d] bf16   (written)
+ *   lse              device [B*Ld, Hq] fp32      (written; nullable)
+ * Draft j of request b sees the whole prefix of b plus drafts 0..j.
+ * d in {64, 128, 256}; Hq % Hkv == 0; Ld * Hq / Hkv <= 128.
+ * nsplit in [1, 256], or 0 for psa_verify_auto_splits.  Split s of request
+ * b covers prefix tokens [s*c, min((s+1)*c, L_b)) with c = ceil(L_b/nsplit)
+ * rounded up to the key tile; empty splits contribute nothing.
+ */
+int psa_verify_fwd(const void *q_draft, const void *k_draft, const void *v_draft,
+                   const void *k_cache, const void *v_cache, int64_t n_cache_tokens,
+                   const int32_t *dev_kv_indptr,
+                   int64_t max_prefix_len, const int32_t *kv_indices, void *o, float *lse,
+                   int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                   float scale, int32_t nsplit, const psa_verify_features *features,
+                   void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Shared-latent sparse attention                     [MLA] environment,
+ * analysis (head-blocked tiles; the latent is shared by every head)
+ * --------------------------------------------------------------------- */
+
+/*
+ *   q       device [T, H, dl] bf16     queries, all heads of a token together
+ *   latent  device [Tk, dl] bf16       the one shared latent: K = V = latent
+ *   idx     device [T, topk] int32     per-query key rows; -1 entries are
+ *                                      skipped; others must be in [0, Tk)
+ *   o       device [T, H, dl] bf16     (written)
+ *   lse     device [T, H] fp32         (written; nullable)
+ * dl == 512, H <= 128, topk >= 1.  Row t attends to the listed latent rows
+ * only; a row whose list is all -1 gets O = 0 and LSE = -inf.
+ */
+int psa_sparse_latent_fwd(const void *q, const void *latent, const int32_t *idx, void *o,
+                          float *lse, int32_t T, int32_t Tk, int32_t H, int32_t dl,
+                          int32_t topk, float scale, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Status word
+ * --------------------------------------------------------------------- */
+
+/* Copies the device status word to *host_out after draining `stream`.
+ * This is the one call that waits on the device. */
+int psa_read_status(const int32_t *dev_status, int32_t *host_out, void *stream);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PSA_H */

@@ -1,0 +1,252 @@
+// C-ABI layer of libpsa: argument validation, workspace sizing and kernel
+// launches.  No allocation, no host synchronisation (psa_read_status
+// excepted), no fallback: an unsupported case returns PSA_ERR_UNSUPPORTED.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "psa.h"
+#include "psa_internal.h"
+
+namespace psa {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+int encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return PSA_ERR_CUDA;
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides_bytes[i];
+  CUresult r = fn(map, dtype, cuuint32_t(rank), const_cast<void*>(base), d, st, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PSA_OK : PSA_ERR_CUDA;
+}
+
+int sm_count(int device) {
+  static int cached[64] = {0};
+  if (device < 0 || device >= 64) return 0;
+  if (cached[device] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+      return 0;
+    cached[device] = n;
+  }
+  return cached[device];
+}
+
+}  // namespace psa
+
+using namespace psa;
+
+extern "C" int psa_version(void) { return PSA_VERSION; }
+
+extern "C" const char* psa_status_string(int status) {
+  switch (status) {
+    case PSA_OK:
+      return "ok";
+    case PSA_ERR_INVALID_ARG:
+      return "invalid argument";
+    case PSA_ERR_UNSUPPORTED:
+      return "unsupported case (no fallback path exists)";
+    case PSA_ERR_WORKSPACE:
+      return "workspace missing or too small";
+    case PSA_ERR_CUDA:
+      return "CUDA call failed";
+    case PSA_ERR_TIMEOUT:
+      return "device-side wait timed out";
+    case PSA_ERR_CAPACITY:
+      return "output capacity too small";
+    default:
+      return "unknown status";
+  }
+}
+
+extern "C" int psa_read_status(const int32_t* dev_status, int32_t* host_out, void* stream) {
+  if (!dev_status || !host_out) return PSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(host_out, dev_status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return PSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return PSA_ERR_CUDA;
+  return PSA_OK;
+}
+
+// ------------------------------------------------------------------ verify
+
+extern "C" int32_t psa_verify_auto_splits(int32_t B, int64_t max_prefix_len, int32_t Hkv,
+                                          int32_t head_dim) {
+  (void)Hkv;
+  (void)head_dim;
+  if (B <= 0 || max_prefix_len <= 0) return 1;
+  // Aim for about four (request, split) units per SM of a 148-SM part, but
+  // keep every split at least 256 keys long so each unit streams enough.
+  const int64_t target_units = 4 * 148;
+  int64_t n = (target_units + B - 1) / B;
+  const int64_t by_len = max_prefix_len / 256;
+  if (n > by_len) n = by_len;
+  if (n < 1) n = 1;
+  if (n > 256) n = 256;
+  return int32_t(n);
+}
+
+extern "C" size_t psa_verify_workspace_size(int32_t B, int32_t Ld, int32_t Hq,
+                                            int32_t head_dim, int32_t nsplit) {
+  if (B <= 0 || Ld <= 0 || Hq <= 0 || head_dim <= 0 || nsplit <= 0) return 0;
+  const size_t rows = size_t(nsplit) * B * Ld * Hq;
+  const size_t o_bytes = (rows * head_dim * sizeof(float) + 255) / 256 * 256;
+  const size_t l_bytes = (rows * sizeof(float) + 255) / 256 * 256;
+  return o_bytes + l_bytes;
+}
+
+extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const void* v_draft,
+                              const void* k_cache, const void* v_cache, int64_t n_cache_tokens,
+                              const int32_t* dev_kv_indptr, int64_t max_prefix_len,
+                              const int32_t* kv_indices, void* o, float* lse, int32_t B,
+                              int32_t Ld, int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
+                              int32_t nsplit, const psa_verify_features* features,
+                              void* workspace, size_t ws_bytes, int32_t* dev_status,
+                              void* stream) {
+  // The split-KV path's gating ("can_handle"): everything else is refused.
+  if (features) {
+    if (features->has_custom_mask || !features->is_causal || features->sliding_window > 0 ||
+        features->has_sinks || features->logit_cap != 0.f ||
+        features->xai_temperature_len > 0 || features->ragged_extend)
+      return PSA_ERR_UNSUPPORTED;
+  }
+  if (kv_indices) return PSA_ERR_UNSUPPORTED;
+  if (B < 0 || Ld <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n_cache_tokens < 0 ||
+      max_prefix_len < 0 || n_cache_tokens > INT32_MAX || !(scale > 0.f))
+    return PSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PSA_ERR_UNSUPPORTED;
+  if (B == 0) return PSA_OK;
+  if (!q_draft || !k_draft || !v_draft || !k_cache || !v_cache || !dev_kv_indptr || !o)
+    return PSA_ERR_INVALID_ARG;
+  if (!aligned16(q_draft) || !aligned16(k_draft) || !aligned16(v_draft) ||
+      !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return PSA_ERR_INVALID_ARG;
+  int32_t HB = 0, MT = 0;
+  if (!verify_plan(Ld, Hq, Hkv, head_dim, &HB, &MT)) return PSA_ERR_UNSUPPORTED;
+  if (nsplit == 0) nsplit = psa_verify_auto_splits(B, max_prefix_len, Hkv, head_dim);
+  if (nsplit < 1 || nsplit > 256) return PSA_ERR_INVALID_ARG;
+  const size_t need = psa_verify_workspace_size(B, Ld, Hq, head_dim, nsplit);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PSA_ERR_WORKSPACE;
+  if (n_cache_tokens == 0) n_cache_tokens = 1;  // a tensor map needs a non-empty extent
+
+  VerifyArgs a;
+  a.q = q_draft;
+  a.kd = k_draft;
+  a.vd = v_draft;
+  a.kc = k_cache;
+  a.vc = v_cache;
+  a.indptr = dev_kv_indptr;
+  a.n_cache_tokens = n_cache_tokens;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.Ld = Ld;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = head_dim;
+  a.scale = scale;
+  a.nsplit = nsplit;
+  const size_t rows = size_t(nsplit) * B * Ld * Hq;
+  const size_t o_bytes = (rows * head_dim * sizeof(float) + 255) / 256 * 256;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + o_bytes);
+  a.status = dev_status;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_verify(a);
+}
+
+// ------------------------------------------------------------------ prefill
+
+extern "C" int psa_prefill_tiles(int32_t head_dim, int32_t* tile_m, int32_t* tile_n) {
+  if (!tile_m || !tile_n) return PSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PSA_ERR_UNSUPPORTED;
+  *tile_m = 128;
+  *tile_n = 128;
+  return PSA_OK;
+}
+
+extern "C" size_t psa_prefill_workspace_size(int dtype, int32_t T, int32_t Hq, int32_t Hkv,
+                                             int32_t head_dim) {
+  size_t bytes = 256;  // scheduler counter
+  if (dtype == PSA_F32 && T > 0) {
+    auto r = [](size_t x) { return (x + 255) / 256 * 256; };
+    bytes += r(size_t(T) * Hq * head_dim * 2) + 2 * r(size_t(T) * Hkv * head_dim * 2);
+  }
+  return bytes;
+}
+
+extern "C" int psa_prefill_fwd(const void* q, const void* k, const void* v, void* o,
+                               float* lse, int dtype, int32_t T, int32_t Hq, int32_t Hkv,
+                               int32_t head_dim, float scale, const int32_t* dev_schedule,
+                               int64_t sched_len, void* workspace, size_t ws_bytes,
+                               int32_t* dev_status, void* stream) {
+  (void)sched_len;
+  if (dtype != PSA_BF16 && dtype != PSA_F32) return PSA_ERR_INVALID_ARG;
+  if (T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || !(scale > 0.f))
+    return PSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PSA_ERR_UNSUPPORTED;
+  if (T == 0) return PSA_OK;
+  if (!q || !k || !v || !o || !dev_schedule) return PSA_ERR_INVALID_ARG;
+  (void)lse;
+  (void)workspace;
+  (void)ws_bytes;
+  (void)dev_status;
+  (void)stream;
+  return PSA_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ sparse latent
+
+extern "C" int psa_sparse_latent_fwd(const void* q, const void* latent, const int32_t* idx,
+                                     void* o, float* lse, int32_t T, int32_t Tk, int32_t H,
+                                     int32_t dl, int32_t topk, float scale,
+                                     int32_t* dev_status, void* stream) {
+  if (T < 0 || Tk <= 0 || H <= 0 || topk <= 0 || !(scale > 0.f)) return PSA_ERR_INVALID_ARG;
+  if (dl != 512 || H > 128) return PSA_ERR_UNSUPPORTED;
+  if (T == 0) return PSA_OK;
+  if (!q || !latent || !idx || !o) return PSA_ERR_INVALID_ARG;
+  (void)lse;
+  (void)dev_status;
+  (void)stream;
+  return PSA_ERR_UNSUPPORTED;
+}

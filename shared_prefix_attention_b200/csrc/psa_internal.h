@@ -1,0 +1,84 @@
+// Internal launchers shared between the C-ABI layer (psa_api.cpp) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "psa.h"
+
+namespace psa {
+
+// Encodes a tiled TMA descriptor through the driver entry point (no link
+// dependency on libcuda).  rank <= 5; dims/strides innermost first; strides
+// are in bytes for dims 1..rank-1.  Returns PSA_OK or PSA_ERR_CUDA.
+int encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* base,
+                const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                CUtensorMapSwizzle swizzle);
+
+int sm_count(int device);
+
+// ---------------------------------------------------------------- verify
+
+struct VerifyArgs {
+  const void* q;
+  const void* kd;
+  const void* vd;
+  const void* kc;
+  const void* vc;
+  const int32_t* indptr;
+  int64_t n_cache_tokens;
+  void* o;
+  float* lse;
+  int32_t B, Ld, Hq, Hkv, D;
+  float scale;
+  int32_t nsplit;
+  float* part_o;    // [nsplit][B*Ld][Hq][D]
+  float* part_lse;  // [nsplit][B*Ld][Hq], log2 domain
+  int32_t* status;
+  cudaStream_t stream;
+};
+
+// Heads per CTA block and m-tiles per KV head; 0 if the shape is unsupported.
+int verify_plan(int32_t Ld, int32_t Hq, int32_t Hkv, int32_t D, int32_t* heads_per_block,
+                int32_t* mtiles);
+int launch_verify(const VerifyArgs& a);
+
+// ---------------------------------------------------------------- prefill
+
+struct PrefillArgs {
+  const void* q;  // bf16 [T, Hq, D]
+  const void* k;  // bf16 [T, Hkv, D]
+  const void* v;
+  void* o;        // [T, Hq, D], bf16 or fp32 (out_f32)
+  bool out_f32;
+  float* lse;
+  int32_t T, Hq, Hkv, D;
+  float scale;
+  const int32_t* sched;
+  int32_t n_items, n_kv, n_rect;
+  int32_t* counter;  // device scratch for the dynamic tile scheduler
+  int32_t* status;
+  cudaStream_t stream;
+};
+int launch_prefill(const PrefillArgs& a);
+int launch_convert_f32_bf16(const float* src, void* dst, int64_t n, cudaStream_t s);
+
+// ---------------------------------------------------------------- sparse latent
+
+struct SparseArgs {
+  const void* q;       // bf16 [T, H, dl]
+  const void* latent;  // bf16 [Tk, dl]
+  const int32_t* idx;  // [T, topk]
+  void* o;
+  float* lse;
+  int32_t T, Tk, H, dl, topk;
+  float scale;
+  int32_t* status;
+  cudaStream_t stream;
+};
+int launch_sparse_latent(const SparseArgs& a);
+
+}  // namespace psa

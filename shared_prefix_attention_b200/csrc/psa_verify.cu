@@ -1,0 +1,501 @@
+// Speculative-verify attention: split-KV over the cached prefix (stage 1)
+// and a log-sum-exp combine that folds in the causal draft block (stage 2).
+// "Split-KV flash-decode attention for EAGLE target-verify" (sglang PR
+// #27382), implementation breakdown item 1 and motivation (the pre-split
+// verify path reached about 8% of HBM bandwidth at 16k context).
+//
+// Stage 1 is an HBM stream.  A persistent CTA walks work units
+// (request b, split s, block of KV heads); for each unit one producer
+// thread streams 16-token K/V tiles with TMA (128-byte swizzle, no
+// multicast) into a ring of shared-memory stages, and one consumer warp per
+// (KV head, 16-row m-tile) forms S = Q K^T and O += P V with warp MMAs.
+// The 16 rows of an m-tile are all query heads of the KV head's group times
+// all draft tokens, so each shared K/V row is read from HBM once for every
+// query head that uses it (GQA/MQA grouping).  The output of a unit is the
+// normalised partial O and its log2-domain LSE in the workspace.
+//
+// Stage 2 has one warp per (draft row, query head): it scores the draft
+// keys 0..j, then merges them with every split by LSE weights.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "psa_device.cuh"
+#include "psa_internal.h"
+
+namespace psa {
+namespace {
+
+constexpr int kTileKeys = 16;      // keys per pipeline stage
+// Consumer warps per CTA: with the producer warp, 9 warps leave each warp
+// 168 registers; head_dim 256 needs more, so it runs 4 consumer warps.
+__host__ __device__ constexpr int max_consumer_warps(int D) { return D > 128 ? 4 : 8; }
+
+struct Stage1Params {
+  const __nv_bfloat16* q;  // [B*Ld, Hq, D]
+  const int32_t* indptr;   // [B+1]
+  float* part_o;
+  float* part_lse;
+  int32_t B, Ld, Hq, Hkv, G, R, MT, HB, nhb, nsplit;
+  float scale_log2;
+  int32_t* status;
+  int32_t nstage;
+};
+
+__device__ __forceinline__ void split_range(const Stage1Params& p, int b, int s, int32_t& t0,
+                                            int32_t& t1) {
+  const int32_t a = __ldg(p.indptr + b), e = __ldg(p.indptr + b + 1);
+  const int32_t L = e - a;
+  int32_t c = (L + p.nsplit - 1) / p.nsplit;
+  c = (c + kTileKeys - 1) / kTileKeys * kTileKeys;
+  t0 = a + min(L, s * c);
+  t1 = a + min(L, (s + 1) * c);
+}
+
+template <int D>
+__global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
+    verify_stage1_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                         const __grid_constant__ CUtensorMap tmap_v, Stage1Params p) {
+  constexpr int KSTEPS = D / 16;  // MMA k-steps over the head dimension
+  constexpr int NPART = D / 64;   // 128-byte swizzle atoms across the head dimension
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ int abort_flag;
+
+  const int NW = p.HB * p.MT;
+  const uint32_t head_bytes = kTileKeys * 128;                // one head, one part
+  const uint32_t kv_bytes = uint32_t(NPART) * p.HB * head_bytes;  // K (or V) per stage
+  const uint32_t stage_bytes = 2 * kv_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.nstage * stage_bytes);
+  uint64_t* empty = full + p.nstage;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < p.nstage; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], NW);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int units = p.B * p.nsplit * p.nhb;
+
+  if (warp == NW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int last_phase[8];
+      for (int i = 0; i < 8; ++i) last_phase[i] = -1;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int hb = u % p.nhb;
+        const int bs = u / p.nhb;
+        const int b = bs / p.nsplit, s = bs % p.nsplit;
+        int32_t t0, t1;
+        split_range(p, b, s, t0, t1);
+        for (int32_t t = t0; t < t1; t += kTileKeys) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, &abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], stage_bytes);
+          last_phase[stage] = int(phase);
+          uint8_t* kdst = smem + stage * stage_bytes;
+          uint8_t* vdst = kdst + kv_bytes;
+#pragma unroll
+          for (int part = 0; part < NPART; ++part) {
+            tma_load_3d(kdst + part * p.HB * head_bytes, &tmap_k, &full[stage], part * 64, t,
+                        hb * p.HB);
+            tma_load_3d(vdst + part * p.HB * head_bytes, &tmap_v, &full[stage], part * 64, t,
+                        hb * p.HB);
+          }
+          if (++stage == p.nstage) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let copies already in flight land before the CTA exits.
+        for (int i = 0; i < p.nstage; ++i) {
+          if (last_phase[i] < 0) continue;
+          const uint64_t w0 = globaltimer();
+          while (!mbar_try_wait(&full[i], uint32_t(last_phase[i])) &&
+                 globaltimer() - w0 < kWaitTimeoutNs) {
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int hh = warp / p.MT;  // KV head within the block
+  const int mt = warp % p.MT;  // 16-row m-tile of that head's rows
+  const int g = lane >> 2, c = lane & 3;
+  const int BL = p.B * p.Ld;
+  int stage = 0;
+  uint32_t phase = 0;
+
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int hb = u % p.nhb;
+    const int bs = u / p.nhb;
+    const int b = bs / p.nsplit, s = bs % p.nsplit;
+    const int kvh = hb * p.HB + hh;
+    int32_t t0, t1;
+    split_range(p, b, s, t0, t1);
+
+    // rows of this thread: g and g + 8 of the m-tile
+    int rrow[2], rqh[2];
+    bool rvalid[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int rr = mt * 16 + g + 8 * i;
+      rvalid[i] = rr < p.R;
+      const int j = rvalid[i] ? rr / p.G : 0;
+      rqh[i] = kvh * p.G + (rvalid[i] ? rr % p.G : 0);
+      rrow[i] = b * p.Ld + j;
+    }
+
+    // Q fragments for every k-step (A operand, row-major 16x16 per step)
+    uint32_t qa[KSTEPS][4];
+    {
+      const __nv_bfloat16* q0 = p.q + (size_t(rrow[0]) * p.Hq + rqh[0]) * D;
+      const __nv_bfloat16* q1 = p.q + (size_t(rrow[1]) * p.Hq + rqh[1]) * D;
+#pragma unroll
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        const int col = ks * 16 + 2 * c;
+        qa[ks][0] = rvalid[0] ? __ldg(reinterpret_cast<const uint32_t*>(q0 + col)) : 0u;
+        qa[ks][1] = rvalid[1] ? __ldg(reinterpret_cast<const uint32_t*>(q1 + col)) : 0u;
+        qa[ks][2] = rvalid[0] ? __ldg(reinterpret_cast<const uint32_t*>(q0 + col + 8)) : 0u;
+        qa[ks][3] = rvalid[1] ? __ldg(reinterpret_cast<const uint32_t*>(q1 + col + 8)) : 0u;
+      }
+    }
+
+    float acc[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    bool ok = true;
+
+    for (int32_t t = t0; t < t1; t += kTileKeys) {
+      if (!mbar_wait(&full[stage], phase, &abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      const uint32_t kbase = smem_u32(smem + stage * stage_bytes) + hh * head_bytes;
+      const uint32_t vbase = kbase + kv_bytes;
+
+      // S = Q K^T over 16 keys: two n-tiles of 8 keys
+      float sc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+        const uint32_t key = nt * 8 + (lane & 7);
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ks += 2) {
+          const uint32_t chunk = ks * 2 + (lane >> 3);  // 16-byte chunk of the head dim
+          const uint32_t addr =
+              kbase + (chunk >> 3) * (p.HB * head_bytes) + sw128(key, chunk & 7);
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4(addr, b0, b1, b2, b3);
+          mma_bf16_16816(sc[nt], qa[ks], b0, b1);
+          mma_bf16_16816(sc[nt], qa[ks + 1], b2, b3);
+        }
+      }
+
+      // online softmax in the log2 domain; keys past the split end are masked
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int32_t key = t + nt * 8 + 2 * c + (e & 1);
+          float v = sc[nt][e] * p.scale_log2;
+          v = key < t1 ? v : -INFINITY;
+          sc[nt][e] = v;
+          mx[e >> 1] = fmaxf(mx[e >> 1], v);
+        }
+      float alpha[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
+        const float mn = fmaxf(m_run[i], mx[i]);
+        alpha[i] = fast_exp2(m_run[i] - mn);
+        m_run[i] = mn;
+      }
+      float ps[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ps[nt][e] = fast_exp2(sc[nt][e] - m_run[e >> 1]);
+      l_run[0] = l_run[0] * alpha[0] + ps[0][0] + ps[0][1] + ps[1][0] + ps[1][1];
+      l_run[1] = l_run[1] * alpha[1] + ps[0][2] + ps[0][3] + ps[1][2] + ps[1][3];
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        acc[i][0] *= alpha[0];
+        acc[i][1] *= alpha[0];
+        acc[i][2] *= alpha[1];
+        acc[i][3] *= alpha[1];
+      }
+
+      // O += P V: P as the A operand (16 rows x 16 keys), V^T via ldmatrix.trans
+      uint32_t pa[4];
+      pa[0] = pack_bf16(ps[0][0], ps[0][1]);
+      pa[1] = pack_bf16(ps[0][2], ps[0][3]);
+      pa[2] = pack_bf16(ps[1][0], ps[1][1]);
+      pa[3] = pack_bf16(ps[1][2], ps[1][3]);
+      {
+        const int mi = lane >> 3;
+        const uint32_t key = (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int dt = 0; dt < D / 8; dt += 2) {
+          const uint32_t chunk = dt + (mi >> 1);
+          const uint32_t addr =
+              vbase + (chunk >> 3) * (p.HB * head_bytes) + sw128(key, chunk & 7);
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4_trans(addr, b0, b1, b2, b3);
+          mma_bf16_16816(acc[dt], pa, b0, b1);
+          mma_bf16_16816(acc[dt + 1], pa, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (++stage == p.nstage) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    if (!ok) return;
+
+    // normalise and write this split's partial
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 1);
+      l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 2);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (!rvalid[i]) continue;
+      const float inv = l_run[i] > 0.f ? 1.f / l_run[i] : 0.f;
+      const size_t prow = (size_t(s) * BL + rrow[i]) * p.Hq + rqh[i];
+      float* dst = p.part_o + prow * D;
+#pragma unroll
+      for (int dt = 0; dt < D / 8; ++dt) {
+        float2 v = make_float2(acc[dt][2 * i] * inv, acc[dt][2 * i + 1] * inv);
+        *reinterpret_cast<float2*>(dst + dt * 8 + 2 * c) = v;
+      }
+      if (c == 0)
+        p.part_lse[prow] = l_run[i] > 0.f ? m_run[i] + __log2f(l_run[i]) : -INFINITY;
+    }
+  }
+}
+
+struct Stage2Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* kd;
+  const __nv_bfloat16* vd;
+  const float* part_o;
+  const float* part_lse;
+  __nv_bfloat16* o;
+  float* lse;
+  int32_t B, Ld, Hq, Hkv, G, nsplit;
+  float scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
+  constexpr int E = D / 32;  // head-dim elements per lane
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int BL = p.B * p.Ld;
+  if (gw >= BL * p.Hq) return;
+  const int row = gw / p.Hq, qh = gw % p.Hq;
+  const int b = row / p.Ld, j = row % p.Ld;
+  const int kvh = qh / p.G;
+
+  float qv[E];
+  {
+    const __nv_bfloat16* qp = p.q + (size_t(row) * p.Hq + qh) * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) qv[e] = __bfloat162float(qp[e]);
+  }
+
+  // draft keys 0..j (the causal draft-draft block), log2-domain logits
+  auto draft_logit = [&](int i) {
+    const __nv_bfloat16* kp = p.kd + (size_t(b * p.Ld + i) * p.Hkv + kvh) * D + lane * E;
+    float sdot = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) sdot += qv[e] * __bfloat162float(kp[e]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, off);
+    return sdot * p.scale_log2;
+  };
+  float M = -INFINITY;
+  const int nd = j + 1;
+  for (int i = 0; i < nd; ++i) M = fmaxf(M, draft_logit(i));
+  for (int s = lane; s < p.nsplit; s += 32)
+    M = fmaxf(M, p.part_lse[(size_t(s) * BL + row) * p.Hq + qh]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < p.nsplit; ++s) {
+    const size_t prow = (size_t(s) * BL + row) * p.Hq + qh;
+    const float ls = p.part_lse[prow];
+    const float w = fast_exp2(ls - M);  // empty split: exp2(-inf) = 0
+    if (w == 0.f) continue;
+    const float* op = p.part_o + prow * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; e += 2) {
+      const float2 v = *reinterpret_cast<const float2*>(op + e);
+      acc[e] += w * v.x;
+      acc[e + 1] += w * v.y;
+    }
+    wsum += w;
+  }
+  for (int i = 0; i < nd; ++i) {
+    const float w = fast_exp2(draft_logit(i) - M);
+    const __nv_bfloat16* vp = p.vd + (size_t(b * p.Ld + i) * p.Hkv + kvh) * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] += w * __bfloat162float(vp[e]);
+    wsum += w;
+  }
+  const float inv = 1.f / wsum;
+  __nv_bfloat16* op = p.o + (size_t(row) * p.Hq + qh) * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; e += 2)
+    *reinterpret_cast<__nv_bfloat162*>(op + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+  if (p.lse && lane == 0) p.lse[size_t(row) * p.Hq + qh] = (M + __log2f(wsum)) * kLn2;
+}
+
+template <int D>
+int launch_verify_d(const VerifyArgs& a, int HB, int MT) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PSA_ERR_CUDA;
+  const int G = a.Hq / a.Hkv;
+  const int R = a.Ld * G;
+  const int nhb = a.Hkv / HB;
+
+  CUtensorMap tk, tv;
+  const uint64_t dims[3] = {uint64_t(D), uint64_t(a.n_cache_tokens), uint64_t(a.Hkv)};
+  const uint64_t strides[2] = {uint64_t(a.Hkv) * D * 2, uint64_t(D) * 2};
+  const uint32_t box[3] = {64u, uint32_t(kTileKeys), uint32_t(HB)};
+  int rc = encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.kc, dims, strides, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != PSA_OK) return rc;
+  rc = encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.vc, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != PSA_OK) return rc;
+
+  Stage1Params p1;
+  p1.q = static_cast<const __nv_bfloat16*>(a.q);
+  p1.indptr = a.indptr;
+  p1.part_o = a.part_o;
+  p1.part_lse = a.part_lse;
+  p1.B = a.B;
+  p1.Ld = a.Ld;
+  p1.Hq = a.Hq;
+  p1.Hkv = a.Hkv;
+  p1.G = G;
+  p1.R = R;
+  p1.MT = MT;
+  p1.HB = HB;
+  p1.nhb = nhb;
+  p1.nsplit = a.nsplit;
+  p1.scale_log2 = a.scale * kLog2e;
+  p1.status = a.status;
+
+  const size_t stage_bytes = size_t(2) * (D / 64) * HB * kTileKeys * 128;
+  const size_t budget = 200 * 1024;
+  int nstage = int(budget / stage_bytes);
+  nstage = nstage > 8 ? 8 : nstage;
+  if (nstage < 2) return PSA_ERR_UNSUPPORTED;
+  p1.nstage = nstage;
+  const size_t smem = 1024 + nstage * stage_bytes + 2 * nstage * sizeof(uint64_t);
+  auto k1 = verify_stage1_kernel<D>;
+  if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+      cudaSuccess)
+    return PSA_ERR_CUDA;
+  const int units = a.B * a.nsplit * nhb;
+  int grid = sm_count(dev);
+  if (grid <= 0) return PSA_ERR_CUDA;
+  grid = units < grid ? units : grid;
+  const int threads = (HB * MT + 1) * 32;
+  if (units > 0) {
+    k1<<<grid, threads, smem, a.stream>>>(tk, tv, p1);
+    if (cudaGetLastError() != cudaSuccess) return PSA_ERR_CUDA;
+  }
+
+  Stage2Params p2;
+  p2.q = static_cast<const __nv_bfloat16*>(a.q);
+  p2.kd = static_cast<const __nv_bfloat16*>(a.kd);
+  p2.vd = static_cast<const __nv_bfloat16*>(a.vd);
+  p2.part_o = a.part_o;
+  p2.part_lse = a.part_lse;
+  p2.o = static_cast<__nv_bfloat16*>(a.o);
+  p2.lse = a.lse;
+  p2.B = a.B;
+  p2.Ld = a.Ld;
+  p2.Hq = a.Hq;
+  p2.Hkv = a.Hkv;
+  p2.G = G;
+  p2.nsplit = a.nsplit;
+  p2.scale_log2 = a.scale * kLog2e;
+  const int warps = a.B * a.Ld * a.Hq;
+  const int blocks = (warps + 7) / 8;
+  if (blocks > 0) {
+    verify_stage2_kernel<D><<<blocks, 256, 0, a.stream>>>(p2);
+    if (cudaGetLastError() != cudaSuccess) return PSA_ERR_CUDA;
+  }
+  return PSA_OK;
+}
+
+}  // namespace
+
+int verify_plan(int32_t Ld, int32_t Hq, int32_t Hkv, int32_t D, int32_t* heads_per_block,
+                int32_t* mtiles) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || Ld <= 0 || Ld > 16) return 0;
+  const int R = Ld * (Hq / Hkv);
+  if (R > 128) return 0;
+  const int MT = (R + 15) / 16;
+  // largest divisor of Hkv that fits the warp budget and a <= 64 KB stage
+  int best = 0;
+  for (int hb = 1; hb <= Hkv; ++hb) {
+    if (Hkv % hb) continue;
+    if (hb * MT > max_consumer_warps(D)) continue;
+    if (size_t(2) * (D / 64) * hb * kTileKeys * 128 > 64 * 1024) continue;
+    best = hb;
+  }
+  if (!best) return 0;
+  *heads_per_block = best;
+  *mtiles = MT;
+  return 1;
+}
+
+int launch_verify(const VerifyArgs& a) {
+  int HB = 0, MT = 0;
+  if (!verify_plan(a.Ld, a.Hq, a.Hkv, a.D, &HB, &MT)) return PSA_ERR_UNSUPPORTED;
+  switch (a.D) {
+    case 64:
+      return launch_verify_d<64>(a, HB, MT);
+    case 128:
+      return launch_verify_d<128>(a, HB, MT);
+    case 256:
+      return launch_verify_d<256>(a, HB, MT);
+    default:
+      return PSA_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace psa

@@ -1,0 +1,115 @@
+"""The C-ABI library loads and exports every symbol include/psa.h declares;
+host-side validation returns the documented statuses before any GPU work.
+No call here launches a kernel, so these run without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import shared_prefix_attention_b200 as psa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "psa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(psa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = psa.lib()
+    declared = _declared_symbols()
+    assert declared, "no declarations parsed"
+    assert set(declared) == set(psa.EXPORTS)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings():
+    assert psa.lib().psa_version() == 1
+    for code in range(7):
+        assert psa.status_string(code)
+    assert "unsupported" in psa.status_string(psa.PSA_ERR_UNSUPPORTED)
+
+
+def _verify_call(**kw):
+    """psa_verify_fwd with dummy (never dereferenced) pointers: every case
+    below is refused on the host before any CUDA call."""
+    args = dict(q=16, kd=16, vd=16, kc=16, vc=16, ntok=64, indptr=16, maxlen=64, kvi=None,
+                o=16, lse=None, B=1, Ld=4, Hq=8, Hkv=2, d=128, scale=0.1, nsplit=1,
+                feat=None, ws=None, wsb=0)
+    args.update(kw)
+    a = args
+    P = ctypes.c_void_p
+    return psa.lib().psa_verify_fwd(
+        P(a["q"]), P(a["kd"]), P(a["vd"]), P(a["kc"]), P(a["vc"]), a["ntok"], P(a["indptr"]),
+        a["maxlen"], P(a["kvi"]) if a["kvi"] else None, P(a["o"]), None, a["B"], a["Ld"],
+        a["Hq"], a["Hkv"], a["d"], a["scale"], a["nsplit"],
+        ctypes.byref(a["feat"]) if a["feat"] is not None else None,
+        P(a["ws"]) if a["ws"] else None, a["wsb"], None, None)
+
+
+@pytest.mark.parametrize("field,value", [
+    ("has_custom_mask", 1), ("is_causal", 0), ("sliding_window", 128), ("has_sinks", 1),
+    ("logit_cap", 30.0), ("xai_temperature_len", 5), ("ragged_extend", 1)])
+def test_verify_gating_refuses_unsupported_features(field, value):
+    """Split-KV verify gating ("can_handle" in the split-KV verify PR's key
+    code): each unsupported feature is refused with PSA_ERR_UNSUPPORTED."""
+    f = psa.VerifyFeatures(0, 1, -1, 0, 0.0, -1, 0)
+    setattr(f, field, value)
+    assert _verify_call(feat=f) == psa.PSA_ERR_UNSUPPORTED
+
+
+def test_verify_host_validation():
+    assert _verify_call(kvi=16) == psa.PSA_ERR_UNSUPPORTED          # paged cache
+    assert _verify_call(d=96) == psa.PSA_ERR_UNSUPPORTED             # head dim
+    assert _verify_call(Hq=6, Hkv=4) == psa.PSA_ERR_INVALID_ARG      # Hq % Hkv
+    assert _verify_call(scale=0.0) == psa.PSA_ERR_INVALID_ARG
+    assert _verify_call(q=8) == psa.PSA_ERR_INVALID_ARG              # misaligned
+    assert _verify_call(Ld=17) == psa.PSA_ERR_UNSUPPORTED            # draft block too big
+    assert _verify_call(nsplit=257) == psa.PSA_ERR_INVALID_ARG
+    assert _verify_call(ws=None) == psa.PSA_ERR_WORKSPACE
+    need = psa.verify_workspace_size(1, 4, 8, 128, 1)
+    assert _verify_call(ws=256, wsb=need - 1) == psa.PSA_ERR_WORKSPACE
+    assert _verify_call(ws=8, wsb=need) == psa.PSA_ERR_WORKSPACE     # alignment
+    assert _verify_call(B=0) == psa.PSA_OK                           # nothing to do
+
+
+def test_verify_workspace_size_formula():
+    B, Ld, Hq, d, ns = 32, 4, 32, 128, 32
+    rows = ns * B * Ld * Hq
+    assert psa.verify_workspace_size(B, Ld, Hq, d, ns) >= rows * (d + 1) * 4
+    assert psa.verify_workspace_size(0, Ld, Hq, d, ns) == 0
+
+
+def test_auto_splits_bounds():
+    assert 1 <= psa.verify_auto_splits(32, 16384, 8, 128) <= 256
+    assert psa.verify_auto_splits(1, 100, 8, 128) == 1
+    assert psa.verify_auto_splits(1, 1 << 20, 8, 128) <= 256
+
+
+def test_prefill_and_sparse_host_validation():
+    L = psa.lib()
+    P = ctypes.c_void_p
+    assert L.psa_prefill_fwd(P(16), P(16), P(16), P(16), None, 0, 10, 4, 3, 128, 0.1, P(16), 8,
+                             None, 0, None, None) == psa.PSA_ERR_INVALID_ARG
+    assert L.psa_prefill_fwd(P(16), P(16), P(16), P(16), None, 0, 10, 4, 2, 96, 0.1, P(16), 8,
+                             None, 0, None, None) == psa.PSA_ERR_UNSUPPORTED
+    assert L.psa_prefill_fwd(P(16), P(16), P(16), P(16), None, 7, 10, 4, 2, 128, 0.1, P(16), 8,
+                             None, 0, None, None) == psa.PSA_ERR_INVALID_ARG
+    assert L.psa_sparse_latent_fwd(P(16), P(16), P(16), P(16), None, 4, 8, 64, 256, 16, 0.1,
+                                   None, None) == psa.PSA_ERR_UNSUPPORTED
+    assert L.psa_sparse_latent_fwd(P(16), P(16), P(16), P(16), None, 4, 8, 64, 512, 0, 0.1,
+                                   None, None) == psa.PSA_ERR_INVALID_ARG
+    assert psa.prefill_tiles(128) == (128, 128)
+    with pytest.raises(psa.PsaError):
+        psa.prefill_tiles(80)
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        psa.sparse_latent(x, x[:, 0], torch.zeros(4, 1, dtype=torch.int32), 0.1)
