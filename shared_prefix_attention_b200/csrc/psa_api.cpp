@@ -160,8 +160,8 @@ extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const vo
       !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return PSA_ERR_INVALID_ARG;
-  int32_t HB = 0, MT = 0;
-  if (!verify_plan(Ld, Hq, Hkv, head_dim, &HB, &MT)) return PSA_ERR_UNSUPPORTED;
+  int32_t HB = 0, MT = 0, NRB = 0;
+  if (!verify_plan(Ld, Hq, Hkv, head_dim, &HB, &MT, &NRB)) return PSA_ERR_UNSUPPORTED;
   if (nsplit == 0) nsplit = psa_verify_auto_splits(B, max_prefix_len, Hkv, head_dim);
   if (nsplit < 1 || nsplit > 256) return PSA_ERR_INVALID_ARG;
   const size_t need = psa_verify_workspace_size(B, Ld, Hq, head_dim, nsplit);

@@ -41,9 +41,10 @@ struct VerifyArgs {
   cudaStream_t stream;
 };
 
-// Heads per CTA block and m-tiles per KV head; 0 if the shape is unsupported.
+// KV heads per CTA, 16-row m-tiles per CTA and row blocks per KV head;
+// returns 0 if the shape is unsupported.
 int verify_plan(int32_t Ld, int32_t Hq, int32_t Hkv, int32_t D, int32_t* heads_per_block,
-                int32_t* mtiles);
+                int32_t* mtiles, int32_t* row_blocks);
 int launch_verify(const VerifyArgs& a);
 
 // ---------------------------------------------------------------- prefill

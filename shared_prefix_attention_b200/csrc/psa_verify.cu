@@ -35,11 +35,30 @@ struct Stage1Params {
   const int32_t* indptr;   // [B+1]
   float* part_o;
   float* part_lse;
-  int32_t B, Ld, Hq, Hkv, G, R, MT, HB, nhb, nsplit;
+  int32_t B, Ld, Hq, Hkv, G, R;
+  int32_t MT;   // m-tiles per CTA for each KV head
+  int32_t nrb;  // row blocks: a head's m-tiles are split over nrb CTAs
+  int32_t HB, nhb, nsplit;
   float scale_log2;
   int32_t* status;
   int32_t nstage;
 };
+
+struct Unit {
+  int b, s, rb, hb;
+};
+
+// Work units are ordered so that consecutive units stream adjacent memory.
+__device__ __forceinline__ Unit decode_unit(const Stage1Params& p, int u) {
+  Unit x;
+  x.hb = u % p.nhb;
+  u /= p.nhb;
+  x.rb = u % p.nrb;
+  u /= p.nrb;
+  x.s = u % p.nsplit;
+  x.b = u / p.nsplit;
+  return x;
+}
 
 __device__ __forceinline__ void split_range(const Stage1Params& p, int b, int s, int32_t& t0,
                                             int32_t& t1) {
@@ -80,7 +99,7 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
   }
   __syncthreads();
 
-  const int units = p.B * p.nsplit * p.nhb;
+  const int units = p.B * p.nsplit * p.nrb * p.nhb;
 
   if (warp == NW) {
     // ------------------------------------------------------------ producer
@@ -93,11 +112,10 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
       int last_phase[8];
       for (int i = 0; i < 8; ++i) last_phase[i] = -1;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const int hb = u % p.nhb;
-        const int bs = u / p.nhb;
-        const int b = bs / p.nsplit, s = bs % p.nsplit;
+        const Unit x = decode_unit(p, u);
+        const int hb = x.hb;
         int32_t t0, t1;
-        split_range(p, b, s, t0, t1);
+        split_range(p, x.b, x.s, t0, t1);
         for (int32_t t = t0; t < t1; t += kTileKeys) {
           if (!mbar_wait(&empty[stage], phase ^ 1, &abort_flag, p.status)) {
             ok = false;
@@ -143,10 +161,9 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
   uint32_t phase = 0;
 
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const int hb = u % p.nhb;
-    const int bs = u / p.nhb;
-    const int b = bs / p.nsplit, s = bs % p.nsplit;
-    const int kvh = hb * p.HB + hh;
+    const Unit x = decode_unit(p, u);
+    const int b = x.b, s = x.s;
+    const int kvh = x.hb * p.HB + hh;
     int32_t t0, t1;
     split_range(p, b, s, t0, t1);
 
@@ -155,7 +172,7 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
     bool rvalid[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const int rr = mt * 16 + g + 8 * i;
+      const int rr = (x.rb * p.MT + mt) * 16 + g + 8 * i;
       rvalid[i] = rr < p.R;
       const int j = rvalid[i] ? rr / p.G : 0;
       rqh[i] = kvh * p.G + (rvalid[i] ? rr % p.G : 0);
@@ -380,7 +397,7 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
 }
 
 template <int D>
-int launch_verify_d(const VerifyArgs& a, int HB, int MT) {
+int launch_verify_d(const VerifyArgs& a, int HB, int MT, int NRB) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PSA_ERR_CUDA;
   const int G = a.Hq / a.Hkv;
@@ -410,6 +427,7 @@ int launch_verify_d(const VerifyArgs& a, int HB, int MT) {
   p1.G = G;
   p1.R = R;
   p1.MT = MT;
+  p1.nrb = NRB;
   p1.HB = HB;
   p1.nhb = nhb;
   p1.nsplit = a.nsplit;
@@ -427,7 +445,7 @@ int launch_verify_d(const VerifyArgs& a, int HB, int MT) {
   if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
     return PSA_ERR_CUDA;
-  const int units = a.B * a.nsplit * nhb;
+  const int units = a.B * a.nsplit * NRB * nhb;
   int grid = sm_count(dev);
   if (grid <= 0) return PSA_ERR_CUDA;
   grid = units < grid ? units : grid;
@@ -464,35 +482,45 @@ int launch_verify_d(const VerifyArgs& a, int HB, int MT) {
 }  // namespace
 
 int verify_plan(int32_t Ld, int32_t Hq, int32_t Hkv, int32_t D, int32_t* heads_per_block,
-                int32_t* mtiles) {
+                int32_t* mtiles, int32_t* row_blocks) {
   if (Hkv <= 0 || Hq % Hkv != 0 || Ld <= 0 || Ld > 16) return 0;
+  if (D != 64 && D != 128 && D != 256) return 0;
   const int R = Ld * (Hq / Hkv);
   if (R > 128) return 0;
   const int MT = (R + 15) / 16;
+  const int maxw = max_consumer_warps(D);
+  if (MT > maxw) {
+    // one KV head per CTA; its m-tiles are spread over several CTAs
+    *heads_per_block = 1;
+    *mtiles = maxw;
+    *row_blocks = (MT + maxw - 1) / maxw;
+    return 1;
+  }
   // largest divisor of Hkv that fits the warp budget and a <= 64 KB stage
   int best = 0;
   for (int hb = 1; hb <= Hkv; ++hb) {
     if (Hkv % hb) continue;
-    if (hb * MT > max_consumer_warps(D)) continue;
+    if (hb * MT > maxw) continue;
     if (size_t(2) * (D / 64) * hb * kTileKeys * 128 > 64 * 1024) continue;
     best = hb;
   }
   if (!best) return 0;
   *heads_per_block = best;
   *mtiles = MT;
+  *row_blocks = 1;
   return 1;
 }
 
 int launch_verify(const VerifyArgs& a) {
-  int HB = 0, MT = 0;
-  if (!verify_plan(a.Ld, a.Hq, a.Hkv, a.D, &HB, &MT)) return PSA_ERR_UNSUPPORTED;
+  int HB = 0, MT = 0, NRB = 0;
+  if (!verify_plan(a.Ld, a.Hq, a.Hkv, a.D, &HB, &MT, &NRB)) return PSA_ERR_UNSUPPORTED;
   switch (a.D) {
     case 64:
-      return launch_verify_d<64>(a, HB, MT);
+      return launch_verify_d<64>(a, HB, MT, NRB);
     case 128:
-      return launch_verify_d<128>(a, HB, MT);
+      return launch_verify_d<128>(a, HB, MT, NRB);
     case 256:
-      return launch_verify_d<256>(a, HB, MT);
+      return launch_verify_d<256>(a, HB, MT, NRB);
     default:
       return PSA_ERR_UNSUPPORTED;
   }
