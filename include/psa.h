@@ -203,6 +203,45 @@ int psa_verify_fwd(const void *q_draft, const void *k_draft, const void *v_draft
                    float scale, int32_t nsplit, const psa_verify_features *features,
                    void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/* Size of the library's fixed device scratch used by psa_verify_fwd_noalloc:
+ * 16 MiB, held by every GPU that loads the library until the process exits. */
+#define PSA_VERIFY_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * psa_verify_fwd without a caller workspace.  The pages have no counterpart
+ * of this call; it exists for callers that cannot allocate device memory
+ * where they call attention -- for example a host whose device memory is
+ * owned by another allocator (a framework's caching allocator or a serving
+ * engine's preallocated pool) that must not see cudaMalloc behind its back,
+ * or a latency-critical loop where cudaMalloc's implicit device-wide
+ * synchronisation, or its failure under memory pressure, is unacceptable.
+ *
+ * The split partials go to one file-scope device array of
+ * PSA_VERIFY_NOALLOC_SCRATCH_BYTES instead of a workspace.  Arguments,
+ * layouts and results are those of psa_verify_fwd (minus workspace and
+ * ws_bytes); the caller still owns every input and output.
+ *   - Returns PSA_ERR_WORKSPACE when the call would need more than
+ *     PSA_VERIFY_NOALLOC_SCRATCH_BYTES, that is when
+ *     psa_verify_workspace_size(B, Ld, Hq, head_dim, nsplit) exceeds it
+ *     (nsplit == 0 is resolved with psa_verify_auto_splits first).
+ *   - Allocates and frees nothing, directly or through any library.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture on the device.
+ *   - Every call on a device shares the one array, which keeps whatever the
+ *     last call left there.  Nothing in it needs to start at zero (stage 1
+ *     writes every partial that stage 2 reads).  Calls whose GPU work
+ *     overlaps -- on different streams, or from different host threads --
+ *     race on the array and corrupt each other's results; order them.
+ */
+int psa_verify_fwd_noalloc(const void *q_draft, const void *k_draft, const void *v_draft,
+                           const void *k_cache, const void *v_cache, int64_t n_cache_tokens,
+                           const int32_t *dev_kv_indptr, int64_t max_prefix_len,
+                           const int32_t *kv_indices, void *o, float *lse, int32_t B,
+                           int32_t Ld, int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
+                           int32_t nsplit, const psa_verify_features *features,
+                           int32_t *dev_status, void *stream);
+
 /* ------------------------------------------------------------------------
  * Shared-latent sparse attention                     [MLA] environment,
  * analysis (head-blocked tiles; the latent is shared by every head)

@@ -30,7 +30,7 @@ EXPORTS = [
     "psa_version", "psa_status_string", "psa_spec_flat", "psa_build_spec",
     "psa_build_schedule", "psa_prefill_tiles", "psa_prefill_workspace_size",
     "psa_prefill_fwd", "psa_verify_auto_splits", "psa_verify_workspace_size",
-    "psa_verify_fwd", "psa_sparse_latent_fwd", "psa_read_status",
+    "psa_verify_fwd", "psa_verify_fwd_noalloc", "psa_sparse_latent_fwd", "psa_read_status",
 ]
 
 
@@ -84,6 +84,8 @@ def lib():
         "psa_verify_workspace_size": ([I32, I32, I32, I32, I32], SZ),
         "psa_verify_fwd": ([P, P, P, P, P, I64, P, I64, P, P, P, I32, I32, I32, I32, I32, F, I32,
                             P, P, SZ, P, P], ctypes.c_int),
+        "psa_verify_fwd_noalloc": ([P, P, P, P, P, I64, P, I64, P, P, P, I32, I32, I32, I32, I32,
+                                    F, I32, P, P, P], ctypes.c_int),
         "psa_sparse_latent_fwd": ([P, P, P, P, P, I32, I32, I32, I32, I32, F, P, P],
                                   ctypes.c_int),
         "psa_read_status": ([P, P, P], ctypes.c_int),
@@ -233,6 +235,28 @@ def verify(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr: torch.Tensor,
                               _ptr(workspace), workspace.numel(), _ptr(status),
                               _stream(q_draft.device))
     _check(rc, "psa_verify_fwd")
+    return out, lse
+
+
+def verify_noalloc(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr: torch.Tensor,
+                   max_prefix_len: int, scale: float, Ld: int, nsplit: int = 0, out=None,
+                   lse=None, status=None):
+    """Split-KV verify through psa_verify_fwd_noalloc: the library's fixed
+    device scratch replaces the workspace (for callers that cannot allocate
+    device memory at the call site).  Outputs are allocated here only for
+    convenience; pass ``out`` / ``lse`` to avoid that too."""
+    _require_cuda(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr)
+    BL, Hq, d = q_draft.shape
+    Hkv = k_cache.shape[1]
+    B = BL // Ld
+    out = torch.empty_like(q_draft) if out is None else out
+    lse = torch.empty((BL, Hq), dtype=torch.float32, device=q_draft.device) if lse is None else lse
+    rc = lib().psa_verify_fwd_noalloc(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft),
+                                      _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
+                                      _ptr(kv_indptr), int(max_prefix_len), None, _ptr(out),
+                                      _ptr(lse), B, Ld, Hq, Hkv, d, float(scale), nsplit, None,
+                                      _ptr(status), _stream(q_draft.device))
+    _check(rc, "psa_verify_fwd_noalloc")
     return out, lse
 
 

@@ -19,6 +19,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "psa_device.cuh"
 #include "psa_internal.h"
 
@@ -527,3 +529,56 @@ int launch_verify(const VerifyArgs& a) {
 }
 
 }  // namespace psa
+
+// ---------------------------------------------------------------------------
+// Verify without a caller workspace: the partials live in a fixed file-scope
+// device array.  Host code cannot use the array's name as a device address,
+// so the address is looked up once per device with that device current.
+
+namespace psa {
+namespace {
+
+static __device__ __align__(256) uint8_t g_verify_scratch[PSA_VERIFY_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+
+int scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_verify_scratch) != cudaSuccess || !p) return PSA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return PSA_OK;
+}
+
+}  // namespace
+}  // namespace psa
+
+extern "C" int psa_verify_fwd_noalloc(const void* q_draft, const void* k_draft,
+                                      const void* v_draft, const void* k_cache,
+                                      const void* v_cache, int64_t n_cache_tokens,
+                                      const int32_t* dev_kv_indptr, int64_t max_prefix_len,
+                                      const int32_t* kv_indices, void* o, float* lse, int32_t B,
+                                      int32_t Ld, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                                      float scale, int32_t nsplit,
+                                      const psa_verify_features* features, int32_t* dev_status,
+                                      void* stream) {
+  int32_t ns = nsplit;
+  if (ns == 0 && B > 0) ns = psa_verify_auto_splits(B, max_prefix_len, Hkv, head_dim);
+  if (B > 0 && ns >= 1 && ns <= 256 &&
+      psa_verify_workspace_size(B, Ld, Hq, head_dim, ns) > PSA_VERIFY_NOALLOC_SCRATCH_BYTES)
+    return PSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const int rc = psa::scratch_address(&scratch);
+  if (rc != PSA_OK) return rc;
+  return psa_verify_fwd(q_draft, k_draft, v_draft, k_cache, v_cache, n_cache_tokens,
+                        dev_kv_indptr, max_prefix_len, kv_indices, o, lse, B, Ld, Hq, Hkv,
+                        head_dim, scale, ns, features, scratch, PSA_VERIFY_NOALLOC_SCRATCH_BYTES,
+                        dev_status, stream);
+}
