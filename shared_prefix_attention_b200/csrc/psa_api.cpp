@@ -220,19 +220,55 @@ extern "C" int psa_prefill_fwd(const void* q, const void* k, const void* v, void
                                int32_t head_dim, float scale, const int32_t* dev_schedule,
                                int64_t sched_len, void* workspace, size_t ws_bytes,
                                int32_t* dev_status, void* stream) {
-  (void)sched_len;
   if (dtype != PSA_BF16 && dtype != PSA_F32) return PSA_ERR_INVALID_ARG;
   if (T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || !(scale > 0.f))
     return PSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return PSA_ERR_UNSUPPORTED;
   if (T == 0) return PSA_OK;
-  if (!q || !k || !v || !o || !dev_schedule) return PSA_ERR_INVALID_ARG;
-  (void)lse;
-  (void)workspace;
-  (void)ws_bytes;
-  (void)dev_status;
-  (void)stream;
-  return PSA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !dev_schedule || sched_len < 8) return PSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !aligned16(dev_schedule) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return PSA_ERR_INVALID_ARG;
+  const size_t need = psa_prefill_workspace_size(dtype, T, Hq, Hkv, head_dim);
+  if (dtype == PSA_F32 &&
+      (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+    return PSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  PrefillArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.out_f32 = dtype == PSA_F32;
+  a.lse = lse;
+  a.T = T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = head_dim;
+  a.scale = scale;
+  a.sched = dev_schedule;
+  a.sched_len = sched_len;
+  a.status = dev_status;
+  a.stream = s;
+  if (dtype == PSA_F32) {
+    // fp32 inputs are rounded once to bf16 in the workspace (fp32 accumulate,
+    // fp32 output)
+    auto r = [](size_t x) { return (x + 255) / 256 * 256; };
+    uint8_t* w = static_cast<uint8_t*>(workspace) + 256;
+    const size_t nq = size_t(T) * Hq * head_dim, nk = size_t(T) * Hkv * head_dim;
+    void* qb = w;
+    void* kb = w + r(nq * 2);
+    void* vb = w + r(nq * 2) + r(nk * 2);
+    int rc = launch_convert_f32_bf16(static_cast<const float*>(q), qb, int64_t(nq), s);
+    if (rc == PSA_OK) rc = launch_convert_f32_bf16(static_cast<const float*>(k), kb, int64_t(nk), s);
+    if (rc == PSA_OK) rc = launch_convert_f32_bf16(static_cast<const float*>(v), vb, int64_t(nk), s);
+    if (rc != PSA_OK) return rc;
+    a.q = qb;
+    a.k = kb;
+    a.v = vb;
+  }
+  return launch_prefill(a);
 }
 
 // ------------------------------------------------------------------ sparse latent

@@ -58,9 +58,8 @@ struct PrefillArgs {
   float* lse;
   int32_t T, Hq, Hkv, D;
   float scale;
-  const int32_t* sched;
-  int32_t n_items, n_kv, n_rect;
-  int32_t* counter;  // device scratch for the dynamic tile scheduler
+  const int32_t* sched;  // device copy of a psa_build_schedule result
+  int64_t sched_len;
   int32_t* status;
   cudaStream_t stream;
 };
