@@ -318,8 +318,13 @@ class SparseRunner(Runner):
                                lse=self.lse)
 
 
+VERIFY_SMALL = W.VerifyWorkload("verify B=8 L=16384 drafts=4 H=32/8 d=128 splits=32 bf16", B=8,
+                                L=16384, Ld=4, Hq=32, Hkv=8, d=128, nsplit=32, seed=4)
+
+
 def make_runner(name: str, dev):
     return {"grpo": lambda: PrefillRunner(W.GRPO, dev),
+            "verify8": lambda: VerifyRunner(VERIFY_SMALL, dev),
             "tiny": lambda: PrefillRunner(W.TINY, dev),
             "large": lambda: PrefillRunner(W.LARGE, dev),
             "verify": lambda: VerifyRunner(W.VERIFY, dev),
@@ -390,7 +395,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="grpo",
-                    choices=["grpo", "tiny", "large", "verify", "sparse"])
+                    choices=["grpo", "tiny", "large", "verify", "verify8", "sparse"])
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -455,7 +460,7 @@ def main():
             torch.cuda.empty_cache()
         out["extras"] = extras
 
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and args.cpu_budget > 0:
         done, secs, sample = runner.oracle_sample(args.cpu_budget)
         scale = 1e12 if runner.unit == "TFLOP/s" else 1e9
         out["cpu_baseline"] = {"value": done / secs / scale, "unit": runner.unit,

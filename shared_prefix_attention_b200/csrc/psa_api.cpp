@@ -207,12 +207,12 @@ extern "C" int psa_prefill_tiles(int32_t head_dim, int32_t* tile_m, int32_t* til
 
 extern "C" size_t psa_prefill_workspace_size(int dtype, int32_t T, int32_t Hq, int32_t Hkv,
                                              int32_t head_dim) {
-  size_t bytes = 256;  // scheduler counter
-  if (dtype == PSA_F32 && T > 0) {
-    auto r = [](size_t x) { return (x + 255) / 256 * 256; };
-    bytes += r(size_t(T) * Hq * head_dim * 2) + 2 * r(size_t(T) * Hkv * head_dim * 2);
-  }
-  return bytes;
+  (void)dtype;
+  (void)T;
+  (void)Hq;
+  (void)Hkv;
+  (void)head_dim;
+  return 256;  // the tile scheduler's counter
 }
 
 extern "C" int psa_prefill_fwd(const void* q, const void* k, const void* v, void* o,
@@ -230,8 +230,7 @@ extern "C" int psa_prefill_fwd(const void* q, const void* k, const void* v, void
       !aligned16(dev_schedule) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return PSA_ERR_INVALID_ARG;
   const size_t need = psa_prefill_workspace_size(dtype, T, Hq, Hkv, head_dim);
-  if (dtype == PSA_F32 &&
-      (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return PSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -251,23 +250,7 @@ extern "C" int psa_prefill_fwd(const void* q, const void* k, const void* v, void
   a.sched_len = sched_len;
   a.status = dev_status;
   a.stream = s;
-  if (dtype == PSA_F32) {
-    // fp32 inputs are rounded once to bf16 in the workspace (fp32 accumulate,
-    // fp32 output)
-    auto r = [](size_t x) { return (x + 255) / 256 * 256; };
-    uint8_t* w = static_cast<uint8_t*>(workspace) + 256;
-    const size_t nq = size_t(T) * Hq * head_dim, nk = size_t(T) * Hkv * head_dim;
-    void* qb = w;
-    void* kb = w + r(nq * 2);
-    void* vb = w + r(nq * 2) + r(nk * 2);
-    int rc = launch_convert_f32_bf16(static_cast<const float*>(q), qb, int64_t(nq), s);
-    if (rc == PSA_OK) rc = launch_convert_f32_bf16(static_cast<const float*>(k), kb, int64_t(nk), s);
-    if (rc == PSA_OK) rc = launch_convert_f32_bf16(static_cast<const float*>(v), vb, int64_t(nk), s);
-    if (rc != PSA_OK) return rc;
-    a.q = qb;
-    a.k = kb;
-    a.v = vb;
-  }
+  a.counter = static_cast<int32_t*>(workspace);
   return launch_prefill(a);
 }
 

@@ -53,18 +53,18 @@ struct PrefillArgs {
   const void* q;  // bf16 [T, Hq, D]
   const void* k;  // bf16 [T, Hkv, D]
   const void* v;
-  void* o;        // [T, Hq, D], bf16 or fp32 (out_f32)
+  void* o;        // [T, Hq, D], bf16, or fp32 when out_f32 (then q/k/v are fp32 too)
   bool out_f32;
   float* lse;
   int32_t T, Hq, Hkv, D;
   float scale;
   const int32_t* sched;  // device copy of a psa_build_schedule result
   int64_t sched_len;
+  int32_t* counter;      // device word for the dynamic tile scheduler
   int32_t* status;
   cudaStream_t stream;
 };
 int launch_prefill(const PrefillArgs& a);
-int launch_convert_f32_bf16(const float* src, void* dst, int64_t n, cudaStream_t s);
 
 // ---------------------------------------------------------------- sparse latent
 

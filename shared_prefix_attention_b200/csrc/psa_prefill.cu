@@ -6,7 +6,9 @@
 // forward that is mathematically equivalent to running each [prefix; s_i]).
 //
 // sm_100a design (one CTA per SM, persistent over (Q tile, query head)
-// units taken longest-first from the host schedule):
+// units; the host schedule lists them longest-first and the producer hands
+// them out dynamically through a global counter, so the long suffix tiles
+// start first and the short prefix tiles fill the tail):
 //   warp 0      TMA producer: Q tile once per unit; K and V tiles of the
 //               unit's visible KV tiles only (invisible tiles are never
 //               touched) into two-slot rings, 128-byte swizzle, no multicast.
@@ -39,6 +41,7 @@ constexpr int kSoftmaxWarp0 = 4;   // warps 4..7 own TMEM lanes 0..127
 constexpr float kRescaleLog2 = 8.f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSCol0 = 0, kSCol1 = 128, kOCol = 256;
+constexpr int kSchedSlots = 4;  // units the producer may fetch ahead
 
 template <int D>
 struct Cfg {
@@ -52,7 +55,7 @@ struct Cfg {
   static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
   static constexpr uint32_t OFF_P = OFF_V + NS * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr uint32_t NBAR = 2 + 4 * NS + 8 + 2;
+  static constexpr uint32_t NBAR = 2 + 4 * NS + 8 + 2 + 2 * kSchedSlots;
   static constexpr uint32_t SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
 };
 
@@ -65,11 +68,13 @@ struct Params {
   int32_t out_f32;
   float scale_log2;
   int32_t* status;
+  int32_t* counter;  // next unit to hand out (zeroed before every launch)
 };
 
 struct Bars {
   uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty;
   uint64_t *s_full, *s_free, *p_full, *p_free, *o_full, *o_free;
+  uint64_t *sch_full, *sch_empty;
 };
 
 __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int a, int b) {
@@ -95,6 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
+  __shared__ int sch_unit[kSchedSlots];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -128,6 +134,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.p_free = B.p_full + 2;
   B.o_full = B.p_free + 2;
   B.o_free = B.o_full + 1;
+  B.sch_full = B.o_free + 1;
+  B.sch_empty = B.sch_full + kSchedSlots;
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -147,6 +155,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(B.o_full, 1);
     mbar_init(B.o_free, 4);
+    for (int i = 0; i < kSchedSlots; ++i) {
+      mbar_init(B.sch_full + i, 1);
+      mbar_init(B.sch_empty + i, 5);  // the MMA thread and the four softmax warps
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -171,7 +183,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmap_v);
       uint32_t kc = 0, uc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (uint32_t i = 0; ok; ++i) {
+        // dynamic scheduler: hand the next unit to every role through smem
+        const int slot = i % kSchedSlots;
+        if (!mbar_wait(B.sch_empty + slot, ((i / kSchedSlots) & 1) ^ 1, &abort_flag, p.status))
+          break;
+        const int u = atomicAdd(p.counter, 1);
+        sch_unit[slot] = u;
+        mbar_arrive(B.sch_full + slot);
+        if (u >= units) break;
         const int4 it = __ldg(items + u / p.Hq);
         const int h = u % p.Hq, kvh = h / p.G;
         if (it.w == 0) continue;
@@ -244,7 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (uint32_t i = 0; ok; ++i) {
+        const int slot_s = i % kSchedSlots;
+        if (!mbar_wait(B.sch_full + slot_s, (i / kSchedSlots) & 1, &abort_flag, p.status)) break;
+        const int u = sch_unit[slot_s];
+        mbar_arrive(B.sch_empty + slot_s);
+        if (u >= units) break;
         const int4 it = __ldg(items + u / p.Hq);
         if (it.w == 0) continue;
         if (!mbar_wait(B.q_full, uc & 1, &abort_flag, p.status)) break;
@@ -295,7 +320,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
     uint32_t tg = 0, uc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+    for (uint32_t i = 0; ok; ++i) {
+      const int slot_s = i % kSchedSlots;
+      if (!mbar_wait(B.sch_full + slot_s, (i / kSchedSlots) & 1, &abort_flag, p.status)) break;
+      const int u = sch_unit[slot_s];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(B.sch_empty + slot_s);
+      if (u >= units) break;
       const int4 it = __ldg(items + u / p.Hq);
       const int h = u % p.Hq;
       const int q = it.x + r;
@@ -357,14 +388,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        float mx = -INFINITY;
+        // raw logits stay unscaled (scale > 0 commutes with max); masked
+        // entries become -inf.  Eight independent max chains.
+        if (need_mask) {
 #pragma unroll
-        for (int i = 0; i < BN; ++i) {
-          const bool on = (vis[i >> 5] >> (i & 31)) & 1u;
-          const float x = on ? s[i] * p.scale_log2 : -INFINITY;
-          s[i] = x;
-          mx = fmaxf(mx, x);
+          for (int i = 0; i < BN; ++i)
+            s[i] = ((vis[i >> 5] >> (i & 31)) & 1u) ? s[i] : -INFINITY;
         }
+        float mx8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+#pragma unroll
+        for (int i = 8; i < BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
+                         p.scale_log2;
         const float m_new = fmaxf(m_run, mx);
         const bool resc = m_new > m_run + kRescaleLog2;
         if (__any_sync(0xffffffffu, resc) && j > 0) {
@@ -399,15 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint32_t prow = sP + sb * C::P_BYTES + r * 128;
-        float lsum = 0.f;
+        const float sc = p.scale_log2, neg_m = -m_use;
+        float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < BN / 8; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const float p0 = fast_exp2(s[c * 8 + 2 * k] - m_use);
-            const float p1 = fast_exp2(s[c * 8 + 2 * k + 1] - m_use);
-            lsum += p0 + p1;
+            const float p0 = fast_exp2(fmaf(s[c * 8 + 2 * k], sc, neg_m));
+            const float p1 = fast_exp2(fmaf(s[c * 8 + 2 * k + 1], sc, neg_m));
+            ls8[2 * k] += p0;
+            ls8[2 * k + 1] += p1;
             w[k] = pack_bf16(p0, p1);
           }
           const uint32_t addr = prow + (c >> 3) * (BM * 128) + (((c & 7) ^ (r & 7)) << 4);
@@ -415,6 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                        "r"(w[1]), "r"(w[2]), "r"(w[3])
                        : "memory");
         }
+        const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) +
+                           ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
         l_run += lsum;
         fence_proxy_async_smem();
         tc_fence_before();
@@ -476,18 +518,88 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-__global__ void convert_f32_bf16_kernel(const float* __restrict__ src,
-                                        __nv_bfloat16* __restrict__ dst, int64_t n) {
-  const int64_t stride = int64_t(gridDim.x) * blockDim.x * 4;
-  for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 4; i < n; i += stride) {
-    if (i + 3 < n) {
-      const float4 v = *reinterpret_cast<const float4*>(src + i);
-      uint2 w = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
-      *reinterpret_cast<uint2*>(dst + i) = w;
-    } else {
-      for (int64_t k = i; k < n; ++k) dst[k] = __float2bfloat16(src[k]);
-    }
+template <int D>
+__global__ void __launch_bounds__(256) prefill_f32_kernel(
+    const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
+    float* __restrict__ o, float* __restrict__ lse, const int32_t* __restrict__ sch,
+    int64_t sched_len, int32_t Hq, int32_t G, float scale_log2, int32_t* status) {
+  constexpr int E = D / 32;
+  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2), n_rect = __ldg(sch + 3);
+  const bool bad = __ldg(sch + 0) != 0x50534131 || __ldg(sch + 4) != BM ||
+                   __ldg(sch + 5) != BN || n_items < 0 || n_kv < 0 || n_rect < 0 ||
+                   8 + 4 * int64_t(n_items) + 4 * int64_t(n_kv) + 5 * int64_t(n_rect) >
+                       sched_len;
+  if (bad) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) report_status(status, PSA_ERR_INVALID_ARG);
+    return;
   }
+  const int4* items = reinterpret_cast<const int4*>(sch + 8);
+  const int4* kvs = reinterpret_cast<const int4*>(sch + 8 + 4 * n_items);
+  const int32_t* rects = sch + 8 + 4 * n_items + 4 * n_kv;
+  const int lane = threadIdx.x & 31;
+  const int64_t total = int64_t(n_items) * BM * Hq;
+  const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t u = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; u < total;
+       u += nwarps) {
+    const int item = int(u / (int64_t(BM) * Hq));
+    const int rem = int(u % (int64_t(BM) * Hq));
+    const int r = rem / Hq, h = rem % Hq;
+    const int4 it = __ldg(items + item);
+    if (r >= it.y) continue;
+    const int qi = it.x + r, kvh = h / G;
+    const int Hkv = Hq / G;
+    float qv[E], acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      qv[e] = q[(size_t(qi) * Hq + h) * D + lane * E + e];
+      acc[e] = 0.f;
+    }
+    float m = -INFINITY, l = 0.f;
+    for (int j = 0; j < it.w; ++j) {
+      const int4 ent = __ldg(kvs + it.z + j);
+      for (int kk = ent.x; kk < ent.x + ent.y; ++kk) {
+        bool on = ent.w == 0;
+        for (int ri = 0; ri < ent.w && !on; ++ri) {
+          const int32_t* rc = rects + 5 * (ent.z + ri);
+          const int rq0 = rc[0], rq1 = rc[1], rk0 = rc[2], rk1 = rc[3], causal = rc[4];
+          on = qi >= rq0 && qi < rq1 && kk >= rk0 && kk < rk1 && (!causal || kk - rk0 <= qi - rq0);
+        }
+        if (!on) continue;
+        const float* kr = k + (size_t(kk) * Hkv + kvh) * D + lane * E;
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) d = fmaf(qv[e], kr[e], d);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        const float sv = d * scale_log2;
+        const float mn = fmaxf(m, sv);
+        const float alpha = exp2f(m - mn);
+        const float pe = exp2f(sv - mn);
+        l = l * alpha + pe;
+        const float* vr = v + (size_t(kk) * Hkv + kvh) * D + lane * E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(acc[e], alpha, pe * vr[e]);
+        m = mn;
+      }
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[(size_t(qi) * Hq + h) * D + lane * E + e] = acc[e] * inv;
+    if (lse && lane == 0) lse[size_t(qi) * Hq + h] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+  }
+}
+
+template <int D>
+int launch_prefill_f32_d(const PrefillArgs& a) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PSA_ERR_CUDA;
+  const int grid = 4 * sm_count(dev);
+  if (grid <= 0) return PSA_ERR_CUDA;
+  prefill_f32_kernel<D><<<grid, 256, 0, a.stream>>>(
+      static_cast<const float*>(a.q), static_cast<const float*>(a.k),
+      static_cast<const float*>(a.v), static_cast<float*>(a.o), a.lse, a.sched, a.sched_len,
+      a.Hq, a.Hq / a.Hkv, a.scale * kLog2e, a.status);
+  return cudaGetLastError() == cudaSuccess ? PSA_OK : PSA_ERR_CUDA;
 }
 
 template <int D>
@@ -526,12 +638,15 @@ int launch_prefill_d(const PrefillArgs& a) {
   p.out_f32 = a.out_f32 ? 1 : 0;
   p.scale_log2 = a.scale * kLog2e;
   p.status = a.status;
+  p.counter = a.counter;
   auto kern = prefill_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM)) !=
       cudaSuccess)
     return PSA_ERR_CUDA;
   const int grid = sm_count(dev);
   if (grid <= 0) return PSA_ERR_CUDA;
+  if (cudaMemsetAsync(a.counter, 0, sizeof(int32_t), a.stream) != cudaSuccess)
+    return PSA_ERR_CUDA;
   kern<<<grid, kThreads, C::SMEM, a.stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? PSA_OK : PSA_ERR_CUDA;
 }
@@ -539,6 +654,16 @@ int launch_prefill_d(const PrefillArgs& a) {
 }  // namespace
 
 int launch_prefill(const PrefillArgs& a) {
+  if (a.out_f32) {
+    switch (a.D) {
+      case 64:
+        return launch_prefill_f32_d<64>(a);
+      case 128:
+        return launch_prefill_f32_d<128>(a);
+      default:
+        return PSA_ERR_UNSUPPORTED;
+    }
+  }
   switch (a.D) {
     case 64:
       return launch_prefill_d<64>(a);
@@ -547,15 +672,6 @@ int launch_prefill(const PrefillArgs& a) {
     default:
       return PSA_ERR_UNSUPPORTED;
   }
-}
-
-int launch_convert_f32_bf16(const float* src, void* dst, int64_t n, cudaStream_t s) {
-  if (n <= 0) return PSA_OK;
-  int64_t blocks = (n / 4 + 255) / 256;
-  if (blocks > 4096) blocks = 4096;
-  if (blocks < 1) blocks = 1;
-  convert_f32_bf16_kernel<<<int(blocks), 256, 0, s>>>(src, static_cast<__nv_bfloat16*>(dst), n);
-  return cudaGetLastError() == cudaSuccess ? PSA_OK : PSA_ERR_CUDA;
 }
 
 }  // namespace psa
