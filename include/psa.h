@@ -100,25 +100,30 @@ int psa_spec_flat(int32_t P, int32_t N, int32_t S, psa_segment *out, int32_t cap
 int psa_build_spec(const psa_segment *segs, int32_t nseg, psa_rect *out, int32_t cap,
                    int32_t *nout);
 
-/* Tile schedule for psa_prefill_fwd (host int32 array).  Q tiles of tile_m
- * rows and KV tiles of tile_n keys are cut per group (cu_seqlens, host,
- * ngroups+1 entries); for every Q tile it lists only the KV tiles with at
- * least one visible pair, flagging each as fully visible or partial, and
- * for partial tiles it copies the rectangles that cut them.  Q tiles are
- * ordered longest-first (most KV tiles first).
+/* Tile schedule for psa_prefill_fwd (host int32 array).  Q blocks of
+ * tile_m rows (even; each block is two halves of tile_m/2 rows that one CTA
+ * processes side by side) and KV tiles of tile_n keys are cut per group
+ * (cu_seqlens, host, ngroups+1 entries).  For every Q block it lists only
+ * the KV tiles in which at least one half has a visible pair, and for each
+ * half whether it takes part, whether every pair is visible, and -- for a
+ * partially visible half -- copies of the rectangles that cut it.  Q blocks
+ * are ordered longest-first (most KV tiles first).
  *
- * Layout (int32):  [0] magic 0x50534131  [1] n_items  [2] n_kv  [3] n_rect
+ * Layout (int32):  [0] magic 0x50534132  [1] n_items  [2] n_kv  [3] n_rect
  *   [4] tile_m  [5] tile_n  [6] total tokens  [7] max KV tiles per item
- *   items   at 8:                  {q0, q_len, kv_begin, kv_count} x n_items
- *   kv      at 8 + 4*n_items:      {k0, k_len, rect_begin, rect_count} x n_kv
- *                                  (rect_count == 0: every pair visible)
- *   rects   at 8 + 4*(n_items+n_kv): {q0, q1, k0, k1, causal} x n_rect
+ *   items  at 8:                  {q0, q_len, kv_begin, kv_count} x n_items
+ *   kv     at 8 + 4*n_items:      {k0, k_len, a_rect_begin, a_rect_count,
+ *                                  b_rect_begin, b_rect_count, flags, 0} x n_kv
+ *          flags: bit 0 / 1 = half A / B has visible pairs in the tile,
+ *                 bit 2 / 3 = every pair of half A / B is visible
+ *   rects  at 8 + 4*n_items + 8*n_kv: {q0, q1, k0, k1, causal} x n_rect
  * Returns PSA_ERR_CAPACITY (with *nout = needed length) if cap is short. */
 int psa_build_schedule(const psa_rect *rects, int32_t nrect, const int32_t *cu_seqlens,
                        int32_t ngroups, int32_t tile_m, int32_t tile_n, int32_t *out,
                        int64_t cap, int64_t *nout);
 
-/* The tile sizes psa_prefill_fwd expects in its schedule (tile_m, tile_n). */
+/* The block and tile sizes psa_prefill_fwd expects in its schedule:
+ * tile_m query rows per block (two halves), tile_n keys per KV tile. */
 int psa_prefill_tiles(int32_t head_dim, int32_t *tile_m, int32_t *tile_n);
 
 /* ------------------------------------------------------------------------

@@ -200,7 +200,7 @@ extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const vo
 extern "C" int psa_prefill_tiles(int32_t head_dim, int32_t* tile_m, int32_t* tile_n) {
   if (!tile_m || !tile_n) return PSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return PSA_ERR_UNSUPPORTED;
-  *tile_m = 128;
+  *tile_m = 256;  // two 128-row halves per block
   *tile_n = 128;
   return PSA_OK;
 }

@@ -5,24 +5,25 @@
 // dedup layout, block-causal rectangle spec instead of a dense mask, one
 // forward that is mathematically equivalent to running each [prefix; s_i]).
 //
-// sm_100a design (one CTA per SM, persistent over (Q tile, query head)
-// units; the host schedule lists them longest-first and the producer hands
-// them out dynamically through a global counter, so the long suffix tiles
-// start first and the short prefix tiles fill the tail):
-//   warp 0      TMA producer: Q tile once per unit; K and V tiles of the
-//               unit's visible KV tiles only (invisible tiles are never
-//               touched) into two-slot rings, 128-byte swizzle, no multicast.
-//   warp 1      tcgen05 issuer (one thread): S = Q K^T into a double-
-//               buffered TMEM S, then O += P V into a TMEM O accumulator,
-//               ordered QK_0, QK_1, PV_0, QK_2, PV_1, ... so the tensor
-//               pipe computes the next S while the softmax works.
-//   warps 4..7  softmax warpgroup, one query row per thread (= TMEM lane):
-//               masks partial tiles from the copied rectangles, keeps the
-//               running max in the log2 domain with lazy rescaling (O is
-//               rescaled only when the max grows by more than 2^8), writes
-//               P as bf16 into a double-buffered swizzled shared tile that
-//               the next MMA reads as its K-major A operand, and runs the
-//               epilogue (O / l, LSE) straight from TMEM.
+// sm_100a design.  One CTA per SM, persistent over units (Q block of 256
+// rows, query head).  The host schedule lists the blocks longest-first and
+// the producer hands units out through a global counter, so long suffix
+// blocks start first and short prefix blocks fill the tail.  A block is two
+// 128-row halves A and B that share every K/V tile load:
+//   warp 0       TMA producer: the Q block, then the K and V tiles of the
+//                block's visible KV tiles only (invisible tiles are never
+//                touched), 128-byte swizzle, no multicast.
+//   warp 1       tcgen05 issuer (one thread).  Per half X: S_X = Q_X K^T
+//                into TMEM, then O_X += P_X V with P_X read from TMEM where
+//                the softmax left it (aliasing S_X).  Issue order
+//                PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1): while one half's
+//                softmax runs, the tensor pipe works on the other half.
+//   warps 4..7   softmax of half A, warps 8..11 softmax of half B: one query
+//                row per thread (= TMEM lane).  Masks partial tiles from the
+//                copied rectangles, keeps the running max in the log2 domain
+//                with lazy rescaling (O is rescaled in TMEM only when the
+//                max grows by more than 2^8), writes P as bf16 over its S
+//                columns, and runs the epilogue (O / l, LSE) from TMEM.
 // Every wait is bounded: a stuck pipeline reports PSA_ERR_TIMEOUT through
 // the status word, the CTA unwinds and frees its TMEM.
 #include <cuda_bf16.h>
@@ -34,28 +35,26 @@
 namespace psa {
 namespace {
 
-constexpr int BM = 128;            // query rows per tile
+constexpr int BM = 128;            // query rows per half
+constexpr int BLOCK_M = 2 * BM;    // query rows per schedule block
 constexpr int BN = 128;            // keys per tile
-constexpr int kThreads = 256;      // 8 warps
-constexpr int kSoftmaxWarp0 = 4;   // warps 4..7 own TMEM lanes 0..127
+constexpr int kThreads = 384;      // 12 warps
 constexpr float kRescaleLog2 = 8.f;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSCol0 = 0, kSCol1 = 128, kOCol = 256;
-constexpr int kSchedSlots = 4;  // units the producer may fetch ahead
+constexpr uint32_t kTmemCols = 512;  // per half: S at X*256, O at X*256 + 128
+constexpr int kSchedSlots = 4;       // units the producer may fetch ahead
+constexpr int kSchedReaders = 9;     // the MMA thread and the eight softmax warps
 
 template <int D>
 struct Cfg {
   static constexpr int NPART = D / 64;  // 128-byte swizzle atoms across d
-  static constexpr uint32_t Q_BYTES = BM * D * 2;
+  static constexpr uint32_t Q_BYTES = BM * D * 2;   // one half
   static constexpr uint32_t KV_BYTES = BN * D * 2;
-  static constexpr uint32_t P_BYTES = BM * BN * 2;
-  static constexpr int NS = D == 128 ? 2 : 4;  // K and V ring slots
+  static constexpr int NS = D == 128 ? 2 : 4;       // K and V ring slots
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+  static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr uint32_t OFF_P = OFF_V + NS * KV_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr uint32_t NBAR = 2 + 4 * NS + 8 + 2 + 2 * kSchedSlots;
+  static constexpr uint32_t OFF_BAR = OFF_V + NS * KV_BYTES;
+  static constexpr uint32_t NBAR = 2 + 4 * NS + 8 + 2 * kSchedSlots;
   static constexpr uint32_t SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
 };
 
@@ -65,7 +64,6 @@ struct Params {
   void* o;
   float* lse;
   int32_t T, Hq, Hkv, G;
-  int32_t out_f32;
   float scale_log2;
   int32_t* status;
   int32_t* counter;  // next unit to hand out (zeroed before every launch)
@@ -73,7 +71,7 @@ struct Params {
 
 struct Bars {
   uint64_t *q_full, *q_empty, *k_full, *k_empty, *v_full, *v_empty;
-  uint64_t *s_full, *s_free, *p_full, *p_free, *o_full, *o_free;
+  uint64_t *s_full, *p_full, *pv_done, *o_free;  // [2] each, one per half
   uint64_t *sch_full, *sch_empty;
 };
 
@@ -86,6 +84,52 @@ __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int a, int b) {
       const uint32_t bits = n == 32 ? 0xffffffffu : ((1u << n) - 1u);
       m[w] |= bits << (lo - 32 * w);
     }
+  }
+}
+
+// Header check shared by both prefill kernels (uniform across threads).
+__device__ __forceinline__ bool schedule_ok(const int32_t* sch, int64_t len) {
+  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2), n_rect = __ldg(sch + 3);
+  return __ldg(sch + 0) == 0x50534132 && __ldg(sch + 4) == BLOCK_M && __ldg(sch + 5) == BN &&
+         n_items >= 0 && n_kv >= 0 && n_rect >= 0 &&
+         8 + 4 * int64_t(n_items) + 8 * int64_t(n_kv) + 5 * int64_t(n_rect) <= len;
+}
+
+struct KvEntry {
+  int k0, klen, rb[2], rc[2], flags;
+};
+
+__device__ __forceinline__ KvEntry load_kv(const int32_t* kvs, int idx) {
+  const int4 a = __ldg(reinterpret_cast<const int4*>(kvs) + 2 * idx);
+  const int4 b = __ldg(reinterpret_cast<const int4*>(kvs) + 2 * idx + 1);
+  KvEntry e;
+  e.k0 = a.x;
+  e.klen = a.y;
+  e.rb[0] = a.z;
+  e.rc[0] = a.w;
+  e.rb[1] = b.x;
+  e.rc[1] = b.y;
+  e.flags = b.z;
+  return e;
+}
+
+// Visible keys of row q inside KV tile e for half x, as a 128-bit mask.
+__device__ __forceinline__ void row_visibility(const KvEntry& e, int x, int q,
+                                               const int32_t* rects, uint32_t (&vis)[4]) {
+  vis[0] = vis[1] = vis[2] = vis[3] = 0u;
+  if (e.flags & (4 << x)) {
+    set_bits(vis, 0, e.klen);
+    return;
+  }
+  for (int ri = 0; ri < e.rc[x]; ++ri) {
+    const int32_t* rc = rects + 5 * (e.rb[x] + ri);
+    const int rq0 = __ldg(rc), rq1 = __ldg(rc + 1), rk0 = __ldg(rc + 2), rk1 = __ldg(rc + 3),
+              causal = __ldg(rc + 4);
+    if (q < rq0 || q >= rq1) continue;
+    int hi = causal ? min(rk1, rk0 + (q - rq0) + 1) : rk1;
+    hi = min(hi, e.k0 + e.klen);
+    const int lo = max(rk0, e.k0);
+    if (lo < hi) set_bits(vis, lo - e.k0, hi - e.k0);
   }
 }
 
@@ -104,20 +148,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- schedule header (every thread reads it; the decision is uniform)
   const int32_t* sch = p.sched;
-  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2), n_rect = __ldg(sch + 3);
-  const bool bad = __ldg(sch + 0) != 0x50534131 || __ldg(sch + 4) != BM ||
-                   __ldg(sch + 5) != BN || n_items < 0 || n_kv < 0 || n_rect < 0 ||
-                   8 + 4 * int64_t(n_items) + 4 * int64_t(n_kv) + 5 * int64_t(n_rect) >
-                       p.sched_len;
-  if (bad) {
+  if (!schedule_ok(sch, p.sched_len)) {
     if (threadIdx.x == 0) report_status(p.status, PSA_ERR_INVALID_ARG);
     return;
   }
+  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2);
   const int4* items = reinterpret_cast<const int4*>(sch + 8);
-  const int4* kvs = reinterpret_cast<const int4*>(sch + 8 + 4 * n_items);
-  const int32_t* rects = sch + 8 + 4 * n_items + 4 * n_kv;
+  const int32_t* kvs = sch + 8 + 4 * n_items;
+  const int32_t* rects = kvs + 8 * n_kv;
   const int units = n_items * p.Hq;
 
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -129,12 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.v_full = B.k_empty + C::NS;
   B.v_empty = B.v_full + C::NS;
   B.s_full = B.v_empty + C::NS;
-  B.s_free = B.s_full + 2;
-  B.p_full = B.s_free + 2;
-  B.p_free = B.p_full + 2;
-  B.o_full = B.p_free + 2;
-  B.o_free = B.o_full + 1;
-  B.sch_full = B.o_free + 1;
+  B.p_full = B.s_full + 2;
+  B.pv_done = B.p_full + 2;
+  B.o_free = B.pv_done + 2;
+  B.sch_full = B.o_free + 2;
   B.sch_empty = B.sch_full + kSchedSlots;
 
   if (threadIdx.x == 0) {
@@ -147,17 +184,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(B.v_full + i, 1);
       mbar_init(B.v_empty + i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(B.s_full + i, 1);
-      mbar_init(B.s_free + i, 4);
-      mbar_init(B.p_full + i, 4);
-      mbar_init(B.p_free + i, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(B.s_full + x, 1);
+      mbar_init(B.p_full + x, 4);
+      mbar_init(B.pv_done + x, 1);
+      mbar_init(B.o_free + x, 4);
     }
-    mbar_init(B.o_full, 1);
-    mbar_init(B.o_free, 4);
     for (int i = 0; i < kSchedSlots; ++i) {
       mbar_init(B.sch_full + i, 1);
-      mbar_init(B.sch_empty + i, 5);  // the MMA thread and the four softmax warps
+      mbar_init(B.sch_empty + i, kSchedReaders);
     }
     fence_barrier_init();
   }
@@ -170,11 +205,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_slot;
 
-  const uint32_t sQ = smem_u32(smem + C::OFF_Q);
-  const uint32_t sK = smem_u32(smem + C::OFF_K);
-  const uint32_t sV = smem_u32(smem + C::OFF_V);
-  const uint32_t sP = smem_u32(smem + C::OFF_P);
-
   if (warp == 0) {
     // ================================================================ producer
     if (lane == 0) {
@@ -184,24 +214,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kc = 0, uc = 0;
       bool ok = true;
       for (uint32_t i = 0; ok; ++i) {
-        // dynamic scheduler: hand the next unit to every role through smem
-        const int slot = i % kSchedSlots;
-        if (!mbar_wait(B.sch_empty + slot, ((i / kSchedSlots) & 1) ^ 1, &abort_flag, p.status))
+        const int slot_s = i % kSchedSlots;
+        if (!mbar_wait(B.sch_empty + slot_s, ((i / kSchedSlots) & 1) ^ 1, &abort_flag,
+                       p.status))
           break;
         const int u = atomicAdd(p.counter, 1);
-        sch_unit[slot] = u;
-        mbar_arrive(B.sch_full + slot);
+        sch_unit[slot_s] = u;
+        mbar_arrive(B.sch_full + slot_s);
         if (u >= units) break;
         const int4 it = __ldg(items + u / p.Hq);
         const int h = u % p.Hq, kvh = h / p.G;
         if (it.w == 0) continue;
         if (!mbar_wait(B.q_empty, (uc & 1) ^ 1, &abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(B.q_full, C::Q_BYTES);
+        mbar_arrive_expect_tx(B.q_full, 2 * C::Q_BYTES);
 #pragma unroll
-        for (int part = 0; part < C::NPART; ++part)
-          tma_load_3d(smem + C::OFF_Q + part * BM * 128, &tmap_q, B.q_full, part * 64, h, it.x);
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+          for (int part = 0; part < C::NPART; ++part)
+            tma_load_3d(smem + C::OFF_Q + x * C::Q_BYTES + part * BM * 128, &tmap_q, B.q_full,
+                        part * 64, h, it.x + x * BM);
         for (int j = 0; j < it.w; ++j) {
-          const int k0 = __ldg(&kvs[it.z + j].x);
+          const int k0 = __ldg(kvs + 8 * (it.z + j));
           const int slot = kc % C::NS;
           const uint32_t ph = (kc / C::NS) & 1;
           if (!mbar_wait(B.k_empty + slot, ph ^ 1, &abort_flag, p.status)) {
@@ -238,29 +271,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = umma_idesc_bf16(BM, BN, false, false);
       const uint32_t idesc_pv = umma_idesc_bf16(BM, D, false, true);
-      uint32_t kc = 0, vc = 0, tg = 0, uc = 0;
+      const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+      const uint32_t sK = smem_u32(smem + C::OFF_K);
+      const uint32_t sV = smem_u32(smem + C::OFF_V);
+      uint32_t kc = 0, uc = 0;
+      uint32_t pvc[2] = {0, 0};  // PVs issued per half (all units)
+      uint32_t uhc[2] = {0, 0};  // units in which the half had work
       bool ok = true;
 
-      auto issue_pv = [&](uint32_t t, bool first, bool last) -> bool {
-        const uint32_t pb = t & 1;
-        if (!mbar_wait(B.p_full + pb, (t >> 1) & 1, &abort_flag, p.status)) return false;
-        const int slot = vc % C::NS;
-        if (!mbar_wait(B.v_full + slot, (vc / C::NS) & 1, &abort_flag, p.status)) return false;
-        if (first && !mbar_wait(B.o_free, (uc & 1) ^ 1, &abort_flag, p.status)) return false;
+      // S_X = Q_X K_t^T into the S columns of half x
+      auto issue_qk = [&](int x, uint32_t t_glob) -> bool {
+        const int slot = t_glob % C::NS;
+        if (!mbar_wait(B.k_full + slot, (t_glob / C::NS) & 1, &abort_flag, p.status))
+          return false;
         tc_fence_after();
-        const uint32_t pbase = sP + pb * C::P_BYTES;
+        const uint32_t qbase = sQ + x * C::Q_BYTES, kbase = sK + slot * C::KV_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
+          umma_ss(tmem + x * 256, umma_desc_sw128(qbase + off, 16, 1024),
+                  umma_desc_sw128(kbase + off, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(B.s_full + x);
+        return true;
+      };
+      // O_X += P_X V_t, P_X in TMEM over the first 64 columns of S_X
+      auto issue_pv = [&](int x, uint32_t t_glob, bool first) -> bool {
+        if (!mbar_wait(B.p_full + x, pvc[x] & 1, &abort_flag, p.status)) return false;
+        const int slot = t_glob % C::NS;
+        if (!mbar_wait(B.v_full + slot, (t_glob / C::NS) & 1, &abort_flag, p.status))
+          return false;
+        if (first && !mbar_wait(B.o_free + x, (uhc[x] & 1) ^ 1, &abort_flag, p.status))
+          return false;
+        tc_fence_after();
         const uint32_t vbase = sV + slot * C::KV_BYTES;
 #pragma unroll
-        for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t a = umma_desc_sw128(pbase + (ks >> 2) * (BM * 128) + (ks & 3) * 32, 16,
-                                             1024);
-          const uint64_t b = umma_desc_sw128(vbase + ks * 2048, BN * 128, 1024);
-          umma_ss(tmem + kOCol, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
-        }
-        umma_commit(B.p_free + pb);
-        umma_commit(B.v_empty + slot);
-        if (last) umma_commit(B.o_full);
-        ++vc;
+        for (int ks = 0; ks < BN / 16; ++ks)
+          umma_ts(tmem + x * 256 + 128, tmem + x * 256 + ks * 8,
+                  umma_desc_sw128(vbase + ks * 2048, BN * 128, 1024), idesc_pv,
+                  (first && ks == 0) ? 0u : 1u);
+        umma_commit(B.pv_done + x);
+        ++pvc[x];
         return true;
       };
 
@@ -271,54 +322,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(B.sch_empty + slot_s);
         if (u >= units) break;
         const int4 it = __ldg(items + u / p.Hq);
-        if (it.w == 0) continue;
+        const int n = it.w;
+        if (n == 0) continue;
         if (!mbar_wait(B.q_full, uc & 1, &abort_flag, p.status)) break;
-        for (int j = 0; j < it.w; ++j) {
-          const int slot = kc % C::NS;
-          const uint32_t sb = tg & 1;
-          if (!mbar_wait(B.k_full + slot, (kc / C::NS) & 1, &abort_flag, p.status) ||
-              !mbar_wait(B.s_free + sb, ((tg >> 1) & 1) ^ 1, &abort_flag, p.status)) {
-            ok = false;
-            break;
+        bool started[2] = {false, false};
+        // prologue: QK of tile 0 for each half that takes part in it
+        {
+          const int f = __ldg(kvs + 8 * it.z + 6);
+          for (int x = 0; x < 2 && ok; ++x)
+            if (f & (1 << x)) ok = issue_qk(x, kc);
+          if (!ok) break;
+          umma_commit(B.k_empty + (kc % C::NS));
+          if (n == 1) umma_commit(B.q_empty);
+        }
+        for (int j = 0; j < n && ok; ++j) {
+          const int f = __ldg(kvs + 8 * (it.z + j) + 6);
+          const int fn = j + 1 < n ? __ldg(kvs + 8 * (it.z + j + 1) + 6) : 0;
+          const uint32_t t = kc + j;
+          for (int x = 0; x < 2 && ok; ++x) {
+            if (f & (1 << x)) {
+              ok = issue_pv(x, t, !started[x]);
+              started[x] = true;
+            }
+            if (ok && (fn & (1 << x))) ok = issue_qk(x, t + 1);
           }
-          tc_fence_after();
-          const uint32_t kbase = sK + slot * C::KV_BYTES;
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
-            const uint64_t a = umma_desc_sw128(sQ + off, 16, 1024);
-            const uint64_t b = umma_desc_sw128(kbase + off, 16, 1024);
-            umma_ss(tmem + (sb ? kSCol1 : kSCol0), a, b, idesc_qk, ks > 0 ? 1u : 0u);
+          if (!ok) break;
+          umma_commit(B.v_empty + (t % C::NS));
+          if (j + 1 < n) {
+            umma_commit(B.k_empty + ((t + 1) % C::NS));
+            if (j + 2 == n) umma_commit(B.q_empty);
           }
-          umma_commit(B.s_full + sb);
-          umma_commit(B.k_empty + slot);
-          if (j == it.w - 1) umma_commit(B.q_empty);
-          ++kc;
-          if (j > 0 && !issue_pv(tg - 1, j == 1, false)) {
-            ok = false;
-            break;
-          }
-          ++tg;
         }
         if (!ok) break;
-        if (!issue_pv(tg - 1, it.w == 1, true)) break;
+        kc += n;
+        for (int x = 0; x < 2; ++x)
+          if (started[x]) ++uhc[x];
         ++uc;
       }
       if (!ok || abort_flag) {
-        // wait (bounded) for every MMA already issued before TMEM is freed
-        uint64_t* drain = B.o_free;  // reuse: arrive count is irrelevant for a commit
-        (void)drain;
+        // give MMAs already issued time to finish before TMEM is freed
         const uint64_t t0 = globaltimer();
         while (globaltimer() - t0 < 1000000ull) {
         }
       }
     }
-  } else if (warp >= kSoftmaxWarp0) {
+  } else if (warp >= 4) {
     // ================================================================ softmax + epilogue
-    const int quarter = warp - kSoftmaxWarp0;
-    const int r = quarter * 32 + lane;  // row within the Q tile = TMEM lane
-    const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
-    uint32_t tg = 0, uc = 0;
+    const int x = (warp - 4) >> 2;      // half
+    const int quarter = warp & 3;       // TMEM lane quarter
+    const int r = quarter * 32 + lane;  // row within the half
+    const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16) + x * 256;
+    const uint32_t tS = trow, tO = trow + 128;
+    uint32_t sc_count = 0;  // S tiles of this half consumed (all units)
     bool ok = true;
     for (uint32_t i = 0; ok; ++i) {
       const int slot_s = i % kSchedSlots;
@@ -329,185 +384,140 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (u >= units) break;
       const int4 it = __ldg(items + u / p.Hq);
       const int h = u % p.Hq;
-      const int q = it.x + r;
-      const bool valid = r < it.y;
-      if (it.w == 0) {
-        if (valid) {
-          if (p.out_f32) {
-            float* dst = static_cast<float*>(p.o) + (size_t(q) * p.Hq + h) * D;
-            for (int c = 0; c < D; ++c) dst[c] = 0.f;
-          } else {
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) + (size_t(q) * p.Hq + h) * D;
-            for (int c = 0; c < D; ++c) dst[c] = __float2bfloat16(0.f);
-          }
-          if (p.lse) p.lse[size_t(q) * p.Hq + h] = -INFINITY;
-        }
-        continue;
-      }
+      const int q = it.x + x * BM + r;
+      const bool valid = x * BM + r < it.y;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + (size_t(q) * p.Hq + h) * D;
+
       float m_run = -INFINITY, l_run = 0.f;
+      int nt = 0;  // tiles of this half in this unit
       for (int j = 0; j < it.w; ++j) {
-        const int4 e = __ldg(kvs + it.z + j);  // k0, k_len, rect_begin, rect_count
-        const uint32_t sb = tg & 1;
-        if (!mbar_wait(B.s_full + sb, (tg >> 1) & 1, &abort_flag, p.status)) {
+        const KvEntry e = load_kv(kvs, it.z + j);
+        if (!(e.flags & (1 << x))) continue;
+        if (!mbar_wait(B.s_full + x, sc_count & 1, &abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float s[BN];
-        {
-          uint32_t rr[32];
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            tmem_ld32(trow + (sb ? kSCol1 : kSCol0) + c * 32, rr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[i]);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(B.s_free + sb);
 
-        // visibility of this row inside the tile
-        const bool need_mask = e.w > 0 || e.y < BN;
+        const bool need_mask = !(e.flags & (4 << x)) || e.klen < BN;
         uint32_t vis[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-        if (need_mask) {
-          vis[0] = vis[1] = vis[2] = vis[3] = 0u;
-          if (e.w == 0) {
-            set_bits(vis, 0, e.y);
-          } else {
-            for (int ri = 0; ri < e.w; ++ri) {
-              const int32_t* rc = rects + 5 * (e.z + ri);
-              const int rq0 = __ldg(rc), rq1 = __ldg(rc + 1), rk0 = __ldg(rc + 2),
-                        rk1 = __ldg(rc + 3), causal = __ldg(rc + 4);
-              if (q < rq0 || q >= rq1) continue;
-              int hi = causal ? min(rk1, rk0 + (q - rq0) + 1) : rk1;
-              hi = min(hi, e.x + e.y);
-              const int lo = max(rk0, e.x);
-              if (lo < hi) set_bits(vis, lo - e.x, hi - e.x);
-            }
-          }
-        }
-        // raw logits stay unscaled (scale > 0 commutes with max); masked
-        // entries become -inf.  Eight independent max chains.
-        if (need_mask) {
-#pragma unroll
-          for (int i = 0; i < BN; ++i)
-            s[i] = ((vis[i >> 5] >> (i & 31)) & 1u) ? s[i] : -INFINITY;
-        }
+        if (need_mask) row_visibility(e, x, q, rects, vis);
+
+        // pass 1: row max of the raw logits (scale > 0 commutes with max)
         float mx8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+        for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
-        for (int i = 8; i < BN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tS + c * 32, rr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            float v = __uint_as_float(rr[k]);
+            if (need_mask) v = ((vis[c] >> k) & 1u) ? v : -INFINITY;
+            mx8[k & 7] = fmaxf(mx8[k & 7], v);
+          }
+        }
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
                          p.scale_log2;
         const float m_new = fmaxf(m_run, mx);
         const bool resc = m_new > m_run + kRescaleLog2;
-        if (__any_sync(0xffffffffu, resc) && j > 0) {
-          // O holds PV of earlier tiles: wait for the latest, rescale in TMEM
-          const uint32_t tp = tg - 1;
-          if (!mbar_wait(B.p_free + (tp & 1), (tp >> 1) & 1, &abort_flag, p.status)) {
+        if (__any_sync(0xffffffffu, resc) && nt > 0) {
+          // O holds the PVs of earlier tiles: wait for the latest, rescale
+          if (!mbar_wait(B.pv_done + x, (sc_count - 1) & 1, &abort_flag, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const float alpha = resc ? fast_exp2(m_run - m_new) : 1.f;
-          uint32_t rr[32];
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
-            tmem_ld32(trow + kOCol + c * 32, rr);
+            uint32_t rr[32];
+            tmem_ld32(tO + c * 32, rr);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-            tmem_st32(trow + kOCol + c * 32, rr);
+            for (int k = 0; k < 32; ++k) rr[k] = __float_as_uint(__uint_as_float(rr[k]) * alpha);
+            tmem_st32(tO + c * 32, rr);
           }
-          tmem_wait_st();
         }
         if (resc) {
           l_run *= fast_exp2(m_run - m_new);
           m_run = m_new;
         }
-        const float m_use = m_run == -INFINITY ? 0.f : m_run;
+        const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
 
-        // P buffer sb is free once the PV two tiles back has completed
-        if (!mbar_wait(B.p_free + sb, ((tg >> 1) & 1) ^ 1, &abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        const uint32_t prow = sP + sb * C::P_BYTES + r * 128;
-        const float sc = p.scale_log2, neg_m = -m_use;
+        // pass 2: P = exp2(s * scale - m) as bf16 over S columns already read
+        const float sc = p.scale_log2;
         float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < BN / 8; ++c) {
-          uint32_t w[4];
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tS + c * 32, rr);
+          tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float p0 = fast_exp2(fmaf(s[c * 8 + 2 * k], sc, neg_m));
-            const float p1 = fast_exp2(fmaf(s[c * 8 + 2 * k + 1], sc, neg_m));
-            ls8[2 * k] += p0;
-            ls8[2 * k + 1] += p1;
-            w[k] = pack_bf16(p0, p1);
+          for (int k = 0; k < 16; ++k) {
+            float v0 = __uint_as_float(rr[2 * k]), v1 = __uint_as_float(rr[2 * k + 1]);
+            if (need_mask) {
+              v0 = ((vis[c] >> (2 * k)) & 1u) ? v0 : -INFINITY;
+              v1 = ((vis[c] >> (2 * k + 1)) & 1u) ? v1 : -INFINITY;
+            }
+            const float p0 = fast_exp2(fmaf(v0, sc, neg_m));
+            const float p1 = fast_exp2(fmaf(v1, sc, neg_m));
+            ls8[(2 * k) & 7] += p0;
+            ls8[(2 * k + 1) & 7] += p1;
+            pk[k] = pack_bf16(p0, p1);
           }
-          const uint32_t addr = prow + (c >> 3) * (BM * 128) + (((c & 7) ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w[0]),
-                       "r"(w[1]), "r"(w[2]), "r"(w[3])
-                       : "memory");
+          tmem_st16(tS + c * 16, pk);
         }
-        const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) +
-                           ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-        l_run += lsum;
-        fence_proxy_async_smem();
+        l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(B.p_full + sb);
-        ++tg;
+        if (lane == 0) mbar_arrive(B.p_full + x);
+        ++sc_count;
+        ++nt;
       }
       if (!ok) break;
 
+      if (nt == 0) {
+        // this half sees nothing in the block (rows past the group end)
+        if (valid) {
+          for (int c = 0; c < D; ++c) orow[c] = __float2bfloat16(0.f);
+          if (p.lse) p.lse[size_t(q) * p.Hq + h] = -INFINITY;
+        }
+        continue;
+      }
       // ---- epilogue: O / l straight from TMEM, LSE
-      if (!mbar_wait(B.o_full, uc & 1, &abort_flag, p.status)) break;
+      if (!mbar_wait(B.pv_done + x, (sc_count - 1) & 1, &abort_flag, p.status)) break;
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      uint32_t rr[32];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        tmem_ld32(trow + kOCol + c * 32, rr);
+        uint32_t rr[32];
+        tmem_ld32(tO + c * 32, rr);
         tmem_wait_ld();
         if (valid) {
-          if (p.out_f32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) +
-                                                    (size_t(q) * p.Hq + h) * D + c * 32);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              dst[k] = make_float4(__uint_as_float(rr[4 * k]) * inv,
-                                   __uint_as_float(rr[4 * k + 1]) * inv,
-                                   __uint_as_float(rr[4 * k + 2]) * inv,
-                                   __uint_as_float(rr[4 * k + 3]) * inv);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
-                                                  (size_t(q) * p.Hq + h) * D + c * 32);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              dst[k] = make_uint4(
-                  pack_bf16(__uint_as_float(rr[8 * k]) * inv, __uint_as_float(rr[8 * k + 1]) * inv),
-                  pack_bf16(__uint_as_float(rr[8 * k + 2]) * inv,
-                            __uint_as_float(rr[8 * k + 3]) * inv),
-                  pack_bf16(__uint_as_float(rr[8 * k + 4]) * inv,
-                            __uint_as_float(rr[8 * k + 5]) * inv),
-                  pack_bf16(__uint_as_float(rr[8 * k + 6]) * inv,
-                            __uint_as_float(rr[8 * k + 7]) * inv));
-          }
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_uint4(
+                pack_bf16(__uint_as_float(rr[8 * k]) * inv, __uint_as_float(rr[8 * k + 1]) * inv),
+                pack_bf16(__uint_as_float(rr[8 * k + 2]) * inv,
+                          __uint_as_float(rr[8 * k + 3]) * inv),
+                pack_bf16(__uint_as_float(rr[8 * k + 4]) * inv,
+                          __uint_as_float(rr[8 * k + 5]) * inv),
+                pack_bf16(__uint_as_float(rr[8 * k + 6]) * inv,
+                          __uint_as_float(rr[8 * k + 7]) * inv));
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(B.o_free);
+      if (lane == 0) mbar_arrive(B.o_free + x);
       if (valid && p.lse)
-        p.lse[size_t(q) * p.Hq + h] =
-            l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
-      ++uc;
+        p.lse[size_t(q) * p.Hq + h] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
     }
   }
 
@@ -518,36 +528,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// fp32 I/O path: the same schedule and visibility, fp32 CUDA-core
+// arithmetic throughout (no rounding of the fp32 inputs).  One warp per
+// (query row, head); lanes split the head dimension.  It serves small fp32
+// problems; the bf16 tensor-core kernel above is the throughput path.
 template <int D>
 __global__ void __launch_bounds__(256) prefill_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
     float* __restrict__ o, float* __restrict__ lse, const int32_t* __restrict__ sch,
     int64_t sched_len, int32_t Hq, int32_t G, float scale_log2, int32_t* status) {
   constexpr int E = D / 32;
-  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2), n_rect = __ldg(sch + 3);
-  const bool bad = __ldg(sch + 0) != 0x50534131 || __ldg(sch + 4) != BM ||
-                   __ldg(sch + 5) != BN || n_items < 0 || n_kv < 0 || n_rect < 0 ||
-                   8 + 4 * int64_t(n_items) + 4 * int64_t(n_kv) + 5 * int64_t(n_rect) >
-                       sched_len;
-  if (bad) {
+  if (!schedule_ok(sch, sched_len)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) report_status(status, PSA_ERR_INVALID_ARG);
     return;
   }
+  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2);
   const int4* items = reinterpret_cast<const int4*>(sch + 8);
-  const int4* kvs = reinterpret_cast<const int4*>(sch + 8 + 4 * n_items);
-  const int32_t* rects = sch + 8 + 4 * n_items + 4 * n_kv;
+  const int32_t* kvs = sch + 8 + 4 * n_items;
+  const int32_t* rects = kvs + 8 * n_kv;
   const int lane = threadIdx.x & 31;
-  const int64_t total = int64_t(n_items) * BM * Hq;
+  const int64_t total = int64_t(n_items) * BLOCK_M * Hq;
   const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  const int Hkv = Hq / G;
   for (int64_t u = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; u < total;
        u += nwarps) {
-    const int item = int(u / (int64_t(BM) * Hq));
-    const int rem = int(u % (int64_t(BM) * Hq));
+    const int item = int(u / (int64_t(BLOCK_M) * Hq));
+    const int rem = int(u % (int64_t(BLOCK_M) * Hq));
     const int r = rem / Hq, h = rem % Hq;
     const int4 it = __ldg(items + item);
     if (r >= it.y) continue;
+    const int x = r / BM;
     const int qi = it.x + r, kvh = h / G;
-    const int Hkv = Hq / G;
     float qv[E], acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -556,16 +567,14 @@ __global__ void __launch_bounds__(256) prefill_f32_kernel(
     }
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < it.w; ++j) {
-      const int4 ent = __ldg(kvs + it.z + j);
-      for (int kk = ent.x; kk < ent.x + ent.y; ++kk) {
-        bool on = ent.w == 0;
-        for (int ri = 0; ri < ent.w && !on; ++ri) {
-          const int32_t* rc = rects + 5 * (ent.z + ri);
-          const int rq0 = rc[0], rq1 = rc[1], rk0 = rc[2], rk1 = rc[3], causal = rc[4];
-          on = qi >= rq0 && qi < rq1 && kk >= rk0 && kk < rk1 && (!causal || kk - rk0 <= qi - rq0);
-        }
-        if (!on) continue;
-        const float* kr = k + (size_t(kk) * Hkv + kvh) * D + lane * E;
+      const KvEntry ent = load_kv(kvs, it.z + j);
+      if (!(ent.flags & (1 << x))) continue;
+      uint32_t vis[4];
+      row_visibility(ent, x, qi, rects, vis);
+      for (int kk = 0; kk < ent.klen; ++kk) {
+        if (!((vis[kk >> 5] >> (kk & 31)) & 1u)) continue;
+        const int key = ent.k0 + kk;
+        const float* kr = k + (size_t(key) * Hkv + kvh) * D + lane * E;
         float d = 0.f;
 #pragma unroll
         for (int e = 0; e < E; ++e) d = fmaf(qv[e], kr[e], d);
@@ -576,7 +585,7 @@ __global__ void __launch_bounds__(256) prefill_f32_kernel(
         const float alpha = exp2f(m - mn);
         const float pe = exp2f(sv - mn);
         l = l * alpha + pe;
-        const float* vr = v + (size_t(kk) * Hkv + kvh) * D + lane * E;
+        const float* vr = v + (size_t(key) * Hkv + kvh) * D + lane * E;
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = fmaf(acc[e], alpha, pe * vr[e]);
         m = mn;
@@ -635,7 +644,6 @@ int launch_prefill_d(const PrefillArgs& a) {
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
   p.G = a.Hq / a.Hkv;
-  p.out_f32 = a.out_f32 ? 1 : 0;
   p.scale_log2 = a.scale * kLog2e;
   p.status = a.status;
   p.counter = a.counter;

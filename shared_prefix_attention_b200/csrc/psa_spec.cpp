@@ -80,11 +80,10 @@ extern "C" int psa_build_spec(const psa_segment* segs, int32_t nseg, psa_rect* o
 }
 
 extern "C" int psa_build_schedule(const psa_rect* rects, int32_t nrect,
-                                  const int32_t* cu_seqlens, int32_t ngroups,
-                                  int32_t tile_m, int32_t tile_n, int32_t* out,
-                                  int64_t cap, int64_t* nout) {
+                                  const int32_t* cu_seqlens, int32_t ngroups, int32_t tile_m,
+                                  int32_t tile_n, int32_t* out, int64_t cap, int64_t* nout) {
   if (!nout || nrect < 0 || (nrect > 0 && !rects) || !cu_seqlens || ngroups <= 0 ||
-      tile_m <= 0 || tile_n <= 0)
+      tile_m <= 0 || (tile_m & 1) || tile_n <= 0)
     return PSA_ERR_INVALID_ARG;
   if (cu_seqlens[0] != 0) return PSA_ERR_INVALID_ARG;
   for (int32_t g = 0; g < ngroups; ++g)
@@ -95,22 +94,22 @@ extern "C" int psa_build_schedule(const psa_rect* rects, int32_t nrect,
     if (x.q0 < 0 || x.q1 > T || x.q0 >= x.q1 || x.k0 < 0 || x.k1 > T || x.k0 >= x.k1)
       return PSA_ERR_INVALID_ARG;
   }
+  const int32_t half = tile_m / 2;
 
   struct Item {
     int32_t q0, qlen, kv_begin, kv_count;
   };
   struct Kv {
-    int32_t k0, klen, rect_begin, rect_count;
+    int32_t k0, klen, rb[2], rc[2], flags;
   };
   std::vector<Item> items;
   std::vector<Kv> kvs;
   std::vector<psa_rect> trects;
-  std::vector<int32_t> cut;  // rect indices cutting the current box
+  std::vector<int32_t> cut;
   int32_t max_kv = 0;
 
   for (int32_t g = 0; g < ngroups; ++g) {
     const int32_t g0 = cu_seqlens[g], g1 = cu_seqlens[g + 1];
-    // rectangles whose query range lies in this group
     std::vector<int32_t> grect;
     for (int32_t r = 0; r < nrect; ++r)
       if (rects[r].q0 < g1 && rects[r].q1 > g0) grect.push_back(r);
@@ -119,21 +118,30 @@ extern "C" int psa_build_schedule(const psa_rect* rects, int32_t nrect,
       Item it{qa, qb - qa, int32_t(kvs.size()), 0};
       for (int32_t ka = g0; ka < g1; ka += tile_n) {
         const int32_t kb = std::min(g1, ka + tile_n);
-        int64_t vis = 0;
-        cut.clear();
-        for (int32_t r : grect) {
-          int64_t n = visible_in_box(rects[r], qa, qb, ka, kb);
-          if (n > 0) {
-            vis += n;
-            cut.push_back(r);
+        Kv e{ka, kb - ka, {0, 0}, {0, 0}, 0};
+        for (int h = 0; h < 2; ++h) {
+          const int32_t ha = qa + h * half, hb = std::min(qb, ha + half);
+          if (ha >= hb) continue;  // the block has no second half
+          int64_t vis = 0;
+          cut.clear();
+          for (int32_t r : grect) {
+            const int64_t n = visible_in_box(rects[r], ha, hb, ka, kb);
+            if (n > 0) {
+              vis += n;
+              cut.push_back(r);
+            }
+          }
+          if (vis == 0) continue;
+          e.flags |= 1 << h;  // this half has visible pairs in the tile
+          if (vis == int64_t(hb - ha) * (kb - ka)) {
+            e.flags |= 4 << h;  // ... and all of them are visible
+          } else {
+            e.rb[h] = int32_t(trects.size());
+            e.rc[h] = int32_t(cut.size());
+            for (int32_t r : cut) trects.push_back(rects[r]);
           }
         }
-        if (vis == 0) continue;
-        Kv e{ka, kb - ka, int32_t(trects.size()), 0};
-        if (vis < int64_t(qb - qa) * (kb - ka)) {
-          for (int32_t r : cut) trects.push_back(rects[r]);
-          e.rect_count = int32_t(cut.size());
-        }
+        if (!e.flags) continue;
         kvs.push_back(e);
         ++it.kv_count;
       }
@@ -146,12 +154,12 @@ extern "C" int psa_build_schedule(const psa_rect* rects, int32_t nrect,
     return a.kv_count > b.kv_count;
   });
 
-  const int64_t need = 8 + 4 * int64_t(items.size()) + 4 * int64_t(kvs.size()) +
+  const int64_t need = 8 + 4 * int64_t(items.size()) + 8 * int64_t(kvs.size()) +
                        5 * int64_t(trects.size());
   *nout = need;
   if (need > INT32_MAX) return PSA_ERR_INVALID_ARG;
   if (cap < need || !out) return PSA_ERR_CAPACITY;
-  out[0] = 0x50534131;
+  out[0] = 0x50534132;
   out[1] = int32_t(items.size());
   out[2] = int32_t(kvs.size());
   out[3] = int32_t(trects.size());
@@ -169,8 +177,12 @@ extern "C" int psa_build_schedule(const psa_rect* rects, int32_t nrect,
   for (const Kv& e : kvs) {
     out[o++] = e.k0;
     out[o++] = e.klen;
-    out[o++] = e.rect_begin;
-    out[o++] = e.rect_count;
+    out[o++] = e.rb[0];
+    out[o++] = e.rc[0];
+    out[o++] = e.rb[1];
+    out[o++] = e.rc[1];
+    out[o++] = e.flags;
+    out[o++] = 0;
   }
   for (const psa_rect& r : trects) {
     out[o++] = r.q0;

@@ -103,7 +103,7 @@ def test_prefill_and_sparse_host_validation():
                                    None, None) == psa.PSA_ERR_UNSUPPORTED
     assert L.psa_sparse_latent_fwd(P(16), P(16), P(16), P(16), None, 4, 8, 64, 512, 0, 0.1,
                                    None, None) == psa.PSA_ERR_INVALID_ARG
-    assert psa.prefill_tiles(128) == (128, 128)
+    assert psa.prefill_tiles(128) == (256, 128)
     with pytest.raises(psa.PsaError):
         psa.prefill_tiles(80)
 

@@ -85,16 +85,19 @@ def test_spec_rejects_bad_trees():
 
 
 def _decode(sched):
-    assert sched[0] == 0x50534131
+    assert sched[0] == 0x50534132
     ni, nk, nr, tm, tn, T, maxkv = (int(x) for x in sched[1:8])
     items = sched[8:8 + 4 * ni].reshape(ni, 4)
-    kvs = sched[8 + 4 * ni:8 + 4 * (ni + nk)].reshape(nk, 4)
-    rects = sched[8 + 4 * (ni + nk):8 + 4 * (ni + nk) + 5 * nr].reshape(nr, 5)
-    assert len(sched) == 8 + 4 * (ni + nk) + 5 * nr
+    kvs = sched[8 + 4 * ni:8 + 4 * ni + 8 * nk].reshape(nk, 8)
+    rects = sched[8 + 4 * ni + 8 * nk:8 + 4 * ni + 8 * nk + 5 * nr].reshape(nr, 5)
+    assert len(sched) == 8 + 4 * ni + 8 * nk + 5 * nr
     return items, kvs, rects, tm, tn, T, maxkv
 
 
 def _check_schedule(segs, cu, tm, tn):
+    """Every Q block (two halves of tm/2 rows) lists exactly the KV tiles in
+    which some half has a visible pair; per half the active / full flags
+    and the copied rectangles reproduce the visibility of the box."""
     rects = psa.build_spec(segs)
     sched = psa.build_schedule(rects, cu, tm, tn)
     items, kvs, trects, tm2, tn2, T, maxkv = _decode(sched)
@@ -103,30 +106,41 @@ def _check_schedule(segs, cu, tm, tn):
     counts = [int(it[3]) for it in items]
     assert counts == sorted(counts, reverse=True)          # longest first
     assert maxkv == max(counts)
+    half = tm // 2
     covered = np.zeros_like(vis)
     seen_q = []
     for q0, ql, kb, kc in items:
-        seen_q.append((q0, ql))
-        # every KV tile of the group with a visible pair is listed exactly once
+        seen_q.append((int(q0), int(ql)))
         g = max(i for i in range(len(cu) - 1) if cu[i] <= q0)
-        listed = {}
-        for e in kvs[kb:kb + kc]:
-            listed[int(e[0])] = e
+        listed = {int(e[0]): e for e in kvs[kb:kb + kc]}
+        assert len(listed) == kc
         for ka in range(cu[g], cu[g + 1], tn):
             kl = min(cu[g + 1], ka + tn) - ka
-            box = vis[q0:q0 + ql, ka:ka + kl]
-            if not box.any():
+            boxes = []
+            for h in range(2):
+                a, b = q0 + h * half, min(q0 + ql, q0 + (h + 1) * half)
+                boxes.append(vis[a:b, ka:ka + kl] if a < b else np.zeros((0, kl), bool))
+            if not any(bx.any() for bx in boxes):
                 assert ka not in listed
                 continue
             e = listed[ka]
             assert int(e[1]) == kl
-            if box.all():
-                assert int(e[3]) == 0
-            else:
-                assert int(e[3]) > 0
-                sub = _expand(trects[e[2]:e[2] + e[3]], T)[q0:q0 + ql, ka:ka + kl]
-                assert np.array_equal(sub.astype(bool), box)
-            covered[q0:q0 + ql, ka:ka + kl] = True
+            flags = int(e[6])
+            for h in range(2):
+                bx = boxes[h]
+                active = bool(bx.any())
+                assert bool(flags & (1 << h)) == active
+                if not active:
+                    continue
+                full = bool(bx.all())
+                assert bool(flags & (4 << h)) == full
+                if not full:
+                    rb, rc = int(e[2 + 2 * h]), int(e[3 + 2 * h])
+                    assert rc > 0
+                    a = q0 + h * half
+                    sub = _expand(trects[rb:rb + rc], T)[a:a + bx.shape[0], ka:ka + kl]
+                    assert np.array_equal(sub.astype(bool), bx)
+                covered[q0 + h * half:q0 + h * half + bx.shape[0], ka:ka + kl] = True
     assert sorted(seen_q) == sorted(
         (a, min(cu[i + 1], a + tm) - a) for i in range(len(cu) - 1)
         for a in range(cu[i], cu[i + 1], tm))
@@ -134,8 +148,8 @@ def _check_schedule(segs, cu, tm, tn):
 
 
 @pytest.mark.parametrize("P,N,S,groups,tm,tn", [
-    (64, 4, 32, 1, 128, 128), (2048, 8, 512, 1, 128, 128), (100, 3, 37, 2, 128, 128),
-    (5, 7, 3, 1, 8, 4), (0, 4, 50, 1, 32, 16), (300, 2, 1, 3, 128, 64)])
+    (64, 4, 32, 1, 256, 128), (2048, 8, 512, 1, 256, 128), (100, 3, 37, 2, 256, 128),
+    (5, 7, 3, 1, 8, 4), (0, 4, 50, 1, 32, 16), (300, 2, 1, 3, 128, 64), (700, 3, 300, 1, 256, 128)])
 def test_schedule_tiles(P, N, S, groups, tm, tn):
     wl = W.PrefillWorkload("t", P=P, N=N, S=S, Hq=1, Hkv=1, d=64, groups=groups)
     _check_schedule(wl.segments(), wl.cu_seqlens(), tm, tn)
@@ -151,10 +165,11 @@ def test_schedule_random_trees():
 
 def test_schedule_tile_counts_grpo():
     """Visible 128x128 tiles per head: 728 for P=2048/N=8/S=512 (16*17/2 +
-    8 * (4*16 + 10)) and 10848 per group of the two-group P=8192 layout."""
-    rects = psa.build_spec(W.GRPO.segments())
-    sched = psa.build_schedule(rects, W.GRPO.cu_seqlens(), 128, 128)
-    assert int(sched[2]) == 728
-    rects = psa.build_spec(W.LARGE.segments())
-    sched = psa.build_schedule(rects, W.LARGE.cu_seqlens(), 128, 128)
-    assert int(sched[2]) == 2 * 10848   # per group: 64*65/2 + 16 * (8*64 + 36)
+    8 * (4*16 + 10)) and 10848 per group of the two-group P=8192 layout,
+    counted as (half, KV tile) pairs that take part."""
+    for wl, want in ((W.GRPO, 728), (W.LARGE, 2 * 10848)):
+        rects = psa.build_spec(wl.segments())
+        sched = psa.build_schedule(rects, wl.cu_seqlens(), 256, 128)
+        items, kvs, *_ = _decode(sched)
+        active = sum(bin(int(f) & 3).count("1") for f in kvs[:, 6])
+        assert active == want
