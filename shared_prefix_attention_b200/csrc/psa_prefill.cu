@@ -10,16 +10,19 @@
 // the producer hands units out through a global counter, so long suffix
 // blocks start first and short prefix blocks fill the tail.  A block is two
 // 128-row halves A and B that share every K/V tile load:
-//   warp 0       TMA producer: the Q block, then the K and V tiles of the
-//                block's visible KV tiles only (invisible tiles are never
-//                touched), 128-byte swizzle, no multicast.
+//   warps 0, 2   TMA producers (Q and K; V): the Q block, then the K and V
+//                tiles of the block's visible KV tiles only (invisible tiles
+//                are never touched), 128-byte swizzle, no multicast.
 //   warp 1       tcgen05 issuer (one thread).  Per half X: S_X = Q_X K^T
 //                into TMEM, then O_X += P_X V with P_X read from TMEM where
 //                the softmax left it (aliasing S_X).  Issue order
 //                PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1): while one half's
 //                softmax runs, the tensor pipe works on the other half.
 //   warps 4..7   softmax of half A, warps 8..11 softmax of half B: one query
-//                row per thread (= TMEM lane).  Masks partial tiles from the
+//                row per thread (= TMEM lane), the whole 128-column S row
+//                read in one TMEM load (setmaxnreg moves registers from the
+//                producer/MMA warpgroup to the softmax warpgroups).  Masks
+//                partial tiles from the
 //                copied rectangles, keeps the running max in the log2 domain
 //                with lazy rescaling (O is rescaled in TMEM only when the
 //                max grows by more than 2^8), writes P as bf16 over its S
@@ -31,6 +34,7 @@
 
 #include "psa_device.cuh"
 #include "psa_internal.h"
+#include "psa_tmem_wide.cuh"
 
 namespace psa {
 namespace {
@@ -42,19 +46,22 @@ constexpr int kThreads = 384;      // 12 warps
 constexpr float kRescaleLog2 = 8.f;
 constexpr uint32_t kTmemCols = 512;  // per half: S at X*256, O at X*256 + 128
 constexpr int kSchedSlots = 4;       // units the producer may fetch ahead
-constexpr int kSchedReaders = 9;     // the MMA thread and the eight softmax warps
+constexpr int kSchedReaders = 10;    // V producer, MMA thread, eight softmax warps
 
 template <int D>
 struct Cfg {
   static constexpr int NPART = D / 64;  // 128-byte swizzle atoms across d
   static constexpr uint32_t Q_BYTES = BM * D * 2;   // one half
   static constexpr uint32_t KV_BYTES = BN * D * 2;
-  static constexpr int NS = D == 128 ? 2 : 4;       // K and V ring slots
+  // K is needed a whole tile before V (QK_{j+1} is issued right after
+  // PV_j), so its ring is one slot deeper.
+  static constexpr int NSK = D == 128 ? 3 : 4;
+  static constexpr int NSV = D == 128 ? 2 : 4;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + 2 * Q_BYTES;
-  static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + NS * KV_BYTES;
-  static constexpr uint32_t NBAR = 2 + 4 * NS + 8 + 2 * kSchedSlots;
+  static constexpr uint32_t OFF_V = OFF_K + NSK * KV_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + NSV * KV_BYTES;
+  static constexpr uint32_t NBAR = 2 + 2 * NSK + 2 * NSV + 8 + 2 * kSchedSlots;
   static constexpr uint32_t SMEM = 1024 + OFF_BAR + NBAR * 8 + 16;
 };
 
@@ -85,6 +92,17 @@ __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int a, int b) {
       m[w] |= bits << (lo - 32 * w);
     }
   }
+}
+
+// Register split between warpgroups: the launch gives every thread 168
+// registers (384 x 168 = 64512); warpgroup 0 (the two producers, the MMA
+// issuer, one idle warp) drops to 72 so the two softmax warpgroups can hold
+// a whole 128-column S row in registers (2 x 128 x 208 + 128 x 72 = 62464).
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 72;" ::: "memory");
+}
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
 }
 
 // Header check shared by both prefill kernels (uniform across threads).
@@ -164,10 +182,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.q_full = bar + 0;
   B.q_empty = bar + 1;
   B.k_full = bar + 2;
-  B.k_empty = B.k_full + C::NS;
-  B.v_full = B.k_empty + C::NS;
-  B.v_empty = B.v_full + C::NS;
-  B.s_full = B.v_empty + C::NS;
+  B.k_empty = B.k_full + C::NSK;
+  B.v_full = B.k_empty + C::NSK;
+  B.v_empty = B.v_full + C::NSV;
+  B.s_full = B.v_empty + C::NSV;
   B.p_full = B.s_full + 2;
   B.pv_done = B.p_full + 2;
   B.o_free = B.pv_done + 2;
@@ -178,9 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     abort_flag = 0;
     mbar_init(B.q_full, 1);
     mbar_init(B.q_empty, 1);
-    for (int i = 0; i < C::NS; ++i) {
+    for (int i = 0; i < C::NSK; ++i) {
       mbar_init(B.k_full + i, 1);
       mbar_init(B.k_empty + i, 1);
+    }
+    for (int i = 0; i < C::NSV; ++i) {
       mbar_init(B.v_full + i, 1);
       mbar_init(B.v_empty + i, 1);
     }
@@ -205,56 +225,67 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_slot;
 
-  if (warp == 0) {
-    // ================================================================ producer
+  if (warp < 4) {
+    regs_dec();
+    if (warp == 0 || warp == 2) {
+    // ================================================================ producers
+    // warp 0 fetches units and loads Q and K; warp 2 loads V.  The two rings
+    // advance independently, so a K load never waits behind a V slot.
     if (lane == 0) {
-      tma_prefetch_desc(&tmap_q);
-      tma_prefetch_desc(&tmap_k);
-      tma_prefetch_desc(&tmap_v);
+      const bool kprod = warp == 0;
+      if (kprod) {
+        tma_prefetch_desc(&tmap_q);
+        tma_prefetch_desc(&tmap_k);
+      } else {
+        tma_prefetch_desc(&tmap_v);
+      }
       uint32_t kc = 0, uc = 0;
       bool ok = true;
       for (uint32_t i = 0; ok; ++i) {
         const int slot_s = i % kSchedSlots;
-        if (!mbar_wait(B.sch_empty + slot_s, ((i / kSchedSlots) & 1) ^ 1, &abort_flag,
-                       p.status))
-          break;
-        const int u = atomicAdd(p.counter, 1);
-        sch_unit[slot_s] = u;
-        mbar_arrive(B.sch_full + slot_s);
+        const uint32_t sph = (i / kSchedSlots) & 1;
+        int u;
+        if (kprod) {
+          if (!mbar_wait(B.sch_empty + slot_s, sph ^ 1, &abort_flag, p.status)) break;
+          u = atomicAdd(p.counter, 1);
+          sch_unit[slot_s] = u;
+          mbar_arrive(B.sch_full + slot_s);
+        } else {
+          if (!mbar_wait(B.sch_full + slot_s, sph, &abort_flag, p.status)) break;
+          u = sch_unit[slot_s];
+          mbar_arrive(B.sch_empty + slot_s);
+        }
         if (u >= units) break;
         const int4 it = __ldg(items + u / p.Hq);
         const int h = u % p.Hq, kvh = h / p.G;
         if (it.w == 0) continue;
-        if (!mbar_wait(B.q_empty, (uc & 1) ^ 1, &abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(B.q_full, 2 * C::Q_BYTES);
+        if (kprod) {
+          if (!mbar_wait(B.q_empty, (uc & 1) ^ 1, &abort_flag, p.status)) break;
+          mbar_arrive_expect_tx(B.q_full, 2 * C::Q_BYTES);
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
+          for (int x = 0; x < 2; ++x)
 #pragma unroll
-          for (int part = 0; part < C::NPART; ++part)
-            tma_load_3d(smem + C::OFF_Q + x * C::Q_BYTES + part * BM * 128, &tmap_q, B.q_full,
-                        part * 64, h, it.x + x * BM);
+            for (int part = 0; part < C::NPART; ++part)
+              tma_load_3d(smem + C::OFF_Q + x * C::Q_BYTES + part * BM * 128, &tmap_q,
+                          B.q_full, part * 64, h, it.x + x * BM);
+        }
         for (int j = 0; j < it.w; ++j) {
           const int k0 = __ldg(kvs + 8 * (it.z + j));
-          const int slot = kc % C::NS;
-          const uint32_t ph = (kc / C::NS) & 1;
-          if (!mbar_wait(B.k_empty + slot, ph ^ 1, &abort_flag, p.status)) {
+          const int ns = kprod ? C::NSK : C::NSV;
+          const int slot = kc % ns;
+          const uint32_t ph = (kc / ns) & 1;
+          uint64_t* empty = kprod ? B.k_empty : B.v_empty;
+          uint64_t* full = kprod ? B.k_full : B.v_full;
+          if (!mbar_wait(empty + slot, ph ^ 1, &abort_flag, p.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(B.k_full + slot, C::KV_BYTES);
+          mbar_arrive_expect_tx(full + slot, C::KV_BYTES);
+          uint8_t* dst = smem + (kprod ? C::OFF_K : C::OFF_V) + slot * C::KV_BYTES;
+          const CUtensorMap* tm = kprod ? &tmap_k : &tmap_v;
 #pragma unroll
           for (int part = 0; part < C::NPART; ++part)
-            tma_load_3d(smem + C::OFF_K + slot * C::KV_BYTES + part * BN * 128, &tmap_k,
-                        B.k_full + slot, part * 64, kvh, k0);
-          if (!mbar_wait(B.v_empty + slot, ph ^ 1, &abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(B.v_full + slot, C::KV_BYTES);
-#pragma unroll
-          for (int part = 0; part < C::NPART; ++part)
-            tma_load_3d(smem + C::OFF_V + slot * C::KV_BYTES + part * BN * 128, &tmap_v,
-                        B.v_full + slot, part * 64, kvh, k0);
+            tma_load_3d(dst + part * BN * 128, tm, full + slot, part * 64, kvh, k0);
           ++kc;
         }
         ++uc;
@@ -266,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+    } else if (warp == 1) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = umma_idesc_bf16(BM, BN, false, false);
@@ -281,8 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // S_X = Q_X K_t^T into the S columns of half x
       auto issue_qk = [&](int x, uint32_t t_glob) -> bool {
-        const int slot = t_glob % C::NS;
-        if (!mbar_wait(B.k_full + slot, (t_glob / C::NS) & 1, &abort_flag, p.status))
+        const int slot = t_glob % C::NSK;
+        if (!mbar_wait(B.k_full + slot, (t_glob / C::NSK) & 1, &abort_flag, p.status))
           return false;
         tc_fence_after();
         const uint32_t qbase = sQ + x * C::Q_BYTES, kbase = sK + slot * C::KV_BYTES;
@@ -298,8 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_X += P_X V_t, P_X in TMEM over the first 64 columns of S_X
       auto issue_pv = [&](int x, uint32_t t_glob, bool first) -> bool {
         if (!mbar_wait(B.p_full + x, pvc[x] & 1, &abort_flag, p.status)) return false;
-        const int slot = t_glob % C::NS;
-        if (!mbar_wait(B.v_full + slot, (t_glob / C::NS) & 1, &abort_flag, p.status))
+        const int slot = t_glob % C::NSV;
+        if (!mbar_wait(B.v_full + slot, (t_glob / C::NSV) & 1, &abort_flag, p.status))
           return false;
         if (first && !mbar_wait(B.o_free + x, (uhc[x] & 1) ^ 1, &abort_flag, p.status))
           return false;
@@ -332,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int x = 0; x < 2 && ok; ++x)
             if (f & (1 << x)) ok = issue_qk(x, kc);
           if (!ok) break;
-          umma_commit(B.k_empty + (kc % C::NS));
+          umma_commit(B.k_empty + (kc % C::NSK));
           if (n == 1) umma_commit(B.q_empty);
         }
         for (int j = 0; j < n && ok; ++j) {
@@ -347,9 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok && (fn & (1 << x))) ok = issue_qk(x, t + 1);
           }
           if (!ok) break;
-          umma_commit(B.v_empty + (t % C::NS));
+          umma_commit(B.v_empty + (t % C::NSV));
           if (j + 1 < n) {
-            umma_commit(B.k_empty + ((t + 1) % C::NS));
+            umma_commit(B.k_empty + ((t + 1) % C::NSK));
             if (j + 2 == n) umma_commit(B.q_empty);
           }
         }
@@ -366,7 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp >= 4) {
+    }
+  } else {
+    regs_inc();
     // ================================================================ softmax + epilogue
     const int x = (warp - 4) >> 2;      // half
     const int quarter = warp & 3;       // TMEM lane quarter
@@ -403,22 +436,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t vis[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         if (need_mask) row_visibility(e, x, q, rects, vis);
 
-        // pass 1: row max of the raw logits (scale > 0 commutes with max)
+        // the whole S row in one TMEM load
+        uint32_t sr[BN];
+        tmem_ld128(tS, sr);
+        tmem_wait_ld();
+        if (need_mask) {
+#pragma unroll
+          for (int k = 0; k < BN; ++k)
+            if (!((vis[k >> 5] >> (k & 31)) & 1u)) sr[k] = __float_as_uint(-INFINITY);
+        }
+        // row max of the raw logits (scale > 0 commutes with max)
         float mx8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+        for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[k]);
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(tS + c * 32, rr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            float v = __uint_as_float(rr[k]);
-            if (need_mask) v = ((vis[c] >> k) & 1u) ? v : -INFINITY;
-            mx8[k & 7] = fmaxf(mx8[k & 7], v);
-          }
-        }
+        for (int k = 8; k < BN; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(sr[k]));
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) *
                          p.scale_log2;
@@ -448,30 +480,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
 
-        // pass 2: P = exp2(s * scale - m) as bf16 over S columns already read
+        // P = exp2(s * scale - m) as bf16, written over the S columns
         const float sc = p.scale_log2;
         float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // packed pairs go into the registers just consumed (k <= 2k)
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(tS + c * 32, rr);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            float v0 = __uint_as_float(rr[2 * k]), v1 = __uint_as_float(rr[2 * k + 1]);
-            if (need_mask) {
-              v0 = ((vis[c] >> (2 * k)) & 1u) ? v0 : -INFINITY;
-              v1 = ((vis[c] >> (2 * k + 1)) & 1u) ? v1 : -INFINITY;
-            }
-            const float p0 = fast_exp2(fmaf(v0, sc, neg_m));
-            const float p1 = fast_exp2(fmaf(v1, sc, neg_m));
-            ls8[(2 * k) & 7] += p0;
-            ls8[(2 * k + 1) & 7] += p1;
-            pk[k] = pack_bf16(p0, p1);
-          }
-          tmem_st16(tS + c * 16, pk);
+        for (int k = 0; k < BN / 2; ++k) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * k]), sc, neg_m));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * k + 1]), sc, neg_m));
+          ls8[(2 * k) & 7] += p0;
+          ls8[(2 * k + 1) & 7] += p1;
+          sr[k] = pack_bf16(p0, p1);
         }
+        tmem_st64(tS, *reinterpret_cast<uint32_t(*)[BN / 2]>(sr));
         l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
         tmem_wait_st();
         tc_fence_before();
@@ -494,23 +515,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(B.pv_done + x, (sc_count - 1) & 1, &abort_flag, p.status)) break;
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tO + c * 32, rr);
+      {
+        uint32_t orr[D];
+        if constexpr (D == 128) {
+          tmem_ld128(tO, orr);
+        } else {
+          tmem_ld64(tO, orr);
+        }
         tmem_wait_ld();
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
+          for (int k = 0; k < D / 8; ++k)
             dst[k] = make_uint4(
-                pack_bf16(__uint_as_float(rr[8 * k]) * inv, __uint_as_float(rr[8 * k + 1]) * inv),
-                pack_bf16(__uint_as_float(rr[8 * k + 2]) * inv,
-                          __uint_as_float(rr[8 * k + 3]) * inv),
-                pack_bf16(__uint_as_float(rr[8 * k + 4]) * inv,
-                          __uint_as_float(rr[8 * k + 5]) * inv),
-                pack_bf16(__uint_as_float(rr[8 * k + 6]) * inv,
-                          __uint_as_float(rr[8 * k + 7]) * inv));
+                pack_bf16(__uint_as_float(orr[8 * k]) * inv, __uint_as_float(orr[8 * k + 1]) * inv),
+                pack_bf16(__uint_as_float(orr[8 * k + 2]) * inv,
+                          __uint_as_float(orr[8 * k + 3]) * inv),
+                pack_bf16(__uint_as_float(orr[8 * k + 4]) * inv,
+                          __uint_as_float(orr[8 * k + 5]) * inv),
+                pack_bf16(__uint_as_float(orr[8 * k + 6]) * inv,
+                          __uint_as_float(orr[8 * k + 7]) * inv));
         }
       }
       tc_fence_before();
