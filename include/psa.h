@@ -256,10 +256,12 @@ int psa_verify_fwd_noalloc(const void *q_draft, const void *k_draft, const void 
  *   q       device [T, H, dl] bf16     queries, all heads of a token together
  *   latent  device [Tk, dl] bf16       the one shared latent: K = V = latent
  *   idx     device [T, topk] int32     per-query key rows; -1 entries are
- *                                      skipped; others must be in [0, Tk)
+ *                                      skipped; an entry >= Tk is skipped too
+ *                                      and sets PSA_ERR_INVALID_ARG in
+ *                                      dev_status
  *   o       device [T, H, dl] bf16     (written)
  *   lse     device [T, H] fp32         (written; nullable)
- * dl == 512, H <= 128, topk >= 1.  Row t attends to the listed latent rows
+ * dl == 512, H <= 64, topk >= 1.  Row t attends to the listed latent rows
  * only; a row whose list is all -1 gets O = 0 and LSE = -inf.
  */
 int psa_sparse_latent_fwd(const void *q, const void *latent, const int32_t *idx, void *o,

@@ -261,11 +261,26 @@ extern "C" int psa_sparse_latent_fwd(const void* q, const void* latent, const in
                                      int32_t dl, int32_t topk, float scale,
                                      int32_t* dev_status, void* stream) {
   if (T < 0 || Tk <= 0 || H <= 0 || topk <= 0 || !(scale > 0.f)) return PSA_ERR_INVALID_ARG;
-  if (dl != 512 || H > 128) return PSA_ERR_UNSUPPORTED;
+  if (dl != 512 || H > 64) return PSA_ERR_UNSUPPORTED;
   if (T == 0) return PSA_OK;
   if (!q || !latent || !idx || !o) return PSA_ERR_INVALID_ARG;
-  (void)lse;
-  (void)dev_status;
-  (void)stream;
-  return PSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(latent) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(idx) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return PSA_ERR_INVALID_ARG;
+  SparseArgs a;
+  a.q = q;
+  a.latent = latent;
+  a.idx = idx;
+  a.o = o;
+  a.lse = lse;
+  a.T = T;
+  a.Tk = Tk;
+  a.H = H;
+  a.dl = dl;
+  a.topk = topk;
+  a.scale = scale;
+  a.status = dev_status;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_sparse_latent(a);
 }

@@ -74,6 +74,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to `hint_ns` inside the
+// instruction while the phase is incomplete, so a waiting warp does not take
+// issue slots from the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Returns false
 // (after reporting PSA_ERR_TIMEOUT) if that takes longer than the budget or
 // if another thread of the CTA has already flagged an abort.
@@ -82,8 +98,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((it & 15u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > kWaitTimeoutNs) {
         *abort_flag = 1;
@@ -160,6 +176,55 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ---------------------------------------------------------------- paired fp32
+// Blackwell executes these on the FMA pipe two lanes' worth at a time.
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair, on the FMA pipe instead of the MUFU: Cody-Waite style
+// range reduction x = j + f with j = round-to-nearest(x) (the 1.5 * 2^23
+// shifter leaves j in the low mantissa bits), f in [-0.5, 0.5]; 2^f from a
+// degree-3 polynomial whose coefficients were fitted by the Remez exchange
+// algorithm for minimal relative error on [-0.5, 0.5] (max relative error
+// 7.5e-5, below the bf16 rounding the result gets); 2^j is added to the
+// exponent field.  x is clamped to -126 so the exponent never underflows.
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  const uint64_t x = f2_pack(x0, x1);
+  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
+  const uint64_t j = f2_add(t, f2_pack(-kShift, -kShift));
+  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f, f2_pack(0.0551716685295105f, 0.0551716685295105f),
+                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  // (bits(t) << 23) == round(x) << 23 modulo 2^32: the shifter's own bits vanish
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // ---------------------------------------------------------------- tcgen05

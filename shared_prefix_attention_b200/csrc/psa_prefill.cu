@@ -480,18 +480,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
 
-        // P = exp2(s * scale - m) as bf16, written over the S columns
-        const float sc = p.scale_log2;
-        float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        // packed pairs go into the registers just consumed (k <= 2k)
+        // P = exp2(s * scale - m) as bf16, written over the S columns.  On
+        // fully visible tiles 3 of every 8 pairs take the polynomial exp2 on
+        // the FMA pipe so the MUFU is not the bottleneck; partial tiles use
+        // the MUFU only (masked logits are -inf and must give exactly 0).
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(neg_m, neg_m);
+        uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+        if (!need_mask) {
 #pragma unroll
-        for (int k = 0; k < BN / 2; ++k) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * k]), sc, neg_m));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * k + 1]), sc, neg_m));
-          ls8[(2 * k) & 7] += p0;
-          ls8[(2 * k + 1) & 7] += p1;
-          sr[k] = pack_bf16(p0, p1);
+          for (int k = 0; k < BN / 2; ++k) {
+            float x0, x1, p0, p1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])),
+                             sc2, nm2),
+                      x0, x1);
+            if ((k & 7) < 3) {
+              exp2_poly_pair(x0, x1, p0, p1);
+            } else {
+              p0 = fast_exp2(x0);
+              p1 = fast_exp2(x1);
+            }
+            acc2[k & 3] = f2_add(acc2[k & 3], f2_pack(p0, p1));
+            sr[k] = pack_bf16(p0, p1);  // packed pairs go into consumed registers (k <= 2k)
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < BN / 2; ++k) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])),
+                             sc2, nm2),
+                      x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            acc2[k & 3] = f2_add(acc2[k & 3], f2_pack(p0, p1));
+            sr[k] = pack_bf16(p0, p1);
+          }
         }
+        float ls8[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) f2_unpack(acc2[k], ls8[2 * k], ls8[2 * k + 1]);
         tmem_st64(tS, *reinterpret_cast<uint32_t(*)[BN / 2]>(sr));
         l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
         tmem_wait_st();

@@ -1,0 +1,513 @@
+// Shared-latent sparse attention: every query attends to the latent rows its
+// own index list names, and the one 512-wide latent serves as both K and V
+// for all heads ("SM8x sparse-MLA prefill fallback re-reads the shared MLA
+// latent once per head", vLLM issue write-up: environment -- index_topk
+// 2048, 64 heads, kv_lora_rank 512, no rope part; analysis -- the per-head
+// program re-reads the shared latent, and head-blocked 2-D tiles are what
+// make the kernel fast).
+//
+// sm_100a design: one CTA per SM, persistent over queries (heaviest first).
+// All heads of a query share every latent row the CTA gathers, and the
+// gathered rows are used twice -- as K and as V -- from one shared-memory
+// copy.  The products are computed transposed so the key dimension fills
+// the 128 rows of a tcgen05 MMA:
+//   S^T [128 keys x H]   = Lat_tile [128 x 512] . Q_t^T [512 x H]
+//   O^T [512 x H]       += Lat_tile^T [512 x 128] . P^T [128 x H]
+// The latent tile is gathered by cp.async (zero fill for -1 entries) in
+// eight 64-column parts; a part is released for the next tile as soon as
+// the O^T block that reads it has completed.
+//   warps 0..3   gather producers (one key row per thread) and the Q^T load
+//   warp 4       tcgen05 issuer (one thread)
+//   warps 8..11  softmax over keys (one key per thread = TMEM lane) with
+//                per-head max / sum reductions across lanes, P^T written to
+//                shared memory, lazy O^T rescaling, and the epilogue (one
+//                latent dimension per thread and M-block).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "psa_device.cuh"
+#include "psa_internal.h"
+#include "psa_tmem_wide.cuh"
+
+namespace psa {
+namespace {
+
+constexpr int DL = 512;          // latent width
+constexpr int KT = 128;          // keys per tile (MMA M for S^T)
+constexpr int NPART = DL / 64;   // 64-column parts of a latent tile
+constexpr int HMAX = 64;         // heads per CTA pass (MMA N)
+constexpr int kThreads = 384;
+constexpr float kRescaleLog2 = 8.f;
+constexpr uint32_t kTmemCols = 512;  // S^T at 0, O^T M-blocks at 128 + 64 * mb
+
+constexpr uint32_t PART_BYTES = KT * 128;       // 16 KB
+constexpr uint32_t QPART_BYTES = HMAX * 128;    // 8 KB
+constexpr uint32_t OFF_LAT = 0;
+constexpr uint32_t OFF_Q = OFF_LAT + NPART * PART_BYTES;     // 128 KB
+constexpr uint32_t OFF_P = OFF_Q + NPART * QPART_BYTES;      // +64 KB
+constexpr uint32_t OFF_RED = OFF_P + KT * 128;               // +16 KB
+constexpr uint32_t RED_BYTES = 4 * HMAX * 4;                 // [4 warps][64] floats
+constexpr uint32_t OFF_HEAD = OFF_RED + RED_BYTES;           // per-head state
+constexpr uint32_t HEAD_BYTES = 4 * HMAX * 4;                // m, l, alpha, m_tile
+constexpr uint32_t OFF_BAR = OFF_HEAD + HEAD_BYTES;
+constexpr uint32_t NBAR = 2 * NPART + 2 + 5;
+constexpr uint32_t SMEM = 1024 + OFF_BAR + NBAR * 8 + 64;
+
+struct Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* lat;
+  const int32_t* idx;
+  __nv_bfloat16* o;
+  float* lse;
+  int32_t T, Tk, H, topk;
+  float scale_log2;
+  int32_t* status;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// Arrives on `bar` once every cp.async this thread issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Reduces v[0..63] across the 32 lanes of the warp (max or sum); afterwards
+// lane L holds the results for entries 2L and 2L+1 in r0, r1.
+template <bool MAX>
+__device__ __forceinline__ void warp_transpose_reduce64(float (&v)[64], int lane, float& r0,
+                                                        float& r1) {
+  float w32[32];
+  {
+    const bool hi = lane & 16;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float mine = hi ? v[32 + i] : v[i];
+      const float other = hi ? v[i] : v[32 + i];
+      const float got = __shfl_xor_sync(0xffffffffu, other, 16);
+      w32[i] = MAX ? fmaxf(mine, got) : mine + got;
+    }
+  }
+  float w16[16];
+  {
+    const bool hi = lane & 8;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float mine = hi ? w32[16 + i] : w32[i];
+      const float other = hi ? w32[i] : w32[16 + i];
+      const float got = __shfl_xor_sync(0xffffffffu, other, 8);
+      w16[i] = MAX ? fmaxf(mine, got) : mine + got;
+    }
+  }
+  float w8[8];
+  {
+    const bool hi = lane & 4;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float mine = hi ? w16[8 + i] : w16[i];
+      const float other = hi ? w16[i] : w16[8 + i];
+      const float got = __shfl_xor_sync(0xffffffffu, other, 4);
+      w8[i] = MAX ? fmaxf(mine, got) : mine + got;
+    }
+  }
+  float w4[4];
+  {
+    const bool hi = lane & 2;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float mine = hi ? w8[4 + i] : w8[i];
+      const float other = hi ? w8[i] : w8[4 + i];
+      const float got = __shfl_xor_sync(0xffffffffu, other, 2);
+      w4[i] = MAX ? fmaxf(mine, got) : mine + got;
+    }
+  }
+  {
+    const bool hi = lane & 1;
+    float w2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float mine = hi ? w4[2 + i] : w4[i];
+      const float other = hi ? w4[i] : w4[2 + i];
+      const float got = __shfl_xor_sync(0xffffffffu, other, 1);
+      w2[i] = MAX ? fmaxf(mine, got) : mine + got;
+    }
+    r0 = w2[0];
+    r1 = w2[1];
+  }
+}
+
+__device__ __forceinline__ bool key_ok(int32_t k, int32_t Tk) { return k >= 0 && k < Tk; }
+
+__global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ uint32_t tmem_base_slot;
+  __shared__ int abort_flag;
+  __shared__ int q_ntiles;
+  __shared__ int prod_red[4];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* part_full = bar;                 // [8] 128 producer arrivals
+  uint64_t* part_empty = bar + NPART;        // [8] MMA commit
+  uint64_t* q_full = bar + 2 * NPART;        // 128 copy arrivals + 1 (tile count)
+  uint64_t* q_empty = q_full + 1;            // MMA commit
+  uint64_t* s_full = q_empty + 1;            // MMA commit
+  uint64_t* p_full = s_full + 1;             // 4 softmax warps
+  uint64_t* pv_done = p_full + 1;            // MMA commit
+  uint64_t* o_full = pv_done + 1;            // MMA commit
+  uint64_t* o_free = o_full + 1;             // 4 softmax warps
+  float* red = reinterpret_cast<float*>(smem + OFF_RED);
+  float* h_m = reinterpret_cast<float*>(smem + OFF_HEAD);  // running max (log2 domain)
+  float* h_l = h_m + HMAX;                                 // running sum
+  float* h_alpha = h_l + HMAX;                             // this tile's rescale factor
+  float* h_flag = h_alpha + HMAX;                          // [0]: any head rescaled
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int i = 0; i < NPART; ++i) {
+      mbar_init(part_full + i, 128);
+      mbar_init(part_empty + i, 1);
+    }
+    mbar_init(q_full, 129);  // 128 copy arrivals + the tile count
+    mbar_init(q_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    mbar_init(o_full, 1);
+    mbar_init(o_free, 4);
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&tmem_base_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_slot;
+  const int tiles_max = (p.topk + KT - 1) / KT;
+
+  // queries heaviest first: the last rows have the longest index lists
+  auto query_of = [&](int i) { return p.T - 1 - (int(blockIdx.x) + i * int(gridDim.x)); };
+
+  if (warp < 4) {
+    // ============================================================ producers
+    const int r = threadIdx.x;  // key slot within a tile
+    uint32_t tile_glob = 0;
+    bool ok = true;
+    for (int qi = 0; ok; ++qi) {
+      const int t = query_of(qi);
+      if (t < 0) break;
+      // tiles this query needs: up to the last valid index
+      int last = -1;
+      for (int s = r; s < p.topk; s += 128)
+        if (key_ok(__ldg(p.idx + size_t(t) * p.topk + s), p.Tk)) last = s;
+      for (int off = 16; off > 0; off >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, off));
+      if (!mbar_wait(q_empty, (qi & 1) ^ 1, &abort_flag, p.status)) break;
+      if (lane == 0) prod_red[warp] = last;
+      named_bar_sync(1, 128);
+      int lmax = -1;
+      for (int w = 0; w < 4; ++w) lmax = max(lmax, prod_red[w]);
+      named_bar_sync(1, 128);
+      if (r == 0) {
+        q_ntiles = (lmax + KT) / KT;
+        mbar_arrive(q_full);  // releases the tile count to the MMA and softmax warps
+      }
+      // Q_t^T: rows = heads (zero rows beyond H), 8 parts of 64 columns
+      const uint32_t sQ = smem_u32(smem + OFF_Q);
+      for (int c = r; c < HMAX * (DL / 8); c += 128) {
+        const int h = c / (DL / 8), ch = c % (DL / 8);  // 16-byte chunk of the row
+        const int part = ch >> 3, cc = ch & 7;
+        const uint32_t dst = sQ + part * QPART_BYTES + h * 128 + ((cc ^ (h & 7)) << 4);
+        const __nv_bfloat16* src = p.q + (size_t(t) * p.H + min(h, p.H - 1)) * DL + ch * 8;
+        cp_async16(dst, src, h < p.H ? 16u : 0u);
+      }
+      cp_async_arrive(q_full);
+      const int ntiles = (lmax + KT) / KT;
+      for (int j = 0; j < ntiles && ok; ++j, ++tile_glob) {
+        const int s = j * KT + r;
+        int32_t kidx = s < p.topk ? __ldg(p.idx + size_t(t) * p.topk + s) : -1;
+        if (kidx >= p.Tk) report_status(p.status, PSA_ERR_INVALID_ARG);
+        const bool valid = key_ok(kidx, p.Tk);
+        const __nv_bfloat16* row = p.lat + size_t(valid ? kidx : 0) * DL;
+        for (int part = 0; part < NPART; ++part) {
+          if (!mbar_wait(part_empty + part, (tile_glob & 1) ^ 1, &abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t base = smem_u32(smem + OFF_LAT + part * PART_BYTES) + r * 128;
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc)
+            cp_async16(base + ((cc ^ (r & 7)) << 4), row + part * 64 + cc * 8, valid ? 16u : 0u);
+          cp_async_arrive(part_full + part);
+        }
+      }
+    }
+    // let every copy this thread issued land before the CTA can exit
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 4) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = umma_idesc_bf16(KT, HMAX, false, false);
+      const uint32_t idesc_o = umma_idesc_bf16(128, HMAX, true, true);
+      const uint32_t sLat = smem_u32(smem + OFF_LAT);
+      const uint32_t sQ = smem_u32(smem + OFF_Q);
+      const uint32_t sP = smem_u32(smem + OFF_P);
+      uint32_t tile_glob = 0;
+      uint32_t oq = 0;  // queries with at least one tile (O^T produced)
+      bool ok = true;
+      for (int qi = 0; ok; ++qi) {
+        const int t = query_of(qi);
+        if (t < 0) break;
+        if (!mbar_wait(q_full, qi & 1, &abort_flag, p.status)) break;
+        const int ntiles = q_ntiles;
+        if (ntiles == 0) {
+          umma_commit(q_empty);
+          continue;
+        }
+        for (int j = 0; j < ntiles && ok; ++j, ++tile_glob) {
+          // S^T = Lat_tile . Q^T, accumulated over the eight parts
+          for (int part = 0; part < NPART && ok; ++part) {
+            if (!mbar_wait(part_full + part, tile_glob & 1, &abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              umma_ss(tmem, umma_desc_sw128(sLat + part * PART_BYTES + ks * 32, 16, 1024),
+                      umma_desc_sw128(sQ + part * QPART_BYTES + ks * 32, 16, 1024), idesc_s,
+                      (part | ks) ? 1u : 0u);
+          }
+          if (!ok) break;
+          umma_commit(s_full);
+          if (j == ntiles - 1) umma_commit(q_empty);
+          // O^T += Lat^T . P^T once the softmax has written P^T
+          if (!mbar_wait(p_full, tile_glob & 1, &abort_flag, p.status) ||
+              (j == 0 && !mbar_wait(o_free, (oq & 1) ^ 1, &abort_flag, p.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int mb = 0; mb < 4; ++mb) {
+#pragma unroll
+            for (int ks = 0; ks < KT / 16; ++ks)
+              umma_ss(tmem + 128 + mb * 64,
+                      umma_desc_sw128(sLat + 2 * mb * PART_BYTES + ks * 2048, PART_BYTES, 1024),
+                      umma_desc_sw128(sP + ks * 2048, 8192, 1024), idesc_o,
+                      (j > 0 || ks > 0) ? 1u : 0u);
+            umma_commit(part_empty + 2 * mb);
+            umma_commit(part_empty + 2 * mb + 1);
+          }
+          umma_commit(pv_done);
+          if (j == ntiles - 1) umma_commit(o_full);
+        }
+        ++oq;
+      }
+      if (!ok || abort_flag) {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 1000000ull) {
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ============================================================ softmax + epilogue
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // key slot (TMEM lane); latent dim in the epilogue
+    const int tid = threadIdx.x - 256;  // 0..127 within the group
+    const uint32_t trow = tmem + (uint32_t(quarter * 32) << 16);
+    uint32_t tile_glob = 0;
+    uint32_t oq = 0;  // queries with at least one tile
+    bool ok = true;
+    for (int qi = 0; ok; ++qi) {
+      const int t = query_of(qi);
+      if (t < 0) break;
+      if (!mbar_wait(q_full, qi & 1, &abort_flag, p.status)) break;
+      const int ntiles = q_ntiles;
+      if (tid < HMAX) {
+        h_m[tid] = -INFINITY;
+        h_l[tid] = 0.f;
+      }
+      named_bar_sync(2, 128);
+      for (int j = 0; j < ntiles && ok; ++j, ++tile_glob) {
+        const int s = j * KT + r;
+        const bool valid = s < p.topk && key_ok(__ldg(p.idx + size_t(t) * p.topk + s), p.Tk);
+        if (!mbar_wait(s_full, tile_glob & 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float v[HMAX];
+        {
+          uint32_t raw[HMAX];
+          tmem_ld64(trow, raw);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < HMAX; ++h) v[h] = valid ? __uint_as_float(raw[h]) : -INFINITY;
+        }
+        // per-head max over the 128 keys: across lanes, then across warps
+        float a0, a1;
+        {
+          float tmp[HMAX];
+#pragma unroll
+          for (int h = 0; h < HMAX; ++h) tmp[h] = v[h];
+          warp_transpose_reduce64<true>(tmp, lane, a0, a1);
+        }
+        red[quarter * HMAX + 2 * lane] = a0;
+        red[quarter * HMAX + 2 * lane + 1] = a1;
+        named_bar_sync(2, 128);
+        if (tid < HMAX) {
+          const float mt = fmaxf(fmaxf(red[tid], red[HMAX + tid]),
+                                 fmaxf(red[2 * HMAX + tid], red[3 * HMAX + tid])) *
+                           p.scale_log2;
+          const float mo = h_m[tid];
+          const float mn = fmaxf(mo, mt);
+          float alpha = 1.f;
+          if (mn > mo + kRescaleLog2) {
+            alpha = fast_exp2(mo - mn);  // 0 when mo = -inf
+            h_m[tid] = mn;
+          }
+          h_alpha[tid] = alpha;
+        }
+        if (tid == 0) h_flag[0] = 0.f;
+        named_bar_sync(2, 128);
+        if (tid < HMAX && h_alpha[tid] != 1.f && j > 0) h_flag[0] = 1.f;
+        // P^T row of this key: exp2(s * scale - m_h)
+        float pr[HMAX];
+#pragma unroll
+        for (int h = 0; h < HMAX; ++h) {
+          const float m = h_m[h];
+          pr[h] = fast_exp2(fmaf(v[h], p.scale_log2, m == -INFINITY ? 0.f : -m));
+        }
+        // the previous O^T product must be done before P^T is overwritten
+        if (j > 0 && !mbar_wait(pv_done, (tile_glob - 1) & 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        {
+          const uint32_t prow = smem_u32(smem + OFF_P) + r * 128;
+#pragma unroll
+          for (int c = 0; c < HMAX / 8; ++c) {
+            const uint32_t w0 = pack_bf16(pr[8 * c], pr[8 * c + 1]);
+            const uint32_t w1 = pack_bf16(pr[8 * c + 2], pr[8 * c + 3]);
+            const uint32_t w2 = pack_bf16(pr[8 * c + 4], pr[8 * c + 5]);
+            const uint32_t w3 = pack_bf16(pr[8 * c + 6], pr[8 * c + 7]);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             prow + ((c ^ (r & 7)) << 4)),
+                         "r"(w0), "r"(w1), "r"(w2), "r"(w3)
+                         : "memory");
+          }
+        }
+        // per-head sums
+        warp_transpose_reduce64<false>(pr, lane, a0, a1);
+        named_bar_sync(2, 128);  // everyone has read red[] for the max
+        red[quarter * HMAX + 2 * lane] = a0;
+        red[quarter * HMAX + 2 * lane + 1] = a1;
+        named_bar_sync(2, 128);
+        if (tid < HMAX)
+          h_l[tid] = h_l[tid] * h_alpha[tid] +
+                     ((red[tid] + red[HMAX + tid]) + (red[2 * HMAX + tid] + red[3 * HMAX + tid]));
+        // lazy O^T rescale: column h of every M-block times alpha_h
+        if (h_flag[0] != 0.f) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int mb = 0; mb < 4; ++mb) {
+            uint32_t ov[HMAX];
+            tmem_ld64(trow + 128 + mb * 64, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < HMAX; ++h)
+              ov[h] = __float_as_uint(__uint_as_float(ov[h]) * h_alpha[h]);
+            tmem_st64(trow + 128 + mb * 64, ov);
+          }
+          tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+      if (!ok) break;
+      named_bar_sync(2, 128);  // h_l final
+      if (ntiles > 0) {
+        if (!mbar_wait(o_full, oq & 1, &abort_flag, p.status)) break;
+        tc_fence_after();
+      }
+      // epilogue: thread owns latent dim d = 128 * mb + r, all heads
+#pragma unroll 1
+      for (int mb = 0; mb < 4; ++mb) {
+        uint32_t ov[HMAX];
+        if (ntiles > 0) {
+          tmem_ld64(trow + 128 + mb * 64, ov);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int h = 0; h < HMAX; ++h) ov[h] = 0u;
+        }
+        const int d = 128 * mb + r;
+        for (int h = 0; h < p.H; ++h) {
+          const float l = h_l[h];
+          const float val = l > 0.f ? __uint_as_float(ov[h]) / l : 0.f;
+          p.o[(size_t(t) * p.H + h) * DL + d] = __float2bfloat16(val);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (ntiles > 0) {
+        if (lane == 0) mbar_arrive(o_free);
+        ++oq;
+      }
+      if (tid < p.H && p.lse) {
+        const float l = h_l[tid];
+        p.lse[size_t(t) * p.H + tid] = l > 0.f ? (h_m[tid] + __log2f(l)) * kLn2 : -INFINITY;
+      }
+      named_bar_sync(2, 128);  // head state is reset at the next query
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 4) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+int launch_sparse_latent(const SparseArgs& a) {
+  if (a.dl != DL || a.H > HMAX || a.H <= 0) return PSA_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PSA_ERR_CUDA;
+  Params p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.lat = static_cast<const __nv_bfloat16*>(a.latent);
+  p.idx = a.idx;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.T = a.T;
+  p.Tk = a.Tk;
+  p.H = a.H;
+  p.topk = a.topk;
+  p.scale_log2 = a.scale * kLog2e;
+  p.status = a.status;
+  if (cudaFuncSetAttribute(sparse_latent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(SMEM)) != cudaSuccess)
+    return PSA_ERR_CUDA;
+  int grid = sm_count(dev);
+  if (grid <= 0) return PSA_ERR_CUDA;
+  if (grid > a.T) grid = a.T;
+  if (grid == 0) return PSA_OK;
+  sparse_latent_kernel<<<grid, kThreads, SMEM, a.stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? PSA_OK : PSA_ERR_CUDA;
+}
+
+}  // namespace psa

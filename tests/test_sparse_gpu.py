@@ -1,0 +1,91 @@
+"""Shared-latent sparse attention on the GPU against the fp64 oracle.
+
+"SM8x sparse-MLA prefill fallback re-reads the shared MLA latent once per
+head" (vLLM issue write-up): environment (one 512-wide latent is K and V for
+all 64 heads; each query attends to its own top-k index list, topk 2048) and
+analysis (head-blocked tiles share each gathered latent row across heads).
+Every call goes through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import shared_prefix_attention_b200 as psa
+from shared_prefix_attention_b200 import workloads as W
+from parity import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(q, lat, idx, scale, rows=None):
+    dev = "cuda"
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    o, lse = psa.sparse_latent(q.to(dev), lat.to(dev), idx.to(dev), scale, status=status)
+    torch.cuda.synchronize()
+    st = psa.read_status(status)
+    ro, rl = oracle.sparse_latent(q.cpu(), lat.cpu(), idx.cpu(), scale, rows=rows)
+    if rows is not None:
+        r = torch.as_tensor(rows, device=dev).long()
+        o, lse = o[r], lse[r]
+    return o, lse, ro, rl, st
+
+
+@pytest.mark.parametrize("T,H,topk", [
+    (300, 64, 256),   # dense causal rows then random lists, two tiles
+    (200, 16, 200),   # fewer heads, topk not a multiple of the tile
+    (129, 40, 128),   # one tile, ragged head count
+    (700, 64, 512),
+])
+def test_sparse_parity(T, H, topk):
+    wl = W.SparseLatentWorkload("t", T=T, H=H, dl=512, topk=topk, seed=T + H)
+    q, lat, idx = wl.make("cpu")
+    o, lse, ro, rl, st = _run(q, lat, idx, wl.scale)
+    assert st == 0
+    assert_parity(o, lse, ro, rl, f"T={T} H={H} topk={topk}")
+
+
+def test_sparse_holes_and_empty_rows():
+    """-1 entries anywhere in a list are skipped; a row with no index gets
+    O = 0 and LSE = -inf."""
+    wl = W.SparseLatentWorkload("t", T=260, H=64, dl=512, topk=256, seed=77)
+    q, lat, idx = wl.make("cpu")
+    g = torch.Generator().manual_seed(1)
+    holes = torch.rand(idx.shape, generator=g) < 0.3
+    idx = torch.where(holes, torch.full_like(idx, -1), idx)
+    idx[5] = -1
+    idx[259] = -1
+    o, lse, ro, rl, st = _run(q, lat, idx, wl.scale)
+    assert st == 0
+    assert torch.all(o[5] == 0) and torch.all(o[259] == 0)
+    assert torch.all(torch.isinf(lse[5])) and torch.all(lse[5] < 0)
+    keep = [r for r in range(260) if r not in (5, 259)]
+    assert_parity(o[keep], lse[keep], ro[keep], rl[keep], "holes")
+
+
+def test_sparse_out_of_range_index_is_skipped_and_reported():
+    wl = W.SparseLatentWorkload("t", T=150, H=8, dl=512, topk=128, seed=5)
+    q, lat, idx = wl.make("cpu")
+    bad = idx.clone()
+    bad[140, 3] = 10_000          # beyond the latent rows
+    o, lse, _, _, st = _run(q, lat, bad, wl.scale)
+    assert st == psa.PSA_ERR_INVALID_ARG
+    ref_idx = bad.clone()
+    ref_idx[140, 3] = -1          # the kernel skips it; the oracle is told so
+    ro, rl = oracle.sparse_latent(q, lat, ref_idx, wl.scale)
+    assert_parity(o, lse, ro, rl, "out of range skipped")
+
+
+def test_sparse_full_size_sampled_rows():
+    """The full 16384-query, 64-head, topk 2048 workload on device-generated
+    inputs (as the benchmark times it), checked on sampled rows."""
+    wl = W.SPARSE
+    q, lat, idx = wl.make("cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = psa.sparse_latent(q, lat, idx, wl.scale, status=status)
+    torch.cuda.synchronize()
+    assert psa.read_status(status) == 0
+    rows = [0, 1, 127, 128, 2047, 2048, 2049, 5000, 9999, 16383]
+    ro, rl = oracle.sparse_latent(q.cpu(), lat.cpu(), idx.cpu(), wl.scale, rows=rows)
+    r = torch.tensor(rows, device="cuda")
+    assert_parity(o[r], lse[r], ro, rl, "sparse full size")
+    assert torch.isfinite(o.float()).all()
