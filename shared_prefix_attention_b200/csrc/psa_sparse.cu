@@ -80,6 +80,16 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// A group barrier that every member skips once the CTA has aborted (a member
+// that gave up on a bounded wait never reaches the barrier); the `break`
+// leaves the enclosing loop.
+#define GROUP_SYNC(id)                 \
+  if (*(volatile int*)&abort_flag) {   \
+    ok = false;                        \
+    break;                             \
+  } else                               \
+    named_bar_sync((id), 128)
+
 // Reduces v[0..63] across the 32 lanes of the warp (max or sum); afterwards
 // lane L holds the results for entries 2L and 2L+1 in r0, r1.
 template <bool MAX>
@@ -215,9 +225,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
       for (int off = 16; off > 0; off >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, off));
       if (!mbar_wait(q_empty, (qi & 1) ^ 1, &abort_flag, p.status)) break;
       if (lane == 0) prod_red[warp] = last;
+      if (*(volatile int*)&abort_flag) break;
       named_bar_sync(1, 128);
       int lmax = -1;
       for (int w = 0; w < 4; ++w) lmax = max(lmax, prod_red[w]);
+      if (*(volatile int*)&abort_flag) break;
       named_bar_sync(1, 128);
       if (r == 0) {
         q_ntiles = (lmax + KT) / KT;
@@ -338,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
         h_m[tid] = -INFINITY;
         h_l[tid] = 0.f;
       }
-      named_bar_sync(2, 128);
+      GROUP_SYNC(2);
       for (int j = 0; j < ntiles && ok; ++j, ++tile_glob) {
         const int s = j * KT + r;
         const bool valid = s < p.topk && key_ok(__ldg(p.idx + size_t(t) * p.topk + s), p.Tk);
@@ -365,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
         }
         red[quarter * HMAX + 2 * lane] = a0;
         red[quarter * HMAX + 2 * lane + 1] = a1;
-        named_bar_sync(2, 128);
+        GROUP_SYNC(2);
         if (tid < HMAX) {
           const float mt = fmaxf(fmaxf(red[tid], red[HMAX + tid]),
                                  fmaxf(red[2 * HMAX + tid], red[3 * HMAX + tid])) *
@@ -380,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
           h_alpha[tid] = alpha;
         }
         if (tid == 0) h_flag[0] = 0.f;
-        named_bar_sync(2, 128);
+        GROUP_SYNC(2);
         if (tid < HMAX && h_alpha[tid] != 1.f && j > 0) h_flag[0] = 1.f;
         // P^T row of this key: exp2(s * scale - m_h)
         float pr[HMAX];
@@ -410,10 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
         }
         // per-head sums
         warp_transpose_reduce64<false>(pr, lane, a0, a1);
-        named_bar_sync(2, 128);  // everyone has read red[] for the max
+        GROUP_SYNC(2);  // everyone has read red[] for the max
         red[quarter * HMAX + 2 * lane] = a0;
         red[quarter * HMAX + 2 * lane + 1] = a1;
-        named_bar_sync(2, 128);
+        GROUP_SYNC(2);
         if (tid < HMAX)
           h_l[tid] = h_l[tid] * h_alpha[tid] +
                      ((red[tid] + red[HMAX + tid]) + (red[2 * HMAX + tid] + red[3 * HMAX + tid]));
@@ -438,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
         if (lane == 0) mbar_arrive(p_full);
       }
       if (!ok) break;
-      named_bar_sync(2, 128);  // h_l final
+      GROUP_SYNC(2);  // h_l final
       if (ntiles > 0) {
         if (!mbar_wait(o_full, oq & 1, &abort_flag, p.status)) break;
         tc_fence_after();
@@ -471,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
         const float l = h_l[tid];
         p.lse[size_t(t) * p.H + tid] = l > 0.f ? (h_m[tid] + __log2f(l)) * kLn2 : -INFINITY;
       }
-      named_bar_sync(2, 128);  // head state is reset at the next query
+      GROUP_SYNC(2);  // head state is reset at the next query
     }
   }
 
