@@ -320,11 +320,14 @@ class SparseRunner(Runner):
 
 VERIFY_SMALL = W.VerifyWorkload("verify B=8 L=16384 drafts=4 H=32/8 d=128 splits=32 bf16", B=8,
                                 L=16384, Ld=4, Hq=32, Hkv=8, d=128, nsplit=32, seed=4)
+SPARSE_SMALL = W.SparseLatentWorkload("sparse T=4096 H=64 dl=512 topk=2048 bf16", T=4096, H=64,
+                                      dl=512, topk=2048, seed=5)
 
 
 def make_runner(name: str, dev):
     return {"grpo": lambda: PrefillRunner(W.GRPO, dev),
             "verify8": lambda: VerifyRunner(VERIFY_SMALL, dev),
+            "sparse4k": lambda: SparseRunner(SPARSE_SMALL, dev),
             "tiny": lambda: PrefillRunner(W.TINY, dev),
             "large": lambda: PrefillRunner(W.LARGE, dev),
             "verify": lambda: VerifyRunner(W.VERIFY, dev),
@@ -395,7 +398,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="grpo",
-                    choices=["grpo", "tiny", "large", "verify", "verify8", "sparse"])
+                    choices=["grpo", "tiny", "large", "verify", "verify8", "sparse", "sparse4k"])
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
