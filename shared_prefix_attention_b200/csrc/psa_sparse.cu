@@ -46,9 +46,9 @@ constexpr uint32_t OFF_LAT = 0;
 constexpr uint32_t OFF_Q = OFF_LAT + NPART * PART_BYTES;     // 128 KB
 constexpr uint32_t OFF_P = OFF_Q + NPART * QPART_BYTES;      // +64 KB
 constexpr uint32_t OFF_RED = OFF_P + KT * 128;               // +16 KB
-constexpr uint32_t RED_BYTES = 4 * HMAX * 4;                 // [4 warps][64] floats
+constexpr uint32_t RED_BYTES = 2 * 4 * HMAX * 4;             // max and sum: [4 warps][64]
 constexpr uint32_t OFF_HEAD = OFF_RED + RED_BYTES;           // per-head state
-constexpr uint32_t HEAD_BYTES = 4 * HMAX * 4;                // m, l, alpha, m_tile
+constexpr uint32_t HEAD_BYTES = 4 * HMAX * 4;                // m, l, alpha, 1/l
 constexpr uint32_t OFF_BAR = OFF_HEAD + HEAD_BYTES;
 constexpr uint32_t NBAR = 2 * NPART + 2 + 5;
 constexpr uint32_t SMEM = 1024 + OFF_BAR + NBAR * 8 + 64;
@@ -93,7 +93,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 // Reduces v[0..63] across the 32 lanes of the warp (max or sum); afterwards
 // lane L holds the results for entries 2L and 2L+1 in r0, r1.
 template <bool MAX>
-__device__ __forceinline__ void warp_transpose_reduce64(float (&v)[64], int lane, float& r0,
+__device__ __forceinline__ void warp_transpose_reduce64(const float (&v)[64], int lane, float& r0,
                                                         float& r1) {
   float w32[32];
   {
@@ -156,6 +156,17 @@ __device__ __forceinline__ void warp_transpose_reduce64(float (&v)[64], int lane
 
 __device__ __forceinline__ bool key_ok(int32_t k, int32_t Tk) { return k >= 0 && k < Tk; }
 
+// Register split: 384 threads x 168 at launch = 64512.  The producer and
+// MMA warpgroups drop to 80 so the softmax warpgroup can keep a key's 64
+// logits, its 64 probabilities and the reduction scratch in registers
+// (2 x 128 x 80 + 128 x 248 = 52224).
+__device__ __forceinline__ void regs_dec80() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
+}
+__device__ __forceinline__ void regs_inc248() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 248;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -176,11 +187,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
   uint64_t* pv_done = p_full + 1;            // MMA commit
   uint64_t* o_full = pv_done + 1;            // MMA commit
   uint64_t* o_free = o_full + 1;             // 4 softmax warps
-  float* red = reinterpret_cast<float*>(smem + OFF_RED);
+  float* red_max = reinterpret_cast<float*>(smem + OFF_RED);  // [4 warps][64]
+  float* red_sum = red_max + 4 * HMAX;                         // [4 warps][64]
   float* h_m = reinterpret_cast<float*>(smem + OFF_HEAD);  // running max (log2 domain)
   float* h_l = h_m + HMAX;                                 // running sum
   float* h_alpha = h_l + HMAX;                             // this tile's rescale factor
-  float* h_flag = h_alpha + HMAX;                          // [0]: any head rescaled
+  float* h_inv = h_alpha + HMAX;                           // 1 / l for the epilogue
+  __shared__ int h_flagw[2];                               // a head-owner warp rescaled
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -211,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
   auto query_of = [&](int i) { return p.T - 1 - (int(blockIdx.x) + i * int(gridDim.x)); };
 
   if (warp < 4) {
+    regs_dec80();
     // ============================================================ producers
     const int r = threadIdx.x;  // key slot within a tile
     uint32_t tile_glob = 0;
@@ -267,9 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
     }
     // let every copy this thread issued land before the CTA can exit
     asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 4) {
+  } else if (warp < 8) {
+    regs_dec80();
     // ============================================================ MMA issuer
-    if (lane == 0) {
+    if (warp == 4 && lane == 0) {
       const uint32_t idesc_s = umma_idesc_bf16(KT, HMAX, false, false);
       const uint32_t idesc_o = umma_idesc_bf16(128, HMAX, true, true);
       const uint32_t sLat = smem_u32(smem + OFF_LAT);
@@ -332,7 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
         }
       }
     }
-  } else if (warp >= 8) {
+  } else {
+    regs_inc248();
     // ============================================================ softmax + epilogue
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key slot (TMEM lane); latent dim in the epilogue
@@ -344,6 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
     for (int qi = 0; ok; ++qi) {
       const int t = query_of(qi);
       if (t < 0) break;
+      const int32_t* qidx = p.idx + size_t(t) * p.topk;
+      // index of this thread's key slot in tile 0, fetched before the wait
+      int32_t kidx_next = r < p.topk ? __ldg(qidx + r) : -1;
       if (!mbar_wait(q_full, qi & 1, &abort_flag, p.status)) break;
       const int ntiles = q_ntiles;
       if (tid < HMAX) {
@@ -352,8 +371,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
       }
       GROUP_SYNC(2);
       for (int j = 0; j < ntiles && ok; ++j, ++tile_glob) {
-        const int s = j * KT + r;
-        const bool valid = s < p.topk && key_ok(__ldg(p.idx + size_t(t) * p.topk + s), p.Tk);
+        const bool valid = key_ok(kidx_next, p.Tk);
+        {
+          const int s = (j + 1) * KT + r;  // prefetch the next tile's index
+          kidx_next = s < p.topk ? __ldg(qidx + s) : -1;
+        }
         if (!mbar_wait(s_full, tile_glob & 1, &abort_flag, p.status)) {
           ok = false;
           break;
@@ -369,18 +391,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
         }
         // per-head max over the 128 keys: across lanes, then across warps
         float a0, a1;
-        {
-          float tmp[HMAX];
-#pragma unroll
-          for (int h = 0; h < HMAX; ++h) tmp[h] = v[h];
-          warp_transpose_reduce64<true>(tmp, lane, a0, a1);
-        }
-        red[quarter * HMAX + 2 * lane] = a0;
-        red[quarter * HMAX + 2 * lane + 1] = a1;
+        warp_transpose_reduce64<true>(v, lane, a0, a1);
+        red_max[quarter * HMAX + 2 * lane] = a0;
+        red_max[quarter * HMAX + 2 * lane + 1] = a1;
         GROUP_SYNC(2);
-        if (tid < HMAX) {
-          const float mt = fmaxf(fmaxf(red[tid], red[HMAX + tid]),
-                                 fmaxf(red[2 * HMAX + tid], red[3 * HMAX + tid])) *
+        if (tid < HMAX) {  // head owners: warps 8 and 9
+          const float mt = fmaxf(fmaxf(red_max[tid], red_max[HMAX + tid]),
+                                 fmaxf(red_max[2 * HMAX + tid], red_max[3 * HMAX + tid])) *
                            p.scale_log2;
           const float mo = h_m[tid];
           const float mn = fmaxf(mo, mt);
@@ -390,10 +407,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
             h_m[tid] = mn;
           }
           h_alpha[tid] = alpha;
+          const bool any = __any_sync(0xffffffffu, alpha != 1.f && j > 0);
+          if (lane == 0) h_flagw[quarter] = any ? 1 : 0;
         }
-        if (tid == 0) h_flag[0] = 0.f;
         GROUP_SYNC(2);
-        if (tid < HMAX && h_alpha[tid] != 1.f && j > 0) h_flag[0] = 1.f;
+        const bool rescale = (h_flagw[0] | h_flagw[1]) != 0;
         // P^T row of this key: exp2(s * scale - m_h)
         float pr[HMAX];
 #pragma unroll
@@ -420,17 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
                          : "memory");
           }
         }
-        // per-head sums
-        warp_transpose_reduce64<false>(pr, lane, a0, a1);
-        GROUP_SYNC(2);  // everyone has read red[] for the max
-        red[quarter * HMAX + 2 * lane] = a0;
-        red[quarter * HMAX + 2 * lane + 1] = a1;
-        GROUP_SYNC(2);
-        if (tid < HMAX)
-          h_l[tid] = h_l[tid] * h_alpha[tid] +
-                     ((red[tid] + red[HMAX + tid]) + (red[2 * HMAX + tid] + red[3 * HMAX + tid]));
         // lazy O^T rescale: column h of every M-block times alpha_h
-        if (h_flag[0] != 0.f) {
+        if (rescale) {
           tc_fence_after();
 #pragma unroll 1
           for (int mb = 0; mb < 4; ++mb) {
@@ -448,14 +457,26 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
+        // per-head sums (off the MMA's critical path)
+        warp_transpose_reduce64<false>(pr, lane, a0, a1);
+        red_sum[quarter * HMAX + 2 * lane] = a0;
+        red_sum[quarter * HMAX + 2 * lane + 1] = a1;
+        GROUP_SYNC(2);
+        if (tid < HMAX)
+          h_l[tid] = h_l[tid] * h_alpha[tid] + ((red_sum[tid] + red_sum[HMAX + tid]) +
+                                                (red_sum[2 * HMAX + tid] + red_sum[3 * HMAX + tid]));
       }
       if (!ok) break;
-      GROUP_SYNC(2);  // h_l final
+      if (tid < HMAX) h_inv[tid] = h_l[tid] > 0.f ? 1.f / h_l[tid] : 0.f;
+      GROUP_SYNC(2);  // h_l, h_inv final
       if (ntiles > 0) {
         if (!mbar_wait(o_full, oq & 1, &abort_flag, p.status)) break;
         tc_fence_after();
       }
-      // epilogue: thread owns latent dim d = 128 * mb + r, all heads
+      // epilogue: per M-block, thread d = r scales its O^T lane by 1/l_h and
+      // stages it as [head][128 dims] in the (now idle) P^T buffer; the block
+      // then goes out as contiguous 16-byte rows.
+      __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem + OFF_P);
 #pragma unroll 1
       for (int mb = 0; mb < 4; ++mb) {
         uint32_t ov[HMAX];
@@ -466,13 +487,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_latent_kernel(Params p) {
 #pragma unroll
           for (int h = 0; h < HMAX; ++h) ov[h] = 0u;
         }
-        const int d = 128 * mb + r;
-        for (int h = 0; h < p.H; ++h) {
-          const float l = h_l[h];
-          const float val = l > 0.f ? __uint_as_float(ov[h]) / l : 0.f;
-          p.o[(size_t(t) * p.H + h) * DL + d] = __float2bfloat16(val);
+#pragma unroll
+        for (int h = 0; h < HMAX; ++h)
+          stage[h * 128 + r] = __float2bfloat16(__uint_as_float(ov[h]) * h_inv[h]);
+        GROUP_SYNC(2);
+#pragma unroll
+        for (int k = 0; k < (HMAX * 16) / 128; ++k) {
+          const int c = k * 128 + tid;  // 16-byte chunk: head c / 16, piece c % 16
+          const int h = c >> 4, piece = c & 15;
+          if (h < p.H)
+            *reinterpret_cast<uint4*>(p.o + (size_t(t) * p.H + h) * DL + mb * 128 + piece * 8) =
+                *reinterpret_cast<const uint4*>(stage + h * 128 + piece * 8);
         }
+        GROUP_SYNC(2);
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (ntiles > 0) {
