@@ -13,11 +13,11 @@
 // the 128 rows of a tcgen05 MMA:
 //   S^T [128 keys x H]   = Lat_tile [128 x 512] . Q_t^T [512 x H]
 //   O^T [512 x H]       += Lat_tile^T [512 x 128] . P^T [128 x H]
-// The latent tile is gathered by TMA gather4 (four rows per instruction,
-// zero fill for -1 entries, no multicast) in eight 64-column parts; a part
+// The latent tile is gathered by cp.async (whole 128-byte rows per group of
+// eight threads, zero fill for -1 entries) in eight 64-column parts; a part
 // is released for the next tile as soon as the O^T block that reads it has
-// completed.
-//   warp 0       gather producer (four key slots per lane) and the Q^T load
+// completed.  Q_t^T arrives by TMA.
+//   warps 0..3   gather producers and the Q^T load
 //   warp 4       tcgen05 issuer (one thread)
 //   warps 8..11  softmax over keys (one key per thread = TMEM lane) with
 //                per-head max / sum reductions across lanes, P^T written to
@@ -65,18 +65,16 @@ struct Params {
   int32_t* status;
 };
 
-// Four latent rows (one 64-column box each) into consecutive 128-byte rows of
-// shared memory, 128-byte swizzle; rows outside [0, Tk) read as zeros.  No
-// multicast.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t x, int32_t r0, int32_t r1, int32_t r2,
-                                            int32_t r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1),
-      "r"(r2), "r"(r3)
-      : "memory");
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// Arrives on `bar` once every cp.async this thread issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
@@ -171,18 +169,18 @@ __device__ __forceinline__ void regs_inc248() {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_latent_kernel(const __grid_constant__ CUtensorMap tmap_lat,
-                         const __grid_constant__ CUtensorMap tmap_q, Params p) {
+    sparse_latent_kernel(const __grid_constant__ CUtensorMap tmap_q, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
   __shared__ int q_ntiles;
+  __shared__ int prod_ntiles;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* part_full = bar;                 // [8] producer arrive + TMA bytes
+  uint64_t* part_full = bar;                 // [8] 128 producer copy arrivals
   uint64_t* part_empty = bar + NPART;        // [8] MMA commit
   uint64_t* q_full = bar + 2 * NPART;        // producer arrive (tile count) + TMA bytes
   uint64_t* q_empty = q_full + 1;            // MMA commit
@@ -202,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int i = 0; i < NPART; ++i) {
-      mbar_init(part_full + i, 1);
+      mbar_init(part_full + i, 128);
       mbar_init(part_empty + i, 1);
     }
     mbar_init(q_full, 1);
@@ -229,61 +227,76 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     regs_dec80();
-    // ============================================================ producer
-    // Warp 0: each lane owns four key slots of a tile and gathers their
-    // latent rows with TMA gather4, one 64-column part at a time.
-    if (warp == 0) {
-      tma_prefetch_desc(&tmap_lat);
+    // ============================================================ producers
+    // Warps 0..3 gather the latent tile with cp.async: eight threads cover
+    // one 128-byte row of a part, so every warp instruction moves four whole
+    // rows.  Lane 0 of warp 0 loads Q^T with TMA and publishes the tile count.
+    const int pt = threadIdx.x;      // 0..127
+    const int chunk = pt & 7;        // 16-byte piece of a part row
+    const int rsub = pt >> 3;        // 0..15: row within a round of 16
+    if (pt == 0) {
       tma_prefetch_desc(&tmap_q);
-      uint32_t tile_glob = 0;
-      bool ok = true;
-      for (int qi = 0; ok; ++qi) {
-        const int t = query_of(qi);
-        if (t < 0) break;
-        const int32_t* qidx = p.idx + size_t(t) * p.topk;
-        // tiles this query needs: up to the last valid index
+    }
+    uint32_t tile_glob = 0;
+    bool ok = true;
+    for (int qi = 0; ok; ++qi) {
+      const int t = query_of(qi);
+      if (t < 0) break;
+      const int32_t* qidx = p.idx + size_t(t) * p.topk;
+      int ntiles = 0;
+      if (warp == 0) {
         int last = -1;
         for (int sl = lane; sl < p.topk; sl += 32)
           if (key_ok(__ldg(qidx + sl), p.Tk)) last = sl;
         for (int off = 16; off > 0; off >>= 1)
           last = max(last, __shfl_xor_sync(0xffffffffu, last, off));
-        const int ntiles = (last + KT) / KT;
-        if (!mbar_wait(q_empty, (qi & 1) ^ 1, &abort_flag, p.status)) break;
-        if (lane == 0) {
+        ntiles = (last + KT) / KT;
+        if (!mbar_wait(q_empty, (qi & 1) ^ 1, &abort_flag, p.status)) ntiles = -1;
+        if (lane == 0 && ntiles >= 0) {
           q_ntiles = ntiles;  // published by the arrive below
           mbar_arrive_expect_tx(q_full, NPART * QPART_BYTES);
 #pragma unroll
           for (int part = 0; part < NPART; ++part)
             tma_load_2d(smem + OFF_Q + part * QPART_BYTES, &tmap_q, q_full, part * 64, t * p.H);
         }
-        for (int j = 0; j < ntiles && ok; ++j, ++tile_glob) {
-          int32_t rows[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int sl = j * KT + 4 * lane + i;
-            const int32_t k = sl < p.topk ? __ldg(qidx + sl) : -1;
-            if (k >= p.Tk) report_status(p.status, PSA_ERR_INVALID_ARG);
-            rows[i] = key_ok(k, p.Tk) ? k : p.Tk;  // out of range: zero fill
-          }
-          for (int part = 0; part < NPART; ++part) {
-            if (!mbar_wait(part_empty + part, (tile_glob & 1) ^ 1, &abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            if (lane == 0) mbar_arrive_expect_tx(part_full + part, PART_BYTES);
-            __syncwarp();
-            tma_gather4(smem_u32(smem + OFF_LAT + part * PART_BYTES) + lane * 4 * 128, &tmap_lat,
-                        part_full + part, part * 64, rows[0], rows[1], rows[2], rows[3]);
-          }
-        }
+        if (lane == 0) prod_ntiles = ntiles;
       }
-      if (!ok || abort_flag) {
-        // let copies in flight land before the CTA exits
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 1000000ull) {
+      if (*(volatile int*)&abort_flag) break;
+      named_bar_sync(1, 128);
+      ntiles = prod_ntiles;
+      if (*(volatile int*)&abort_flag) break;
+      named_bar_sync(1, 128);
+      if (ntiles < 0) break;
+      for (int j = 0; j < ntiles && ok; ++j, ++tile_glob) {
+        const __nv_bfloat16* src[8];
+        uint32_t sz[8];
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int sl = j * KT + it * 16 + rsub;
+          const int32_t k = sl < p.topk ? __ldg(qidx + sl) : -1;
+          if (k >= p.Tk) report_status(p.status, PSA_ERR_INVALID_ARG);
+          const bool valid = key_ok(k, p.Tk);
+          src[it] = p.lat + size_t(valid ? k : 0) * DL + chunk * 8;
+          sz[it] = valid ? 16u : 0u;  // zero fill for skipped slots
+        }
+        for (int part = 0; part < NPART; ++part) {
+          if (!mbar_wait(part_empty + part, (tile_glob & 1) ^ 1, &abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t base = smem_u32(smem + OFF_LAT + part * PART_BYTES);
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int row = it * 16 + rsub;
+            cp_async16(base + row * 128 + ((chunk ^ (row & 7)) << 4), src[it] + part * 64,
+                       sz[it]);
+          }
+          cp_async_arrive(part_full + part);
         }
       }
     }
+    // let every copy this thread issued land before the CTA can exit
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp < 8) {
     regs_dec80();
     // ============================================================ MMA issuer
@@ -543,15 +556,7 @@ int launch_sparse_latent(const SparseArgs& a) {
   p.topk = a.topk;
   p.scale_log2 = a.scale * kLog2e;
   p.status = a.status;
-  CUtensorMap tl, tq;
-  {
-    const uint64_t dims[2] = {uint64_t(DL), uint64_t(a.Tk)};
-    const uint64_t strides[1] = {uint64_t(DL) * 2};
-    const uint32_t box[2] = {64u, 1u};  // gather4 boxes are one row high
-    const int rc = encode_tmap(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.latent, dims, strides,
-                               box, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (rc != PSA_OK) return rc;
-  }
+  CUtensorMap tq;
   {
     const uint64_t dims[2] = {uint64_t(DL), uint64_t(a.T) * a.H};
     const uint64_t strides[1] = {uint64_t(DL) * 2};
@@ -567,7 +572,7 @@ int launch_sparse_latent(const SparseArgs& a) {
   if (grid <= 0) return PSA_ERR_CUDA;
   if (grid > a.T) grid = a.T;
   if (grid == 0) return PSA_OK;
-  sparse_latent_kernel<<<grid, kThreads, SMEM, a.stream>>>(tl, tq, p);
+  sparse_latent_kernel<<<grid, kThreads, SMEM, a.stream>>>(tq, p);
   return cudaGetLastError() == cudaSuccess ? PSA_OK : PSA_ERR_CUDA;
 }
 
