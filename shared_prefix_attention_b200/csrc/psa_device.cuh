@@ -200,33 +200,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x for a pair, on the FMA pipe instead of the MUFU: Cody-Waite style
-// range reduction x = j + f with j = round-to-nearest(x) (the 1.5 * 2^23
-// shifter leaves j in the low mantissa bits), f in [-0.5, 0.5]; 2^f from a
-// degree-3 polynomial whose coefficients were fitted by the Remez exchange
-// algorithm for minimal relative error on [-0.5, 0.5] (max relative error
-// 7.5e-5, below the bf16 rounding the result gets); 2^j is added to the
-// exponent field.  x is clamped to -126 so the exponent never underflows.
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t t = f2_add(x, f2_pack(kShift, kShift));
-  const uint64_t j = f2_add(t, f2_pack(-kShift, -kShift));
-  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);
-  uint64_t p = f2_fma(f, f2_pack(0.0551716685295105f, 0.0551716685295105f),
-                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
-  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  // (bits(t) << 23) == round(x) << 23 modulo 2^32: the shifter's own bits vanish
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {

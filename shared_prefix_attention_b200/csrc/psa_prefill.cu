@@ -480,39 +480,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
 
-        // P = exp2(s * scale - m) as bf16, written over the S columns.  On
-        // fully visible tiles 3 of every 8 pairs take the polynomial exp2 on
-        // the FMA pipe so the MUFU is not the bottleneck; partial tiles use
-        // the MUFU only (masked logits are -inf and must give exactly 0).
+        // P = exp2(s * scale - m) as bf16, written over the S columns (masked
+        // logits are -inf and give exactly 0)
         const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(neg_m, neg_m);
         uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-        if (!need_mask) {
 #pragma unroll
-          for (int k = 0; k < BN / 2; ++k) {
-            float x0, x1, p0, p1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])),
-                             sc2, nm2),
-                      x0, x1);
-            if ((k & 7) < 3) {
-              exp2_poly_pair(x0, x1, p0, p1);
-            } else {
-              p0 = fast_exp2(x0);
-              p1 = fast_exp2(x1);
-            }
-            acc2[k & 3] = f2_add(acc2[k & 3], f2_pack(p0, p1));
-            sr[k] = pack_bf16(p0, p1);  // packed pairs go into consumed registers (k <= 2k)
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < BN / 2; ++k) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])),
-                             sc2, nm2),
-                      x0, x1);
-            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            acc2[k & 3] = f2_add(acc2[k & 3], f2_pack(p0, p1));
-            sr[k] = pack_bf16(p0, p1);
-          }
+        for (int k = 0; k < BN / 2; ++k) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])),
+                           sc2, nm2),
+                    x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          acc2[k & 3] = f2_add(acc2[k & 3], f2_pack(p0, p1));
+          sr[k] = pack_bf16(p0, p1);  // packed pairs go into consumed registers (k <= 2k)
         }
         float ls8[8];
 #pragma unroll
