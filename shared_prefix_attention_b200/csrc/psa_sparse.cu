@@ -160,12 +160,12 @@ __device__ __forceinline__ bool key_ok(int32_t k, int32_t Tk) { return k >= 0 &&
 // Register split: 384 threads x 168 at launch = 64512.  The producer and
 // MMA warpgroups drop to 80 so the softmax warpgroup can keep a key's 64
 // logits, its 64 probabilities and the reduction scratch in registers
-// (2 x 128 x 80 + 128 x 248 = 52224).
+// (2 x 128 x 80 + 128 x 256 = 53248).
 __device__ __forceinline__ void regs_dec80() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
 }
-__device__ __forceinline__ void regs_inc248() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 248;" ::: "memory");
+__device__ __forceinline__ void regs_inc256() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 256;" ::: "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -212,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(o_free, 4);
     fence_barrier_init();
   }
+  if (threadIdx.x >= 256 && threadIdx.x < 256 + HMAX) h_m[threadIdx.x - 256] = -INFINITY;
   if (warp == 4) {
     tmem_alloc(&tmem_base_slot, kTmemCols);
     tmem_relinquish();
@@ -364,8 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    regs_inc248();
+    regs_inc256();
     // ============================================================ softmax + epilogue
+    // One key per thread.  The 64 running maxima (log2 domain) live in shared
+    // memory, each thread keeps its own 64 partial row sums in registers; a
+    // tile only needs
+    // a cross-key max when some logit would exceed its head's running max by
+    // more than 2^8 (the first tile of a query always does), detected with
+    // one OR-reduction barrier.  The partial sums meet once per query.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key slot (TMEM lane); latent dim in the epilogue
     const int tid = threadIdx.x - 256;  // 0..127 within the group
@@ -381,16 +388,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int32_t kidx_next = r < p.topk ? __ldg(qidx + r) : -1;
       if (!mbar_wait(q_full, qi & 1, &abort_flag, p.status)) break;
       const int ntiles = q_ntiles;
-      if (tid < HMAX) {
-        h_m[tid] = -INFINITY;
-        h_l[tid] = 0.f;
-      }
-      GROUP_SYNC(2);
+      float lpart[HMAX];
+#pragma unroll
+      for (int h = 0; h < HMAX; ++h) lpart[h] = 0.f;
       for (int j = 0; j < ntiles && ok; ++j, ++tile_glob) {
         const bool valid = key_ok(kidx_next, p.Tk);
         {
-          const int s = (j + 1) * KT + r;  // prefetch the next tile's index
-          kidx_next = s < p.topk ? __ldg(qidx + s) : -1;
+          const int sl = (j + 1) * KT + r;  // prefetch the next tile's index
+          kidx_next = sl < p.topk ? __ldg(qidx + sl) : -1;
         }
         if (!mbar_wait(s_full, tile_glob & 1, &abort_flag, p.status)) {
           ok = false;
@@ -403,37 +408,77 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld64(trow, raw);
           tmem_wait_ld();
 #pragma unroll
-          for (int h = 0; h < HMAX; ++h) v[h] = valid ? __uint_as_float(raw[h]) : -INFINITY;
+          for (int h = 0; h < HMAX; ++h)
+            v[h] = valid ? __uint_as_float(raw[h]) * p.scale_log2 : -INFINITY;
         }
-        // per-head max over the 128 keys: across lanes, then across warps
-        float a0, a1;
-        warp_transpose_reduce64<true>(v, lane, a0, a1);
-        red_max[quarter * HMAX + 2 * lane] = a0;
-        red_max[quarter * HMAX + 2 * lane + 1] = a1;
-        GROUP_SYNC(2);
-        if (tid < HMAX) {  // head owners: warps 8 and 9
-          const float mt = fmaxf(fmaxf(red_max[tid], red_max[HMAX + tid]),
-                                 fmaxf(red_max[2 * HMAX + tid], red_max[3 * HMAX + tid])) *
-                           p.scale_log2;
-          const float mo = h_m[tid];
-          const float mn = fmaxf(mo, mt);
-          float alpha = 1.f;
-          if (mn > mo + kRescaleLog2) {
-            alpha = fast_exp2(mo - mn);  // 0 when mo = -inf
-            h_m[tid] = mn;
+        // does any logit of this tile outgrow its head's running max?
+        float over = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < HMAX; ++h) over = fmaxf(over, v[h] - h_m[h]);
+        if (*(volatile int*)&abort_flag) {
+          ok = false;
+          break;
+        }
+        uint32_t any_over;
+        asm volatile(
+            "{\n\t.reg .pred pi, po;\n\t"
+            "setp.gt.f32 pi, %1, %2;\n\t"
+            "bar.red.or.pred po, 2, 128, pi;\n\t"
+            "selp.u32 %0, 1, 0, po;\n\t}"
+            : "=r"(any_over)
+            : "f"(over), "f"(kRescaleLog2)
+            : "memory");
+        if (any_over) {
+          // cross-key max per head: across lanes, then across warps
+          float a0, a1;
+          warp_transpose_reduce64<true>(v, lane, a0, a1);
+          red_max[quarter * HMAX + 2 * lane] = a0;
+          red_max[quarter * HMAX + 2 * lane + 1] = a1;
+          GROUP_SYNC(2);
+          if (tid < HMAX) {
+            const float mt = fmaxf(fmaxf(red_max[tid], red_max[HMAX + tid]),
+                                   fmaxf(red_max[2 * HMAX + tid], red_max[3 * HMAX + tid]));
+            const float mo = h_m[tid];
+            const float mn = fmaxf(mo, mt);
+            float alpha = 1.f;
+            if (mn > mo + kRescaleLog2) {
+              alpha = fast_exp2(mo - mn);  // 0 when mo = -inf
+              h_m[tid] = mn;
+            }
+            h_alpha[tid] = alpha;
+            const bool any = __any_sync(0xffffffffu, alpha != 1.f && j > 0);
+            if (lane == 0) h_flagw[quarter] = any ? 1 : 0;
           }
-          h_alpha[tid] = alpha;
-          const bool any = __any_sync(0xffffffffu, alpha != 1.f && j > 0);
-          if (lane == 0) h_flagw[quarter] = any ? 1 : 0;
+          GROUP_SYNC(2);
+#pragma unroll
+          for (int h = 0; h < HMAX; ++h) lpart[h] *= h_alpha[h];
+          if (h_flagw[0] | h_flagw[1]) {
+            // lazy O^T rescale: column h of every M-block times alpha_h, once
+            // the previous O^T product has landed
+            if (!mbar_wait(pv_done, (tile_glob - 1) & 1, &abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int mb = 0; mb < 4; ++mb) {
+              uint32_t ov[HMAX];
+              tmem_ld64(trow + 128 + mb * 64, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int h = 0; h < HMAX; ++h)
+                ov[h] = __float_as_uint(__uint_as_float(ov[h]) * h_alpha[h]);
+              tmem_st64(trow + 128 + mb * 64, ov);
+            }
+            tmem_wait_st();
+          }
         }
-        GROUP_SYNC(2);
-        const bool rescale = (h_flagw[0] | h_flagw[1]) != 0;
         // P^T row of this key: exp2(s * scale - m_h)
-        float pr[HMAX];
 #pragma unroll
         for (int h = 0; h < HMAX; ++h) {
           const float m = h_m[h];
-          pr[h] = fast_exp2(fmaf(v[h], p.scale_log2, m == -INFINITY ? 0.f : -m));
+          v[h] = fast_exp2(v[h] - (m == -INFINITY ? 0.f : m));
+          lpart[h] += v[h];
         }
         // the previous O^T product must be done before P^T is overwritten
         if (j > 0 && !mbar_wait(pv_done, (tile_glob - 1) & 1, &abort_flag, p.status)) {
@@ -444,46 +489,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t prow = smem_u32(smem + OFF_P) + r * 128;
 #pragma unroll
           for (int c = 0; c < HMAX / 8; ++c) {
-            const uint32_t w0 = pack_bf16(pr[8 * c], pr[8 * c + 1]);
-            const uint32_t w1 = pack_bf16(pr[8 * c + 2], pr[8 * c + 3]);
-            const uint32_t w2 = pack_bf16(pr[8 * c + 4], pr[8 * c + 5]);
-            const uint32_t w3 = pack_bf16(pr[8 * c + 6], pr[8 * c + 7]);
+            const uint32_t w0 = pack_bf16(v[8 * c], v[8 * c + 1]);
+            const uint32_t w1 = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
+            const uint32_t w2 = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
+            const uint32_t w3 = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
                              prow + ((c ^ (r & 7)) << 4)),
                          "r"(w0), "r"(w1), "r"(w2), "r"(w3)
                          : "memory");
           }
         }
-        // lazy O^T rescale: column h of every M-block times alpha_h
-        if (rescale) {
-          tc_fence_after();
-#pragma unroll 1
-          for (int mb = 0; mb < 4; ++mb) {
-            uint32_t ov[HMAX];
-            tmem_ld64(trow + 128 + mb * 64, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < HMAX; ++h)
-              ov[h] = __float_as_uint(__uint_as_float(ov[h]) * h_alpha[h]);
-            tmem_st64(trow + 128 + mb * 64, ov);
-          }
-          tmem_wait_st();
-        }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
-        // per-head sums (off the MMA's critical path)
-        warp_transpose_reduce64<false>(pr, lane, a0, a1);
-        red_sum[quarter * HMAX + 2 * lane] = a0;
-        red_sum[quarter * HMAX + 2 * lane + 1] = a1;
-        GROUP_SYNC(2);
-        if (tid < HMAX)
-          h_l[tid] = h_l[tid] * h_alpha[tid] + ((red_sum[tid] + red_sum[HMAX + tid]) +
-                                                (red_sum[2 * HMAX + tid] + red_sum[3 * HMAX + tid]));
       }
       if (!ok) break;
-      if (tid < HMAX) h_inv[tid] = h_l[tid] > 0.f ? 1.f / h_l[tid] : 0.f;
+      // per-head sums: the partial sums of all keys meet once per query
+      {
+        float a0, a1;
+        warp_transpose_reduce64<false>(lpart, lane, a0, a1);
+        red_sum[quarter * HMAX + 2 * lane] = a0;
+        red_sum[quarter * HMAX + 2 * lane + 1] = a1;
+      }
+      GROUP_SYNC(2);
+      if (tid < HMAX) {
+        const float l = (red_sum[tid] + red_sum[HMAX + tid]) +
+                        (red_sum[2 * HMAX + tid] + red_sum[3 * HMAX + tid]);
+        h_l[tid] = l;
+        h_inv[tid] = l > 0.f ? 1.f / l : 0.f;
+      }
       GROUP_SYNC(2);  // h_l, h_inv final
       if (ntiles > 0) {
         if (!mbar_wait(o_full, oq & 1, &abort_flag, p.status)) break;
@@ -528,7 +563,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l = h_l[tid];
         p.lse[size_t(t) * p.H + tid] = l > 0.f ? (h_m[tid] + __log2f(l)) * kLn2 : -INFINITY;
       }
-      GROUP_SYNC(2);  // head state is reset at the next query
+      if (tid < HMAX) h_m[tid] = -INFINITY;  // fresh running max for the next query
+      GROUP_SYNC(2);
     }
   }
 
