@@ -276,6 +276,20 @@ int psa_sparse_latent_fwd(const void *q, const void *latent, const int32_t *idx,
  * This is the one call that waits on the device. */
 int psa_read_status(const int32_t *dev_status, int32_t *host_out, void *stream);
 
+/* Failure-detection self-test of the bounded device wait every kernel uses
+ * (no counterpart on the pages).  Launches one warp on `stream` that waits
+ * on a shared-memory barrier expecting one arrival.
+ *   arrive != 0: the barrier is arrived at first; the wait completes at once
+ *                and *dev_status is left unchanged.
+ *   arrive == 0: nothing arrives; after the library's wait budget (2 s) the
+ *                wait gives up, writes PSA_ERR_TIMEOUT to *dev_status (when
+ *                it still holds 0) and the kernel returns normally, leaving
+ *                the context usable.
+ * dev_status (device int32, required) is owned by the caller, who zeroes it.
+ * Returns PSA_ERR_INVALID_ARG for a null dev_status, PSA_ERR_CUDA if the
+ * launch fails, else PSA_OK. */
+int psa_wait_selftest(int32_t arrive, int32_t *dev_status, void *stream);
+
 #if defined(__GNUC__)
 #pragma GCC visibility pop
 #endif

@@ -31,6 +31,7 @@ EXPORTS = [
     "psa_build_schedule", "psa_prefill_tiles", "psa_prefill_workspace_size",
     "psa_prefill_fwd", "psa_verify_auto_splits", "psa_verify_workspace_size",
     "psa_verify_fwd", "psa_verify_fwd_noalloc", "psa_sparse_latent_fwd", "psa_read_status",
+    "psa_wait_selftest",
 ]
 
 
@@ -89,6 +90,7 @@ def lib():
         "psa_sparse_latent_fwd": ([P, P, P, P, P, I32, I32, I32, I32, I32, F, P, P],
                                   ctypes.c_int),
         "psa_read_status": ([P, P, P], ctypes.c_int),
+        "psa_wait_selftest": ([I32, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -278,3 +280,11 @@ def read_status(status: torch.Tensor) -> int:
     _check(lib().psa_read_status(_ptr(status), ctypes.byref(v), _stream(status.device)),
            "psa_read_status")
     return v.value
+
+
+def wait_selftest(status: torch.Tensor, arrive: bool) -> None:
+    """Launches the library's bounded-wait self-test on ``status``'s device:
+    with ``arrive`` the wait completes at once, without it the wait gives up
+    after the library's budget and writes PSA_ERR_TIMEOUT to ``status``."""
+    _check(lib().psa_wait_selftest(1 if arrive else 0, _ptr(status), _stream(status.device)),
+           "psa_wait_selftest")
