@@ -96,13 +96,14 @@ __device__ __forceinline__ void set_bits(uint32_t (&m)[4], int a, int b) {
 
 // Register split between warpgroups: the launch gives every thread 168
 // registers (384 x 168 = 64512); warpgroup 0 (the two producers, the MMA
-// issuer, one idle warp) drops to 72 so the two softmax warpgroups can hold
-// a whole 128-column S row in registers (2 x 128 x 208 + 128 x 72 = 62464).
+// issuer, one idle warp) drops to 104, the least that keeps the MMA issuer
+// free of spills, so the two softmax warpgroups can hold a whole 128-column
+// S row in registers (2 x 128 x 200 + 128 x 104 = 64512).
 __device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 72;" ::: "memory");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 104;" ::: "memory");
 }
 __device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
 }
 
 // Header check shared by both prefill kernels (uniform across threads).
@@ -113,20 +114,20 @@ __device__ __forceinline__ bool schedule_ok(const int32_t* sch, int64_t len) {
          8 + 4 * int64_t(n_items) + 8 * int64_t(n_kv) + 5 * int64_t(n_rect) <= len;
 }
 
+// One schedule KV entry as seen by half x (its rectangle range selected
+// without indexing, so the entry stays in registers).
 struct KvEntry {
-  int k0, klen, rb[2], rc[2], flags;
+  int k0, klen, rb, rc, flags;
 };
 
-__device__ __forceinline__ KvEntry load_kv(const int32_t* kvs, int idx) {
+__device__ __forceinline__ KvEntry load_kv(const int32_t* kvs, int idx, int x) {
   const int4 a = __ldg(reinterpret_cast<const int4*>(kvs) + 2 * idx);
   const int4 b = __ldg(reinterpret_cast<const int4*>(kvs) + 2 * idx + 1);
   KvEntry e;
   e.k0 = a.x;
   e.klen = a.y;
-  e.rb[0] = a.z;
-  e.rc[0] = a.w;
-  e.rb[1] = b.x;
-  e.rc[1] = b.y;
+  e.rb = x ? b.x : a.z;
+  e.rc = x ? b.y : a.w;
   e.flags = b.z;
   return e;
 }
@@ -139,8 +140,8 @@ __device__ __forceinline__ void row_visibility(const KvEntry& e, int x, int q,
     set_bits(vis, 0, e.klen);
     return;
   }
-  for (int ri = 0; ri < e.rc[x]; ++ri) {
-    const int32_t* rc = rects + 5 * (e.rb[x] + ri);
+  for (int ri = 0; ri < e.rc; ++ri) {
+    const int32_t* rc = rects + 5 * (e.rb + ri);
     const int rq0 = __ldg(rc), rq1 = __ldg(rc + 1), rk0 = __ldg(rc + 2), rk1 = __ldg(rc + 3),
               causal = __ldg(rc + 4);
     if (q < rq0 || q >= rq1) continue;
@@ -163,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
   __shared__ int sch_unit[kSchedSlots];
+  __shared__ int4 sch_item[kSchedSlots];  // the unit's schedule block, fetched once
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -245,18 +247,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot_s = i % kSchedSlots;
         const uint32_t sph = (i / kSchedSlots) & 1;
         int u;
+        int4 it = make_int4(0, 0, 0, 0);
         if (kprod) {
           if (!mbar_wait(B.sch_empty + slot_s, sph ^ 1, &abort_flag, p.status)) break;
           u = atomicAdd(p.counter, 1);
+          if (u < units) it = __ldg(items + u / p.Hq);
+          sch_item[slot_s] = it;
           sch_unit[slot_s] = u;
           mbar_arrive(B.sch_full + slot_s);
         } else {
           if (!mbar_wait(B.sch_full + slot_s, sph, &abort_flag, p.status)) break;
           u = sch_unit[slot_s];
+          it = sch_item[slot_s];
           mbar_arrive(B.sch_empty + slot_s);
         }
         if (u >= units) break;
-        const int4 it = __ldg(items + u / p.Hq);
         const int h = u % p.Hq, kvh = h / p.G;
         if (it.w == 0) continue;
         if (kprod) {
@@ -350,28 +355,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot_s = i % kSchedSlots;
         if (!mbar_wait(B.sch_full + slot_s, (i / kSchedSlots) & 1, &abort_flag, p.status)) break;
         const int u = sch_unit[slot_s];
+        const int4 it = sch_item[slot_s];
         mbar_arrive(B.sch_empty + slot_s);
         if (u >= units) break;
-        const int4 it = __ldg(items + u / p.Hq);
         const int n = it.w;
         if (n == 0) continue;
+        // tile flags (which halves see the tile) are read two tiles ahead so
+        // their latency hides behind the waits
+        int f = __ldg(kvs + 8 * it.z + 6);
+        int fn = n > 1 ? __ldg(kvs + 8 * (it.z + 1) + 6) : 0;
         if (!mbar_wait(B.q_full, uc & 1, &abort_flag, p.status)) break;
         bool started[2] = {false, false};
         // prologue: QK of tile 0 for each half that takes part in it
-        {
-          const int f = __ldg(kvs + 8 * it.z + 6);
-          for (int x = 0; x < 2 && ok; ++x)
-            if (f & (1 << x)) ok = issue_qk(x, kc);
-          if (!ok) break;
-          umma_commit(B.k_empty + (kc % C::NSK));
-          if (n == 1) umma_commit(B.q_empty);
-        }
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+          if (ok && (f & (1 << x))) ok = issue_qk(x, kc);
+        if (!ok) break;
+        umma_commit(B.k_empty + (kc % C::NSK));
+        if (n == 1) umma_commit(B.q_empty);
         for (int j = 0; j < n && ok; ++j) {
-          const int f = __ldg(kvs + 8 * (it.z + j) + 6);
-          const int fn = j + 1 < n ? __ldg(kvs + 8 * (it.z + j + 1) + 6) : 0;
+          const int fnn = j + 2 < n ? __ldg(kvs + 8 * (it.z + j + 2) + 6) : 0;
           const uint32_t t = kc + j;
-          for (int x = 0; x < 2 && ok; ++x) {
-            if (f & (1 << x)) {
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (ok && (f & (1 << x))) {
               ok = issue_pv(x, t, !started[x]);
               started[x] = true;
             }
@@ -383,9 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(B.k_empty + ((t + 1) % C::NSK));
             if (j + 2 == n) umma_commit(B.q_empty);
           }
+          f = fn;
+          fn = fnn;
         }
         if (!ok) break;
         kc += n;
+#pragma unroll
         for (int x = 0; x < 2; ++x)
           if (started[x]) ++uhc[x];
         ++uc;
@@ -412,10 +422,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int slot_s = i % kSchedSlots;
       if (!mbar_wait(B.sch_full + slot_s, (i / kSchedSlots) & 1, &abort_flag, p.status)) break;
       const int u = sch_unit[slot_s];
+      const int4 it = sch_item[slot_s];
       __syncwarp();
       if (lane == 0) mbar_arrive(B.sch_empty + slot_s);
       if (u >= units) break;
-      const int4 it = __ldg(items + u / p.Hq);
       const int h = u % p.Hq;
       const int q = it.x + x * BM + r;
       const bool valid = x * BM + r < it.y;
@@ -423,8 +433,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       float m_run = -INFINITY, l_run = 0.f;
       int nt = 0;  // tiles of this half in this unit
+      // the next tile's schedule entry is read one tile ahead
+      KvEntry e_next{0, 0, 0, 0, 0};
+      if (it.w > 0) e_next = load_kv(kvs, it.z, x);
       for (int j = 0; j < it.w; ++j) {
-        const KvEntry e = load_kv(kvs, it.z + j);
+        const KvEntry e = e_next;
+        if (j + 1 < it.w) e_next = load_kv(kvs, it.z + j + 1, x);
         if (!(e.flags & (1 << x))) continue;
         if (!mbar_wait(B.s_full + x, sc_count & 1, &abort_flag, p.status)) {
           ok = false;
@@ -456,26 +470,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                          p.scale_log2;
         const float m_new = fmaxf(m_run, mx);
         const bool resc = m_new > m_run + kRescaleLog2;
-        if (__any_sync(0xffffffffu, resc) && nt > 0) {
-          // O holds the PVs of earlier tiles: wait for the latest, rescale
-          if (!mbar_wait(B.pv_done + x, (sc_count - 1) & 1, &abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const float alpha = resc ? fast_exp2(m_run - m_new) : 1.f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t rr[32];
-            tmem_ld32(tO + c * 32, rr);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) rr[k] = __float_as_uint(__uint_as_float(rr[k]) * alpha);
-            tmem_st32(tO + c * 32, rr);
-          }
-        }
+        // O (the PVs of earlier tiles) is rescaled after P is stored, when the
+        // S row no longer occupies registers; it only has to happen before
+        // this tile's PV, which waits for p_full.
+        const bool rescale_o = __any_sync(0xffffffffu, resc) && nt > 0;
+        float alpha = 1.f;
         if (resc) {
-          l_run *= fast_exp2(m_run - m_new);
+          alpha = fast_exp2(m_run - m_new);
+          l_run *= alpha;
           m_run = m_new;
         }
         const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
@@ -499,6 +501,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < 4; ++k) f2_unpack(acc2[k], ls8[2 * k], ls8[2 * k + 1]);
         tmem_st64(tS, *reinterpret_cast<uint32_t(*)[BN / 2]>(sr));
         l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+        if (rescale_o) {
+          // wait for the latest PV into O, then scale O by alpha in place
+          if (!mbar_wait(B.pv_done + x, (sc_count - 1) & 1, &abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(tO + c * 32, rr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) rr[k] = __float_as_uint(__uint_as_float(rr[k]) * alpha);
+            tmem_st32(tO + c * 32, rr);
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -596,7 +615,7 @@ __global__ void __launch_bounds__(256) prefill_f32_kernel(
     }
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < it.w; ++j) {
-      const KvEntry ent = load_kv(kvs, it.z + j);
+      const KvEntry ent = load_kv(kvs, it.z + j, x);
       if (!(ent.flags & (1 << x))) continue;
       uint32_t vis[4];
       row_visibility(ent, x, qi, rects, vis);
