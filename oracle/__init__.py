@@ -65,10 +65,12 @@ def load(path: str | None = None):
     D = ctypes.c_double
     lib.oracle_prefill.argtypes = [P, P, P, I, I, I, I, D, P, P, P, I, P, I, P, P, I]
     lib.oracle_verify.argtypes = [P, P, P, P, P, P, I, I, I, I, I, D, P, I, P, P, I]
+    lib.oracle_verify_shared.argtypes = [P, P, P, P, P, ctypes.c_int64, I, I, I, I, I, D, P, I,
+                                         P, P, I]
     lib.oracle_sparse_latent.argtypes = [P, P, P, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_visibility.argtypes = [P, P, P, I, I, I, I, P]
-    for f in (lib.oracle_prefill, lib.oracle_verify, lib.oracle_sparse_latent,
-              lib.oracle_visibility):
+    for f in (lib.oracle_prefill, lib.oracle_verify, lib.oracle_verify_shared,
+              lib.oracle_sparse_latent, lib.oracle_visibility):
         f.restype = I
     if path == _LIB_PATH:
         _lib = lib
@@ -159,6 +161,26 @@ def verify(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr, Ld: int,
                            B, Ld, Hq, Hkv, d, float(scale), _ptr(rows), len(rows),
                            _ptr(o), _ptr(lse), nthreads or default_threads())
     assert rc == 0, "oracle_verify rejected its arguments"
+    return o, lse
+
+
+def verify_shared(q_draft, k_draft, v_draft, k_prefix, v_prefix, Ld: int, scale: float,
+                  rows=None, nthreads: int | None = None, lib=None):
+    """O [nrows, Hq, d] and LSE [nrows, Hq] for draft rows b*Ld + j when every
+    request sees the same prefix k_prefix/v_prefix [L, Hkv, d]."""
+    lib = lib or load()
+    qd, kd, vd = _f32(q_draft), _f32(k_draft), _f32(v_draft)
+    kp, vp = _f32(k_prefix), _f32(v_prefix)
+    BL, Hq, d = qd.shape
+    Hkv = kd.shape[1]
+    B = BL // Ld
+    rows = np.arange(BL, dtype=np.int32) if rows is None else _i32(rows)
+    o = np.zeros((len(rows), Hq, d), dtype=np.float64)
+    lse = np.zeros((len(rows), Hq), dtype=np.float64)
+    rc = lib.oracle_verify_shared(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kp), _ptr(vp),
+                                  int(kp.shape[0]), B, Ld, Hq, Hkv, d, float(scale), _ptr(rows),
+                                  len(rows), _ptr(o), _ptr(lse), nthreads or default_threads())
+    assert rc == 0, "oracle_verify_shared rejected its arguments"
     return o, lse
 
 

@@ -256,7 +256,8 @@ int oracle_prefill(const float *q, const float *k, const float *v, int T, int Hq
 
 typedef struct {
     const float *qd, *kd, *vd, *kc, *vc;
-    const int64_t *indptr;
+    const int64_t *indptr; /* NULL: every request shares cache tokens [0, shared_len) */
+    int64_t shared_len;
     int Ld, Hq, Hkv, d;
     double scale;
     const int32_t *rows;
@@ -267,7 +268,8 @@ static void verify_row(void *p, int r, double *z, const float **vr, double *o) {
     verify_ctx *c = (verify_ctx *)p;
     int row = c->rows[r]; /* row = b * Ld + j */
     int b = row / c->Ld, j = row % c->Ld;
-    int64_t p0 = c->indptr[b], p1 = c->indptr[b + 1];
+    int64_t p0 = c->indptr ? c->indptr[b] : 0;
+    int64_t p1 = c->indptr ? c->indptr[b + 1] : c->shared_len;
     for (int h = 0; h < c->Hq; ++h) {
         int kvh = kv_head_of(h, c->Hq, c->Hkv);
         const float *qrow = c->qd + ((size_t)row * c->Hq + h) * c->d;
@@ -309,8 +311,28 @@ int oracle_verify(const float *qd, const float *kd, const float *vd,
     int64_t maxlen = 0;
     for (int b = 0; b < B; ++b)
         if (indptr[b + 1] - indptr[b] > maxlen) maxlen = indptr[b + 1] - indptr[b];
-    verify_ctx c = {qd, kd, vd, kc, vc, indptr, Ld, Hq, Hkv, d, scale, rows, o, lse};
+    verify_ctx c = {qd, kd, vd, kc, vc, indptr, 0, Ld, Hq, Hkv, d, scale, rows, o, lse};
     run_rows(verify_row, &c, nrows, (int)maxlen + Ld, d, nthreads);
+    return 0;
+}
+
+/*
+ * Verify against one prefix shared by every request: the prefix K/V is
+ * stored once ("KV-0 redundancy prefix sharing attention mask design",
+ * design summary) and every draft row of every request sees all of it plus
+ * its own causal draft block ("Split-KV flash-decode attention for EAGLE
+ * target-verify", implementation item 1).  k_prefix/v_prefix [L, Hkv, d];
+ * the other arguments are those of oracle_verify.  By definition this
+ * equals oracle_verify on a cache holding B copies of the prefix.
+ */
+int oracle_verify_shared(const float *qd, const float *kd, const float *vd,
+                         const float *kp, const float *vp, int64_t L,
+                         int B, int Ld, int Hq, int Hkv, int d, double scale,
+                         const int32_t *rows, int nrows, double *o, double *lse,
+                         int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || B < 0 || Ld <= 0 || L < 0) return -1;
+    verify_ctx c = {qd, kd, vd, kp, vp, NULL, L, Ld, Hq, Hkv, d, scale, rows, o, lse};
+    run_rows(verify_row, &c, nrows, (int)L + Ld, d, nthreads);
     return 0;
 }
 

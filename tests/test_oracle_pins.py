@@ -304,10 +304,38 @@ def pin_sparse_latent(lib):
     return bool(ok)
 
 
+def pin_verify_shared_prefix(lib):
+    """One prefix shared by every request, stored once ([PS] design summary:
+    the flat layout keeps the prefix K/V a single time) and seen by every
+    draft row together with its own causal draft block ([SKV] implementation
+    item 1).  Checked against torch SDPA with an explicit mask, and against
+    the per-request verify on a cache that holds B physical copies of the
+    prefix (the deduplication must not change the result)."""
+    B, Ld, Hq, Hkv, d, L = 3, 4, 6, 2, 16, 45
+    q = _rand((B * Ld, Hq, d), 51)
+    kd, vd = _rand((B * Ld, Hkv, d), 52), _rand((B * Ld, Hkv, d), 53)
+    kp, vp = _rand((L, Hkv, d), 54), _rand((L, Hkv, d), 55)
+    scale = 1 / math.sqrt(d)
+    o, lse = oracle.verify_shared(q, kd, vd, kp, vp, Ld, scale, lib=lib)
+    ok = True
+    for b in range(B):
+        ks = torch.cat([kp, kd[b * Ld:(b + 1) * Ld]])
+        vs = torch.cat([vp, vd[b * Ld:(b + 1) * Ld]])
+        mask = torch.ones((Ld, L + Ld), dtype=torch.bool)
+        mask[:, L:] = torch.tril(torch.ones((Ld, Ld), dtype=torch.bool))
+        ref = _sdpa(q[b * Ld:(b + 1) * Ld], _expand_kv(ks, Hq), _expand_kv(vs, Hq), mask, scale)
+        ok &= np.allclose(o[b * Ld:(b + 1) * Ld], ref, atol=1e-12)
+    kc, vc = kp.repeat(B, 1, 1), vp.repeat(B, 1, 1)
+    indptr = np.arange(B + 1, dtype=np.int64) * L
+    o2, lse2 = oracle.verify(q, kd, vd, kc, vc, indptr, Ld, scale, lib=lib)
+    ok &= np.array_equal(o, o2) and np.array_equal(lse, lse2)
+    return bool(ok)
+
+
 PINS = [pin_golden_masks, pin_golden_tiny_attention, pin_equivalence_route,
         pin_sdpa_random_trees, pin_closed_forms, pin_special_cases,
         pin_brute_force_python, pin_verify_against_sdpa, pin_split_identity,
-        pin_sparse_latent]
+        pin_verify_shared_prefix, pin_sparse_latent]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
