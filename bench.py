@@ -318,6 +318,34 @@ class SparseRunner(Runner):
                                lse=self.lse)
 
 
+class SharedVerifyRunner(Runner):
+    """Verify against one prefix shared by all requests: tensor-bound (the
+    stacked draft rows of a KV head multiply the prefix once)."""
+    unit = "TFLOP/s"
+    bound = "tensor"
+    kernels_per_step = 2
+    kernel_file = "psa_verify_shared.cu"
+
+    def __init__(self, wl: W.SharedVerifyWorkload, dev):
+        import shared_prefix_attention_b200 as psa
+        self.psa, self.wl, self.dev = psa, wl, dev
+        self.name = wl.name
+        self.q, self.kd, self.vd, self.kp, self.vp = wl.make(dev)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=dev)
+        self.ns = wl.nsplit or psa.verify_shared_auto_splits(wl.B, wl.Ld, wl.Hq, wl.Hkv, wl.L)
+        n = psa.verify_workspace_size(wl.B, wl.Ld, wl.Hq, wl.d, self.ns)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+
+    def work(self):
+        return self.wl.flops()
+
+    def step(self):
+        wl = self.wl
+        self.psa.verify_shared(self.q, self.kd, self.vd, self.kp, self.vp, wl.scale, wl.Ld,
+                               nsplit=self.ns, out=self.o, lse=self.lse, workspace=self.ws)
+
+
 VERIFY_SMALL = W.VerifyWorkload("verify B=8 L=16384 drafts=4 H=32/8 d=128 splits=32 bf16", B=8,
                                 L=16384, Ld=4, Hq=32, Hkv=8, d=128, nsplit=32, seed=4)
 SPARSE_SMALL = W.SparseLatentWorkload("sparse T=4096 H=64 dl=512 topk=2048 bf16", T=4096, H=64,
@@ -331,6 +359,7 @@ def make_runner(name: str, dev):
             "tiny": lambda: PrefillRunner(W.TINY, dev),
             "large": lambda: PrefillRunner(W.LARGE, dev),
             "verify": lambda: VerifyRunner(W.VERIFY, dev),
+            "verify-shared": lambda: SharedVerifyRunner(W.VERIFY_SHARED, dev),
             "sparse": lambda: SparseRunner(W.SPARSE, dev)}[name]()
 
 
@@ -398,7 +427,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="grpo",
-                    choices=["grpo", "tiny", "large", "verify", "verify8", "sparse", "sparse4k"])
+                    choices=["grpo", "tiny", "large", "verify", "verify8", "verify-shared",
+                             "sparse", "sparse4k"])
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -450,7 +480,7 @@ def main():
 
     if not args.no_extras and args.workload == "grpo":
         extras = {}
-        for name in ("verify", "large", "sparse"):
+        for name in ("verify", "verify-shared", "large", "sparse"):
             try:
                 r = make_runner(name, dev)
                 v, m, rf = measure(r, max(3, min(args.steps, 10)), 3, flush, dist_on, world,

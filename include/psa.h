@@ -248,6 +248,46 @@ int psa_verify_fwd_noalloc(const void *q_draft, const void *k_draft, const void 
                            int32_t *dev_status, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Speculative verify against one prefix shared by every request.
+ *   [PS] design summary (the prefix K/V is stored once and every sequence
+ *   built on it sees all of it) + [SKV] implementation item 1 (a draft row
+ *   sees the prefix plus drafts 0..j of its own request).
+ * --------------------------------------------------------------------- */
+
+/* nsplit chosen by psa_verify_shared_fwd when it is passed 0: about two
+ * units (chunk, KV head, 256 stacked rows) per SM, chunks of >= 512 keys. */
+int32_t psa_verify_shared_auto_splits(int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv,
+                                      int64_t prefix_len);
+
+/*
+ * The B requests share ONE cached prefix instead of owning one each, so the
+ * prefix is read once for all of them: the B * Ld * (Hq / Hkv) draft rows of
+ * a KV head are stacked into 128-row tensor-core tiles and multiplied
+ * against each prefix chunk, then the chunks and each row's causal draft
+ * block are merged by log-sum-exp weight exactly as in psa_verify_fwd.
+ *   q_draft          device [B*Ld, Hq, d] bf16   draft queries, request-major
+ *   k_draft, v_draft device [B*Ld, Hkv, d] bf16  draft keys / values
+ *   k_prefix,        device [L, Hkv, d] bf16     the shared prefix (nullable
+ *   v_prefix                                     when L == 0)
+ *   prefix_len       host value L, 0 <= L <= 2^30
+ *   o                device [B*Ld, Hq, d] bf16   (written)
+ *   lse              device [B*Ld, Hq] fp32      (written; nullable)
+ * Draft j of request b sees prefix tokens 0..L-1 and drafts 0..j of b; the
+ * result equals psa_verify_fwd on a cache holding B copies of the prefix.
+ * d in {64, 128}; Hq / Hkv must divide 128.  nsplit: 1..256, or 0 for
+ * psa_verify_shared_auto_splits; the prefix is cut into nsplit chunks of
+ * ceil(L / nsplit) keys rounded up to 128 (trailing chunks may be empty).
+ * workspace: device, >= psa_verify_workspace_size(B, Ld, Hq, d, nsplit)
+ * bytes, 256-B aligned (PSA_ERR_WORKSPACE otherwise).  Statuses as for
+ * psa_verify_fwd.
+ */
+int psa_verify_shared_fwd(const void *q_draft, const void *k_draft, const void *v_draft,
+                          const void *k_prefix, const void *v_prefix, int64_t prefix_len,
+                          void *o, float *lse, int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv,
+                          int32_t head_dim, float scale, int32_t nsplit, void *workspace,
+                          size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------
  * Shared-latent sparse attention                     [MLA] environment,
  * analysis (head-blocked tiles; the latent is shared by every head)
  * --------------------------------------------------------------------- */

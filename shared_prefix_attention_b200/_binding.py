@@ -31,7 +31,7 @@ EXPORTS = [
     "psa_build_schedule", "psa_prefill_tiles", "psa_prefill_workspace_size",
     "psa_prefill_fwd", "psa_verify_auto_splits", "psa_verify_workspace_size",
     "psa_verify_fwd", "psa_verify_fwd_noalloc", "psa_sparse_latent_fwd", "psa_read_status",
-    "psa_wait_selftest",
+    "psa_wait_selftest", "psa_verify_shared_auto_splits", "psa_verify_shared_fwd",
 ]
 
 
@@ -91,6 +91,9 @@ def lib():
                                   ctypes.c_int),
         "psa_read_status": ([P, P, P], ctypes.c_int),
         "psa_wait_selftest": ([I32, P, P], ctypes.c_int),
+        "psa_verify_shared_auto_splits": ([I32, I32, I32, I32, I64], I32),
+        "psa_verify_shared_fwd": ([P, P, P, P, P, I64, P, P, I32, I32, I32, I32, I32, F, I32, P,
+                                   ctypes.c_size_t, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -288,3 +291,31 @@ def wait_selftest(status: torch.Tensor, arrive: bool) -> None:
     after the library's budget and writes PSA_ERR_TIMEOUT to ``status``."""
     _check(lib().psa_wait_selftest(1 if arrive else 0, _ptr(status), _stream(status.device)),
            "psa_wait_selftest")
+
+
+def verify_shared_auto_splits(B: int, Ld: int, Hq: int, Hkv: int, prefix_len: int) -> int:
+    return int(lib().psa_verify_shared_auto_splits(B, Ld, Hq, Hkv, int(prefix_len)))
+
+
+def verify_shared(q_draft, k_draft, v_draft, k_prefix, v_prefix, scale: float, Ld: int,
+                  nsplit: int = 0, out=None, lse=None, workspace=None, status=None):
+    """Verify against one prefix shared by every request: O [B*Ld, Hq, d]
+    bf16 and LSE [B*Ld, Hq] fp32; k_prefix/v_prefix [L, Hkv, d]."""
+    _require_cuda(q_draft, k_draft, v_draft, k_prefix, v_prefix)
+    BL, Hq, d = q_draft.shape
+    Hkv = k_draft.shape[1]
+    B = BL // Ld
+    L = k_prefix.shape[0]
+    ns = nsplit or verify_shared_auto_splits(B, Ld, Hq, Hkv, L)
+    out = torch.empty_like(q_draft) if out is None else out
+    lse = torch.empty((BL, Hq), dtype=torch.float32, device=q_draft.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(max(verify_workspace_size(B, Ld, Hq, d, ns), 256),
+                                dtype=torch.uint8, device=q_draft.device)
+    rc = lib().psa_verify_shared_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft),
+                                     _ptr(k_prefix) if L else None,
+                                     _ptr(v_prefix) if L else None, L, _ptr(out), _ptr(lse), B,
+                                     Ld, Hq, Hkv, d, float(scale), ns, _ptr(workspace),
+                                     workspace.numel(), _ptr(status), _stream(q_draft.device))
+    _check(rc, "psa_verify_shared_fwd")
+    return out, lse

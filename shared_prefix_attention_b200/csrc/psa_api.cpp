@@ -195,6 +195,78 @@ extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const vo
   return launch_verify(a);
 }
 
+// ------------------------------------------------------- shared-prefix verify
+
+extern "C" int32_t psa_verify_shared_auto_splits(int32_t B, int32_t Ld, int32_t Hq,
+                                                 int32_t Hkv, int64_t prefix_len) {
+  if (B <= 0 || Ld <= 0 || Hkv <= 0 || Hq <= 0 || prefix_len <= 0) return 1;
+  // Aim for about two units (chunk, KV head, 256-row block) per SM of a
+  // 148-SM part while keeping every chunk at least four 128-key tiles long.
+  const int64_t rows = int64_t(B) * Ld * (Hq / Hkv);
+  const int64_t per_split = int64_t(Hkv) * ((rows + 255) / 256);
+  int64_t n = (2 * 148 + per_split - 1) / per_split;
+  const int64_t by_len = prefix_len / 512;
+  if (n > by_len) n = by_len;
+  if (n < 1) n = 1;
+  if (n > 256) n = 256;
+  return int32_t(n);
+}
+
+extern "C" int psa_verify_shared_fwd(const void* q_draft, const void* k_draft,
+                                     const void* v_draft, const void* k_prefix,
+                                     const void* v_prefix, int64_t prefix_len, void* o,
+                                     float* lse, int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv,
+                                     int32_t head_dim, float scale, int32_t nsplit,
+                                     void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                     void* stream) {
+  if (B < 0 || Ld <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || prefix_len < 0 ||
+      prefix_len > (int64_t(1) << 30) || !(scale > 0.f))
+    return PSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PSA_ERR_UNSUPPORTED;
+  const int32_t G = Hq / Hkv;
+  if (G > 128 || 128 % G != 0) return PSA_ERR_UNSUPPORTED;  // 128-row halves of whole tokens
+  if (int64_t(B) * Ld > INT32_MAX / Hq) return PSA_ERR_INVALID_ARG;
+  if (B == 0) return PSA_OK;
+  if (!q_draft || !k_draft || !v_draft || !o) return PSA_ERR_INVALID_ARG;
+  if (prefix_len > 0 && (!k_prefix || !v_prefix)) return PSA_ERR_INVALID_ARG;
+  if (!aligned16(q_draft) || !aligned16(k_draft) || !aligned16(v_draft) || !aligned16(o) ||
+      (prefix_len > 0 && (!aligned16(k_prefix) || !aligned16(v_prefix))) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return PSA_ERR_INVALID_ARG;
+  if (nsplit == 0) nsplit = psa_verify_shared_auto_splits(B, Ld, Hq, Hkv, prefix_len);
+  if (nsplit < 1 || nsplit > 256) return PSA_ERR_INVALID_ARG;
+  const size_t need = psa_verify_workspace_size(B, Ld, Hq, head_dim, nsplit);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PSA_ERR_WORKSPACE;
+
+  VerifySharedArgs a;
+  a.q = q_draft;
+  a.kd = k_draft;
+  a.vd = v_draft;
+  a.kp = k_prefix;
+  a.vp = v_prefix;
+  a.L = prefix_len;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.Ld = Ld;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = head_dim;
+  a.scale = scale;
+  a.nsplit = nsplit;
+  // whole 128-key tiles per chunk; trailing chunks may be empty
+  const int64_t per = (prefix_len + nsplit - 1) / nsplit;
+  a.chunk = int32_t((per + 127) / 128 * 128);
+  const size_t rows = size_t(nsplit) * B * Ld * Hq;
+  const size_t o_bytes = (rows * head_dim * sizeof(float) + 255) / 256 * 256;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + o_bytes);
+  a.status = dev_status;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_verify_shared(a);
+}
+
 // ------------------------------------------------------------------ prefill
 
 extern "C" int psa_prefill_tiles(int32_t head_dim, int32_t* tile_m, int32_t* tile_n) {

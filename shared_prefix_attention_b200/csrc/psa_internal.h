@@ -46,6 +46,28 @@ struct VerifyArgs {
 int verify_plan(int32_t Ld, int32_t Hq, int32_t Hkv, int32_t D, int32_t* heads_per_block,
                 int32_t* mtiles, int32_t* row_blocks);
 int launch_verify(const VerifyArgs& a);
+// Stage 2 alone: merge a.nsplit partials with the causal draft block.
+int launch_verify_combine(const VerifyArgs& a);
+
+// Verify against one prefix shared by every request.
+struct VerifySharedArgs {
+  const void* q;   // bf16 [B*Ld, Hq, D]
+  const void* kd;  // bf16 [B*Ld, Hkv, D]
+  const void* vd;
+  const void* kp;  // bf16 [L, Hkv, D], the shared prefix
+  const void* vp;
+  int64_t L;
+  void* o;
+  float* lse;
+  int32_t B, Ld, Hq, Hkv, D;
+  float scale;
+  int32_t nsplit, chunk;  // chunk: prefix keys per split, a multiple of 128
+  float* part_o;          // [nsplit][B*Ld][Hq][D]
+  float* part_lse;        // [nsplit][B*Ld][Hq], log2 domain
+  int32_t* status;
+  cudaStream_t stream;
+};
+int launch_verify_shared(const VerifySharedArgs& a);
 
 // ---------------------------------------------------------------- prefill
 

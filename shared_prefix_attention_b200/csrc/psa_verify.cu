@@ -25,6 +25,10 @@
 #include "psa_internal.h"
 
 namespace psa {
+
+template <int D>
+int launch_combine_d(const VerifyArgs& a);
+
 namespace {
 
 constexpr int kTileKeys = 16;      // keys per pipeline stage
@@ -456,7 +460,16 @@ int launch_verify_d(const VerifyArgs& a, int HB, int MT, int NRB) {
     k1<<<grid, threads, smem, a.stream>>>(tk, tv, p1);
     if (cudaGetLastError() != cudaSuccess) return PSA_ERR_CUDA;
   }
+  return launch_combine_d<D>(a);
+}
 
+}  // namespace
+
+// Stage 2 on its own: merge the split partials of a.part_o / a.part_lse with
+// the causal draft block (shared with the shared-prefix verify).
+template <int D>
+int launch_combine_d(const VerifyArgs& a) {
+  const int G = a.Hq / a.Hkv;
   Stage2Params p2;
   p2.q = static_cast<const __nv_bfloat16*>(a.q);
   p2.kd = static_cast<const __nv_bfloat16*>(a.kd);
@@ -481,7 +494,18 @@ int launch_verify_d(const VerifyArgs& a, int HB, int MT, int NRB) {
   return PSA_OK;
 }
 
-}  // namespace
+int launch_verify_combine(const VerifyArgs& a) {
+  switch (a.D) {
+    case 64:
+      return launch_combine_d<64>(a);
+    case 128:
+      return launch_combine_d<128>(a);
+    case 256:
+      return launch_combine_d<256>(a);
+    default:
+      return PSA_ERR_UNSUPPORTED;
+  }
+}
 
 int verify_plan(int32_t Ld, int32_t Hq, int32_t Hkv, int32_t D, int32_t* heads_per_block,
                 int32_t* mtiles, int32_t* row_blocks) {

@@ -13,6 +13,8 @@ storage dtype):
   8 KV heads, d=128, bf16.
 * ``verify`` -- 32 requests, 16384-token cached prefix each, 4 draft tokens,
   32 query / 8 KV heads, d=128, 32 splits, bf16.
+* ``verify-shared`` -- the same 32 requests with 4 drafts each, all sharing
+  one 16384-token cached prefix stored once, 32/8 heads, d=128, bf16.
 * ``sparse`` -- 16384 queries, 64 heads on one 512-wide latent, 2048 indices
   per query drawn from its causal past, bf16.
 
@@ -199,6 +201,54 @@ class VerifyWorkload:
 
 
 @dataclass
+class SharedVerifyWorkload:
+    """Speculative verify where all B requests share one cached prefix of L
+    tokens (stored once) and each has Ld draft tokens."""
+    name: str
+    B: int
+    L: int
+    Ld: int
+    Hq: int
+    Hkv: int
+    d: int
+    nsplit: int = 0          # 0: the library's automatic choice
+    dtype: torch.dtype = torch.bfloat16
+    sigma: float = 0.5
+    seed: int = 6
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        """4 d FLOP per (draft row, query head, visible key): the whole
+        prefix plus drafts 0..j for draft j."""
+        keys = self.B * (self.Ld * self.L + self.Ld * (self.Ld + 1) // 2)
+        return 4.0 * self.d * self.Hq * keys
+
+    def prefix_kv_bytes(self) -> int:
+        """Prefix K and V bytes, read once for all requests."""
+        elem = torch.tensor([], dtype=self.dtype).element_size()
+        return self.L * self.Hkv * self.d * 2 * elem
+
+    def make(self, device="cpu", seed: int | None = None):
+        g = torch.Generator(device=device)
+        g.manual_seed(self.seed if seed is None else seed)
+        BL = self.B * self.Ld
+
+        def draw(shape):
+            x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+            return (x * self.sigma).to(self.dtype)
+
+        q = draw((BL, self.Hq, self.d))
+        kd = draw((BL, self.Hkv, self.d))
+        vd = draw((BL, self.Hkv, self.d))
+        kp = draw((self.L, self.Hkv, self.d))
+        vp = draw((self.L, self.Hkv, self.d))
+        return q, kd, vd, kp, vp
+
+
+@dataclass
 class SparseLatentWorkload:
     name: str
     T: int
@@ -265,5 +315,7 @@ LARGE = PrefillWorkload("large 2x(P=8192 N=16 S=1024) H=32/8 d=128 bf16", P=8192
                         S=1024, Hq=32, Hkv=8, d=128, groups=2, seed=3)
 VERIFY = VerifyWorkload("verify B=32 L=16384 drafts=4 H=32/8 d=128 splits=32 bf16", B=32,
                         L=16384, Ld=4, Hq=32, Hkv=8, d=128, nsplit=32, seed=4)
+VERIFY_SHARED = SharedVerifyWorkload("verify-shared B=32 L=16384 drafts=4 H=32/8 d=128 bf16",
+                                     B=32, L=16384, Ld=4, Hq=32, Hkv=8, d=128, seed=6)
 SPARSE = SparseLatentWorkload("sparse T=16384 H=64 dl=512 topk=2048 bf16", T=16384, H=64,
                               dl=512, topk=2048, seed=5)

@@ -77,6 +77,46 @@ def test_verify_host_validation():
     assert _verify_call(B=0) == psa.PSA_OK                           # nothing to do
 
 
+def _shared_call(**kw):
+    """psa_verify_shared_fwd with dummy (never dereferenced) pointers: every
+    case below is refused on the host before any CUDA call."""
+    a = dict(q=16, kd=16, vd=16, kp=16, vp=16, L=512, o=16, B=2, Ld=4, Hq=8, Hkv=2, d=128,
+             scale=0.1, nsplit=2, ws=None, wsb=0)
+    a.update(kw)
+    P = ctypes.c_void_p
+    return psa.lib().psa_verify_shared_fwd(
+        P(a["q"]), P(a["kd"]), P(a["vd"]), P(a["kp"]) if a["kp"] else None,
+        P(a["vp"]) if a["vp"] else None, a["L"], P(a["o"]), None, a["B"], a["Ld"], a["Hq"],
+        a["Hkv"], a["d"], a["scale"], a["nsplit"], P(a["ws"]) if a["ws"] else None, a["wsb"],
+        None, None)
+
+
+def test_verify_shared_host_validation():
+    assert _shared_call(d=256) == psa.PSA_ERR_UNSUPPORTED             # head dim
+    assert _shared_call(Hq=24, Hkv=1) == psa.PSA_ERR_UNSUPPORTED      # 24 rows per token
+    assert _shared_call(Hq=6, Hkv=4) == psa.PSA_ERR_INVALID_ARG       # Hq % Hkv
+    assert _shared_call(scale=0.0) == psa.PSA_ERR_INVALID_ARG
+    assert _shared_call(L=-1) == psa.PSA_ERR_INVALID_ARG
+    assert _shared_call(L=(1 << 30) + 1) == psa.PSA_ERR_INVALID_ARG
+    assert _shared_call(kp=None) == psa.PSA_ERR_INVALID_ARG            # prefix missing
+    assert _shared_call(q=8) == psa.PSA_ERR_INVALID_ARG                # misaligned
+    assert _shared_call(nsplit=257) == psa.PSA_ERR_INVALID_ARG
+    assert _shared_call(ws=None) == psa.PSA_ERR_WORKSPACE
+    need = psa.verify_workspace_size(2, 4, 8, 128, 2)
+    assert _shared_call(ws=256, wsb=need - 1) == psa.PSA_ERR_WORKSPACE
+    assert _shared_call(ws=8, wsb=need) == psa.PSA_ERR_WORKSPACE       # alignment
+    assert _shared_call(B=0) == psa.PSA_OK                             # nothing to do
+
+
+def test_verify_shared_auto_splits():
+    n = psa.verify_shared_auto_splits(32, 4, 32, 8, 16384)
+    assert 1 <= n <= 256
+    # about two (chunk, KV head, 256-row block) units per SM of a 148-SM part
+    assert n * 8 * 2 >= 148
+    assert psa.verify_shared_auto_splits(32, 4, 32, 8, 100) == 1     # short prefix
+    assert psa.verify_shared_auto_splits(1, 1, 1, 1, 1 << 20) <= 256
+
+
 def test_verify_workspace_size_formula():
     B, Ld, Hq, d, ns = 32, 4, 32, 128, 32
     rows = ns * B * Ld * Hq
