@@ -254,8 +254,9 @@ int psa_verify_fwd_noalloc(const void *q_draft, const void *k_draft, const void 
  *   sees the prefix plus drafts 0..j of its own request).
  * --------------------------------------------------------------------- */
 
-/* nsplit chosen by psa_verify_shared_fwd when it is passed 0: about two
- * units (chunk, KV head, 256 stacked rows) per SM, chunks of >= 512 keys. */
+/* nsplit chosen by psa_verify_shared_fwd when it is passed 0: as many
+ * units (chunk, KV head, 256 stacked rows) as fit one wave of 148 SMs,
+ * chunks of >= 512 keys. */
 int32_t psa_verify_shared_auto_splits(int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv,
                                       int64_t prefix_len);
 

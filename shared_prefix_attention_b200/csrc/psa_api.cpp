@@ -200,11 +200,12 @@ extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const vo
 extern "C" int32_t psa_verify_shared_auto_splits(int32_t B, int32_t Ld, int32_t Hq,
                                                  int32_t Hkv, int64_t prefix_len) {
   if (B <= 0 || Ld <= 0 || Hkv <= 0 || Hq <= 0 || prefix_len <= 0) return 1;
-  // Aim for about two units (chunk, KV head, 256-row block) per SM of a
-  // 148-SM part while keeping every chunk at least four 128-key tiles long.
+  // One wave of units (chunk, KV head, 256-row block) on a 148-SM part:
+  // a unit's fixed cost (Q load, epilogue) is high, so fewer, longer units
+  // beat more waves; every chunk keeps at least four 128-key tiles.
   const int64_t rows = int64_t(B) * Ld * (Hq / Hkv);
   const int64_t per_split = int64_t(Hkv) * ((rows + 255) / 256);
-  int64_t n = (2 * 148 + per_split - 1) / per_split;
+  int64_t n = 148 / per_split;
   const int64_t by_len = prefix_len / 512;
   if (n > by_len) n = by_len;
   if (n < 1) n = 1;

@@ -111,8 +111,9 @@ def test_verify_shared_host_validation():
 def test_verify_shared_auto_splits():
     n = psa.verify_shared_auto_splits(32, 4, 32, 8, 16384)
     assert 1 <= n <= 256
-    # about two (chunk, KV head, 256-row block) units per SM of a 148-SM part
-    assert n * 8 * 2 >= 148
+    # one wave of (chunk, KV head, 256-row block) units on a 148-SM part
+    units = n * 8 * 2
+    assert 74 < units <= 148
     assert psa.verify_shared_auto_splits(32, 4, 32, 8, 100) == 1     # short prefix
     assert psa.verify_shared_auto_splits(1, 1, 1, 1, 1 << 20) <= 256
 
