@@ -388,20 +388,29 @@ def time_steps(fn, steps: int, warmup: int, flush: torch.Tensor, dist_on: bool):
 
 
 def max_over_ranks(x: float, dist_on: bool) -> float:
+    """The slowest rank's time: every rank contributes its own and all get
+    the maximum (NCCL on the GPUs; gloo keeps the tensor on the host)."""
     if not dist_on:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    on_gpu = torch.distributed.get_backend() == "nccl"
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if on_gpu else "cpu")
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, work_per_rank: float, ms_max: float, unit: str) -> float:
+    """Weak scaling: every rank runs the same workload on its own GPU, so the
+    job does world x work in the slowest rank's time."""
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    return world * work_per_rank / (ms_max * 1e-3) / scale
 
 
 def measure(runner, steps, warmup, flush, dist_on, world, peaks):
     per = time_steps(runner.step, steps, warmup, flush, dist_on)
     ms = max_over_ranks(sum(per) / len(per), dist_on)
     work = runner.work()
-    scale = 1e12 if runner.unit == "TFLOP/s" else 1e9
-    value = world * work / (ms * 1e-3) / scale
-    per_gpu = work / (ms * 1e-3) / scale
+    value = job_throughput(world, work, ms, runner.unit)
+    per_gpu = job_throughput(1, work, ms, runner.unit)
     if runner.bound == "tensor":
         peak = peaks["bf16_tflops"]
         unit = "TFLOP/s"
@@ -473,8 +482,7 @@ def main():
         runner.e2e_setup()
         per = time_steps(runner.e2e_step, max(3, min(args.steps, 10)), 2, flush, dist_on)
         ems = max_over_ranks(sum(per) / len(per), dist_on)
-        scale = 1e12 if runner.unit == "TFLOP/s" else 1e9
-        out["e2e"] = {"value": round(world * runner.work() / (ems * 1e-3) / scale, 3),
+        out["e2e"] = {"value": round(job_throughput(world, runner.work(), ems, runner.unit), 3),
                       "unit": runner.unit, "ms_per_step": round(ems, 4),
                       "h2d_bytes_per_step": runner.h2d, "d2h_bytes_per_step": runner.d2h}
 
