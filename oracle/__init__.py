@@ -67,10 +67,13 @@ def load(path: str | None = None):
     lib.oracle_verify.argtypes = [P, P, P, P, P, P, I, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_verify_shared.argtypes = [P, P, P, P, P, ctypes.c_int64, I, I, I, I, I, D, P, I,
                                          P, P, I]
+    lib.oracle_verify_fp8.argtypes = [P, P, P, P, P, D, D, P, I, I, I, I, I, D, P, I, P, P, I]
+    lib.oracle_decode_e4m3.argtypes = [P, P, ctypes.c_int64]
     lib.oracle_sparse_latent.argtypes = [P, P, P, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_visibility.argtypes = [P, P, P, I, I, I, I, P]
     for f in (lib.oracle_prefill, lib.oracle_verify, lib.oracle_verify_shared,
-              lib.oracle_sparse_latent, lib.oracle_visibility):
+              lib.oracle_verify_fp8, lib.oracle_decode_e4m3, lib.oracle_sparse_latent,
+              lib.oracle_visibility):
         f.restype = I
     if path == _LIB_PATH:
         _lib = lib
@@ -181,6 +184,49 @@ def verify_shared(q_draft, k_draft, v_draft, k_prefix, v_prefix, Ld: int, scale:
                                   int(kp.shape[0]), B, Ld, Hq, Hkv, d, float(scale), _ptr(rows),
                                   len(rows), _ptr(o), _ptr(lse), nthreads or default_threads())
     assert rc == 0, "oracle_verify_shared rejected its arguments"
+    return o, lse
+
+
+def _u8(x):
+    if hasattr(x, "cpu"):
+        import torch
+        x = x.cpu()
+        if x.dtype != torch.uint8:
+            x = x.view(torch.uint8)
+        x = x.numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.uint8))
+
+
+def decode_e4m3(codes, lib=None):
+    """fp64 values of e4m3 bytes (any shape)."""
+    lib = lib or load()
+    c = _u8(codes)
+    out = np.zeros(c.shape, dtype=np.float64)
+    lib.oracle_decode_e4m3(_ptr(c), _ptr(out), c.size)
+    return out
+
+
+def verify_fp8(q_draft, k_draft, v_draft, k_cache8, v_cache8, k_scale: float, v_scale: float,
+               kv_indptr, Ld: int, scale: float, rows=None, nthreads: int | None = None,
+               lib=None):
+    """As verify, with e4m3 caches (uint8 or float8 tensors) standing for
+    k_scale * e4m3 and v_scale * e4m3."""
+    lib = lib or load()
+    qd, kd, vd = _f32(q_draft), _f32(k_draft), _f32(v_draft)
+    kc, vc = _u8(k_cache8), _u8(v_cache8)
+    indptr = np.ascontiguousarray(np.asarray(
+        kv_indptr.cpu().numpy() if hasattr(kv_indptr, "cpu") else kv_indptr, dtype=np.int64))
+    BL, Hq, d = qd.shape
+    Hkv = kd.shape[1]
+    B = BL // Ld
+    rows = np.arange(BL, dtype=np.int32) if rows is None else _i32(rows)
+    o = np.zeros((len(rows), Hq, d), dtype=np.float64)
+    lse = np.zeros((len(rows), Hq), dtype=np.float64)
+    rc = lib.oracle_verify_fp8(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kc), _ptr(vc), float(k_scale),
+                               float(v_scale), _ptr(indptr), B, Ld, Hq, Hkv, d, float(scale),
+                               _ptr(rows), len(rows), _ptr(o), _ptr(lse),
+                               nthreads or default_threads())
+    assert rc == 0, "oracle_verify_fp8 rejected its arguments"
     return o, lse
 
 

@@ -337,6 +337,100 @@ int oracle_verify_shared(const float *qd, const float *kd, const float *vd,
 }
 
 /* ------------------------------------------------------------------ */
+/* verify with an fp8 (e4m3) prefix cache and per-tensor scales         */
+/* ------------------------------------------------------------------ */
+
+/*
+ * "Split-KV flash-decode attention for EAGLE target-verify", implementation
+ * item 1 and the entry's signature: stage 1 reads the cached prefix and
+ * applies the fp8 scales k_scale / v_scale.  Reading: a cached key is
+ * k_scale * e4m3(byte), a cached value is v_scale * e4m3(byte); draft keys
+ * and values are not scaled.
+ *
+ * e4m3 (the "E4M3FN" variant): 1 sign bit, 4 exponent bits with bias 7,
+ * 3 mantissa bits; exponent field 0 holds subnormals m/8 * 2^-6; the codes
+ * S.1111.111 are NaN; there is no infinity.
+ */
+static double decode_e4m3(uint8_t b) {
+    int sgn = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+int oracle_decode_e4m3(const uint8_t *in, double *out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = decode_e4m3(in[i]);
+    return 0;
+}
+
+typedef struct {
+    const float *qd, *kd, *vd;
+    const uint8_t *kc, *vc;
+    const int64_t *indptr;
+    int Ld, Hq, Hkv, d;
+    double scale, kscale, vscale;
+    const int32_t *rows;
+    double *o, *lse;
+} verify8_ctx;
+
+static void verify8_row(void *p, int r, double *z, const float **vr, double *o) {
+    verify8_ctx *c = (verify8_ctx *)p;
+    (void)vr;
+    int row = c->rows[r]; /* row = b * Ld + j */
+    int b = row / c->Ld, j = row % c->Ld;
+    int64_t p0 = c->indptr[b], p1 = c->indptr[b + 1];
+    for (int h = 0; h < c->Hq; ++h) {
+        int kvh = kv_head_of(h, c->Hq, c->Hkv);
+        const float *qrow = c->qd + ((size_t)row * c->Hq + h) * c->d;
+        int n = 0;
+        for (int64_t t = p0; t < p1; ++t) { /* the whole cached prefix, scaled keys */
+            const uint8_t *krow = c->kc + ((size_t)t * c->Hkv + kvh) * c->d;
+            double sdot = 0.0;
+            for (int e = 0; e < c->d; ++e) sdot += (double)qrow[e] * decode_e4m3(krow[e]);
+            z[n++] = apply_scale(c->kscale * sdot, c->scale);
+        }
+        for (int i = 0; i <= j; ++i) {     /* drafts 0..j, unscaled */
+            const float *krow = c->kd + (((size_t)b * c->Ld + i) * c->Hkv + kvh) * c->d;
+            z[n++] = apply_scale(dot(qrow, krow, c->d), c->scale);
+        }
+        double m = -INFINITY, l = 0.0;
+        for (int i = 0; i < n; ++i) if (z[i] > m) m = z[i];
+        for (int i = 0; i < n; ++i) l += exp(z[i] - m);
+        for (int e = 0; e < c->d; ++e) o[e] = 0.0;
+        n = 0;
+        for (int64_t t = p0; t < p1; ++t) {
+            double w = exp(z[n++] - m) / l;
+            const uint8_t *vrow = c->vc + ((size_t)t * c->Hkv + kvh) * c->d;
+            for (int e = 0; e < c->d; ++e) o[e] += w * c->vscale * decode_e4m3(vrow[e]);
+        }
+        for (int i = 0; i <= j; ++i) {
+            double w = exp(z[n++] - m) / l;
+            const float *vrow = c->vd + (((size_t)b * c->Ld + i) * c->Hkv + kvh) * c->d;
+            for (int e = 0; e < c->d; ++e) o[e] += w * (double)vrow[e];
+        }
+        memcpy(c->o + ((size_t)r * c->Hq + h) * c->d, o, sizeof(double) * (size_t)c->d);
+        c->lse[(size_t)r * c->Hq + h] = m + log(l);
+    }
+}
+
+/* As oracle_verify, with k_cache / v_cache holding e4m3 bytes that stand
+ * for k_scale * e4m3 and v_scale * e4m3. */
+int oracle_verify_fp8(const float *qd, const float *kd, const float *vd,
+                      const uint8_t *kc, const uint8_t *vc, double kscale, double vscale,
+                      const int64_t *indptr, int B, int Ld, int Hq, int Hkv, int d,
+                      double scale, const int32_t *rows, int nrows, double *o, double *lse,
+                      int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || B < 0 || Ld <= 0) return -1;
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b)
+        if (indptr[b + 1] - indptr[b] > maxlen) maxlen = indptr[b + 1] - indptr[b];
+    verify8_ctx c = {qd, kd, vd, kc, vc, indptr, Ld, Hq, Hkv, d, scale, kscale, vscale,
+                     rows, o, lse};
+    run_rows(verify8_row, &c, nrows, (int)maxlen + Ld, d, nthreads);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* shared-latent sparse attention over per-query index lists            */
 /* ------------------------------------------------------------------ */
 

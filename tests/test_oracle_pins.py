@@ -332,10 +332,53 @@ def pin_verify_shared_prefix(lib):
     return bool(ok)
 
 
+def pin_e4m3_decoder(lib):
+    """The e4m3 decoder behind the fp8 verify (the split-KV verify page's fp8
+    cache scaling) agrees with torch's float8_e4m3fn on all 256 codes."""
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.decode_e4m3(codes, lib=lib)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    nan = np.isnan(ref)
+    return bool(np.array_equal(np.isnan(mine), nan) and np.array_equal(mine[~nan], ref[~nan]))
+
+
+def pin_verify_fp8_cache(lib):
+    """[SKV] implementation item 1 (stage 1 applies the fp8 scales): a cached
+    key is k_scale * e4m3, a cached value v_scale * e4m3, drafts are not
+    scaled.  Checked against torch SDPA fp64 on the decoded, scaled cache,
+    and, with power-of-two scales, against the float verify on that cache."""
+    q, kd, vd, kc, vc, indptr, Ld = _verify_case(seed=71)
+    Hq, d = q.shape[1], q.shape[2]
+    scale = 1 / math.sqrt(d)
+    ok = True
+    for ks, vs in ((0.37, 1.9), (0.25, 2.0)):
+        kc8 = (kc / ks).to(torch.float8_e4m3fn)
+        vc8 = (vc / vs).to(torch.float8_e4m3fn)
+        o, lse = oracle.verify_fp8(q, kd, vd, kc8, vc8, ks, vs, indptr, Ld, scale, lib=lib)
+        kr = torch.from_numpy(oracle.decode_e4m3(kc8, lib=lib) * ks)
+        vr = torch.from_numpy(oracle.decode_e4m3(vc8, lib=lib) * vs)
+        for b in range(len(indptr) - 1):
+            p0, p1 = int(indptr[b]), int(indptr[b + 1])
+            keys = torch.cat([kr[p0:p1], kd[b * Ld:(b + 1) * Ld].double()])
+            vals = torch.cat([vr[p0:p1], vd[b * Ld:(b + 1) * Ld].double()])
+            L = p1 - p0
+            mask = torch.ones((Ld, L + Ld), dtype=torch.bool)
+            mask[:, L:] = torch.tril(torch.ones((Ld, Ld), dtype=torch.bool))
+            ref = _sdpa(q[b * Ld:(b + 1) * Ld], _expand_kv(keys, Hq), _expand_kv(vals, Hq),
+                        mask, scale)
+            ok &= np.allclose(o[b * Ld:(b + 1) * Ld], ref, atol=1e-12)
+        if ks == 0.25:
+            o2, lse2 = oracle.verify(q, kd, vd, kr.float(), vr.float(), indptr, Ld, scale,
+                                     lib=lib)
+            ok &= np.allclose(o, o2, atol=1e-12) and np.allclose(lse, lse2, atol=1e-12)
+    return bool(ok)
+
+
 PINS = [pin_golden_masks, pin_golden_tiny_attention, pin_equivalence_route,
         pin_sdpa_random_trees, pin_closed_forms, pin_special_cases,
         pin_brute_force_python, pin_verify_against_sdpa, pin_split_identity,
-        pin_verify_shared_prefix, pin_sparse_latent]
+        pin_verify_shared_prefix, pin_e4m3_decoder, pin_verify_fp8_cache,
+        pin_sparse_latent]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
