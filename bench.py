@@ -318,6 +318,35 @@ class SparseRunner(Runner):
                                lse=self.lse)
 
 
+class VerifyFp8Runner(Runner):
+    """Split-KV verify over an e4m3 prefix cache: HBM-bound on the cache bytes
+    (one byte per element)."""
+    unit = "GB/s"
+    bound = "hbm"
+    kernels_per_step = 2
+    kernel_file = "psa_verify_fp8.cu"
+
+    def __init__(self, wl: W.VerifyWorkload, dev):
+        import shared_prefix_attention_b200 as psa
+        self.psa, self.wl, self.dev = psa, wl, dev
+        self.name = wl.name
+        self.q, self.kd, self.vd, self.kc8, self.vc8 = wl.make_fp8(dev)
+        self.indptr = torch.tensor(wl.kv_indptr(), dtype=torch.int32, device=dev)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=dev)
+        n = psa.verify_workspace_size(wl.B, wl.Ld, wl.Hq, wl.d, wl.nsplit)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+
+    def work(self):
+        return float(self.wl.prefix_fp8_bytes())
+
+    def step(self):
+        wl = self.wl
+        self.psa.verify_fp8(self.q, self.kd, self.vd, self.kc8, self.vc8, wl.k_scale, wl.v_scale,
+                            self.indptr, wl.L, wl.scale, wl.Ld, nsplit=wl.nsplit, out=self.o,
+                            lse=self.lse, workspace=self.ws)
+
+
 class SharedVerifyRunner(Runner):
     """Verify against one prefix shared by all requests: tensor-bound (the
     stacked draft rows of a KV head multiply the prefix once)."""
@@ -360,6 +389,7 @@ def make_runner(name: str, dev):
             "large": lambda: PrefillRunner(W.LARGE, dev),
             "verify": lambda: VerifyRunner(W.VERIFY, dev),
             "verify-shared": lambda: SharedVerifyRunner(W.VERIFY_SHARED, dev),
+            "verify-fp8": lambda: VerifyFp8Runner(W.VERIFY_FP8, dev),
             "sparse": lambda: SparseRunner(W.SPARSE, dev)}[name]()
 
 
@@ -437,7 +467,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="grpo",
                     choices=["grpo", "tiny", "large", "verify", "verify8", "verify-shared",
-                             "sparse", "sparse4k"])
+                             "verify-fp8", "sparse", "sparse4k"])
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -488,7 +518,7 @@ def main():
 
     if not args.no_extras and args.workload == "grpo":
         extras = {}
-        for name in ("verify", "verify-shared", "large", "sparse"):
+        for name in ("verify", "verify-fp8", "verify-shared", "large", "sparse"):
             try:
                 r = make_runner(name, dev)
                 v, m, rf = measure(r, max(3, min(args.steps, 10)), 3, flush, dist_on, world,

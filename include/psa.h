@@ -247,6 +247,28 @@ int psa_verify_fwd_noalloc(const void *q_draft, const void *k_draft, const void 
                            int32_t nsplit, const psa_verify_features *features,
                            int32_t *dev_status, void *stream);
 
+/*
+ * psa_verify_fwd with an fp8 prefix cache ([SKV] implementation item 1:
+ * stage 1 applies the fp8 scales k_scale / v_scale of the cache).
+ *   k_cache, v_cache device [Ntok, Hkv, d] e4m3 bytes ("E4M3FN": bias 7,
+ *                    3 mantissa bits, no infinities); a cached key stands for
+ *                    k_scale * e4m3, a cached value for v_scale * e4m3
+ *   k_scale, v_scale host values, finite and > 0
+ * Draft keys and values stay bf16 and are not scaled.  Every other argument,
+ * layout and status is that of psa_verify_fwd, except that head_dim must be
+ * 128 (PSA_ERR_UNSUPPORTED otherwise).  The prefix read is half the bytes of
+ * the bf16 cache.  Q is widened to f16 for the tensor cores: |q| must stay
+ * below 65504.
+ */
+int psa_verify_fp8_fwd(const void *q_draft, const void *k_draft, const void *v_draft,
+                       const void *k_cache, const void *v_cache, int64_t n_cache_tokens,
+                       const int32_t *dev_kv_indptr, int64_t max_prefix_len,
+                       const int32_t *kv_indices, float k_scale, float v_scale, void *o,
+                       float *lse, int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv,
+                       int32_t head_dim, float scale, int32_t nsplit,
+                       const psa_verify_features *features, void *workspace, size_t ws_bytes,
+                       int32_t *dev_status, void *stream);
+
 /* ------------------------------------------------------------------------
  * Speculative verify against one prefix shared by every request.
  *   [PS] design summary (the prefix K/V is stored once and every sequence

@@ -32,6 +32,7 @@ EXPORTS = [
     "psa_prefill_fwd", "psa_verify_auto_splits", "psa_verify_workspace_size",
     "psa_verify_fwd", "psa_verify_fwd_noalloc", "psa_sparse_latent_fwd", "psa_read_status",
     "psa_wait_selftest", "psa_verify_shared_auto_splits", "psa_verify_shared_fwd",
+    "psa_verify_fp8_fwd",
 ]
 
 
@@ -92,6 +93,8 @@ def lib():
         "psa_read_status": ([P, P, P], ctypes.c_int),
         "psa_wait_selftest": ([I32, P, P], ctypes.c_int),
         "psa_verify_shared_auto_splits": ([I32, I32, I32, I32, I64], I32),
+        "psa_verify_fp8_fwd": ([P, P, P, P, P, I64, P, I64, P, F, F, P, P, I32, I32, I32, I32,
+                                I32, F, I32, P, P, SZ, P, P], ctypes.c_int),
         "psa_verify_shared_fwd": ([P, P, P, P, P, I64, P, P, I32, I32, I32, I32, I32, F, I32, P,
                                    ctypes.c_size_t, P, P], ctypes.c_int),
     }
@@ -318,4 +321,29 @@ def verify_shared(q_draft, k_draft, v_draft, k_prefix, v_prefix, scale: float, L
                                      Ld, Hq, Hkv, d, float(scale), ns, _ptr(workspace),
                                      workspace.numel(), _ptr(status), _stream(q_draft.device))
     _check(rc, "psa_verify_shared_fwd")
+    return out, lse
+
+
+def verify_fp8(q_draft, k_draft, v_draft, k_cache8, v_cache8, k_scale: float, v_scale: float,
+               kv_indptr: torch.Tensor, max_prefix_len: int, scale: float, Ld: int,
+               nsplit: int = 0, out=None, lse=None, workspace=None, status=None):
+    """Split-KV verify over an e4m3 prefix cache (uint8 or float8_e4m3fn
+    tensors [Ntok, Hkv, d]) standing for k_scale * e4m3 and v_scale * e4m3."""
+    _require_cuda(q_draft, k_draft, v_draft, k_cache8, v_cache8, kv_indptr)
+    BL, Hq, d = q_draft.shape
+    Hkv = k_draft.shape[1]
+    B = BL // Ld
+    ns = nsplit or verify_auto_splits(B, max_prefix_len, Hkv, d)
+    out = torch.empty_like(q_draft) if out is None else out
+    lse = torch.empty((BL, Hq), dtype=torch.float32, device=q_draft.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(max(verify_workspace_size(B, Ld, Hq, d, ns), 256),
+                                dtype=torch.uint8, device=q_draft.device)
+    rc = lib().psa_verify_fp8_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft), _ptr(k_cache8),
+                                  _ptr(v_cache8), k_cache8.shape[0], _ptr(kv_indptr),
+                                  int(max_prefix_len), None, float(k_scale), float(v_scale),
+                                  _ptr(out), _ptr(lse), B, Ld, Hq, Hkv, d, float(scale), ns, None,
+                                  _ptr(workspace), workspace.numel(), _ptr(status),
+                                  _stream(q_draft.device))
+    _check(rc, "psa_verify_fp8_fwd")
     return out, lse

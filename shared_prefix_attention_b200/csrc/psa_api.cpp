@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -193,6 +194,69 @@ extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const vo
   a.status = dev_status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_verify(a);
+}
+
+extern "C" int psa_verify_fp8_fwd(const void* q_draft, const void* k_draft, const void* v_draft,
+                                  const void* k_cache, const void* v_cache,
+                                  int64_t n_cache_tokens, const int32_t* dev_kv_indptr,
+                                  int64_t max_prefix_len, const int32_t* kv_indices,
+                                  float k_scale, float v_scale, void* o, float* lse, int32_t B,
+                                  int32_t Ld, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                                  float scale, int32_t nsplit,
+                                  const psa_verify_features* features, void* workspace,
+                                  size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (features) {
+    if (features->has_custom_mask || !features->is_causal || features->sliding_window > 0 ||
+        features->has_sinks || features->logit_cap != 0.f ||
+        features->xai_temperature_len > 0 || features->ragged_extend)
+      return PSA_ERR_UNSUPPORTED;
+  }
+  if (kv_indices) return PSA_ERR_UNSUPPORTED;
+  if (B < 0 || Ld <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n_cache_tokens < 0 ||
+      max_prefix_len < 0 || n_cache_tokens > INT32_MAX || !(scale > 0.f) ||
+      !(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return PSA_ERR_INVALID_ARG;
+  if (head_dim != 128) return PSA_ERR_UNSUPPORTED;
+  if (B == 0) return PSA_OK;
+  if (!q_draft || !k_draft || !v_draft || !k_cache || !v_cache || !dev_kv_indptr || !o)
+    return PSA_ERR_INVALID_ARG;
+  if (!aligned16(q_draft) || !aligned16(k_draft) || !aligned16(v_draft) ||
+      !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return PSA_ERR_INVALID_ARG;
+  int32_t HB = 0, MT = 0, NRB = 0;
+  if (!verify_plan(Ld, Hq, Hkv, head_dim, &HB, &MT, &NRB)) return PSA_ERR_UNSUPPORTED;
+  if (nsplit == 0) nsplit = psa_verify_auto_splits(B, max_prefix_len, Hkv, head_dim);
+  if (nsplit < 1 || nsplit > 256) return PSA_ERR_INVALID_ARG;
+  const size_t need = psa_verify_workspace_size(B, Ld, Hq, head_dim, nsplit);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PSA_ERR_WORKSPACE;
+  if (n_cache_tokens == 0) n_cache_tokens = 1;  // a tensor map needs a non-empty extent
+
+  VerifyArgs a;
+  a.q = q_draft;
+  a.kd = k_draft;
+  a.vd = v_draft;
+  a.kc = k_cache;
+  a.vc = v_cache;
+  a.indptr = dev_kv_indptr;
+  a.n_cache_tokens = n_cache_tokens;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.Ld = Ld;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = head_dim;
+  a.scale = scale;
+  a.nsplit = nsplit;
+  const size_t rows = size_t(nsplit) * B * Ld * Hq;
+  const size_t o_bytes = (rows * head_dim * sizeof(float) + 255) / 256 * 256;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + o_bytes);
+  a.status = dev_status;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_verify_fp8(a, k_scale, v_scale);
 }
 
 // ------------------------------------------------------- shared-prefix verify

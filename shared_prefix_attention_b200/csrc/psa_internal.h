@@ -48,6 +48,9 @@ int verify_plan(int32_t Ld, int32_t Hq, int32_t Hkv, int32_t D, int32_t* heads_p
 int launch_verify(const VerifyArgs& a);
 // Stage 2 alone: merge a.nsplit partials with the causal draft block.
 int launch_verify_combine(const VerifyArgs& a);
+// The verify with e4m3 caches in a.kc / a.vc (head_dim 128): cached key =
+// k_scale * e4m3, cached value = v_scale * e4m3.
+int launch_verify_fp8(const VerifyArgs& a, float k_scale, float v_scale);
 
 // Verify against one prefix shared by every request.
 struct VerifySharedArgs {

@@ -13,6 +13,8 @@ storage dtype):
   8 KV heads, d=128, bf16.
 * ``verify`` -- 32 requests, 16384-token cached prefix each, 4 draft tokens,
   32 query / 8 KV heads, d=128, 32 splits, bf16.
+* ``verify-fp8`` -- the verify workload with the cached prefix stored as e4m3
+  codes and per-tensor scales k_scale = 1/96, v_scale = 1/80.
 * ``verify-shared`` -- the same 32 requests with 4 drafts each, all sharing
   one 16384-token cached prefix stored once, 32/8 heads, d=128, bf16.
 * ``sparse`` -- 16384 queries, 64 heads on one 512-wide latent, 2048 indices
@@ -199,6 +201,22 @@ class VerifyWorkload:
         vc = draw((ntok, self.Hkv, self.d))
         return q, kd, vd, kc, vc
 
+    # per-tensor scales of the fp8 cache: stored codes are value / scale
+    k_scale: float = 1.0 / 96
+    v_scale: float = 1.0 / 80
+
+    def make_fp8(self, device="cpu", seed: int | None = None):
+        """As make(), with the cached prefix stored as e4m3 codes (uint8) of
+        value / k_scale and value / v_scale (round to nearest)."""
+        q, kd, vd, kc, vc = self.make(device, seed)
+        kc8 = (kc.float() / self.k_scale).to(torch.float8_e4m3fn).view(torch.uint8)
+        vc8 = (vc.float() / self.v_scale).to(torch.float8_e4m3fn).view(torch.uint8)
+        return q, kd, vd, kc8, vc8
+
+    def prefix_fp8_bytes(self) -> int:
+        """Prefix K and V bytes of the e4m3 cache, read once."""
+        return sum(self.lens()) * self.Hkv * self.d * 2
+
 
 @dataclass
 class SharedVerifyWorkload:
@@ -315,6 +333,8 @@ LARGE = PrefillWorkload("large 2x(P=8192 N=16 S=1024) H=32/8 d=128 bf16", P=8192
                         S=1024, Hq=32, Hkv=8, d=128, groups=2, seed=3)
 VERIFY = VerifyWorkload("verify B=32 L=16384 drafts=4 H=32/8 d=128 splits=32 bf16", B=32,
                         L=16384, Ld=4, Hq=32, Hkv=8, d=128, nsplit=32, seed=4)
+VERIFY_FP8 = VerifyWorkload("verify-fp8 B=32 L=16384 drafts=4 H=32/8 d=128 splits=32 e4m3 cache",
+                            B=32, L=16384, Ld=4, Hq=32, Hkv=8, d=128, nsplit=32, seed=7)
 VERIFY_SHARED = SharedVerifyWorkload("verify-shared B=32 L=16384 drafts=4 H=32/8 d=128 bf16",
                                      B=32, L=16384, Ld=4, Hq=32, Hkv=8, d=128, seed=6)
 SPARSE = SparseLatentWorkload("sparse T=16384 H=64 dl=512 topk=2048 bf16", T=16384, H=64,

@@ -118,6 +118,21 @@ def test_verify_shared_auto_splits():
     assert psa.verify_shared_auto_splits(1, 1, 1, 1, 1 << 20) <= 256
 
 
+def test_verify_fp8_host_validation():
+    P = ctypes.c_void_p
+
+    def call(d=128, ks=0.1, vs=0.1, B=1, kvi=None):
+        return psa.lib().psa_verify_fp8_fwd(P(16), P(16), P(16), P(16), P(16), 64, P(16), 64,
+                                            P(kvi) if kvi else None, ks, vs, P(16), None, B, 4,
+                                            8, 2, d, 0.1, 1, None, None, 0, None, None)
+    assert call(d=64) == psa.PSA_ERR_UNSUPPORTED       # e4m3 path is head_dim 128 only
+    assert call(kvi=16) == psa.PSA_ERR_UNSUPPORTED     # paged cache
+    assert call(ks=0.0) == psa.PSA_ERR_INVALID_ARG
+    assert call(vs=float("inf")) == psa.PSA_ERR_INVALID_ARG
+    assert call() == psa.PSA_ERR_WORKSPACE
+    assert call(B=0) == psa.PSA_OK
+
+
 def test_verify_workspace_size_formula():
     B, Ld, Hq, d, ns = 32, 4, 32, 128, 32
     rows = ns * B * Ld * Hq
