@@ -12,9 +12,10 @@
 // (KV head, 16-row m-tile) doing warp-level MMAs) with three changes:
 //   - the ring holds e4m3 tiles (128 bytes per key and head, 128-byte
 //     swizzle);
-//   - each consumer warp widens its head's K and V tile to f16 (exact for
-//     e4m3) in a private shared-memory tile laid out like the bf16 path's,
-//     releases the ring slot at once, and runs the f16 warp MMAs on it;
+//   - each consumer warp reads its K fragments straight from the e4m3 tile
+//     (two bytes per register, widened to f16 in registers, exact for e4m3)
+//     and widens its head's V tile into a private f16 tile laid out like the
+//     bf16 path's, so ldmatrix.trans can feed the PV warp MMAs;
 //   - k_scale is folded into the logit scale and v_scale into the partial
 //     output, so the inner loop never multiplies by a scale.
 // Q is widened from bf16 to f16 for the f16 MMAs (exact for |q| < 65504 and
@@ -34,7 +35,7 @@ constexpr int D8 = 128;           // head dim of the fp8 path (one swizzle atom 
 constexpr int kKeys = 16;         // keys per ring stage
 constexpr int kMaxWarps = 8;      // consumer warps per CTA
 constexpr uint32_t kHeadTile8 = kKeys * D8;        // e4m3 bytes of one head's K (or V) tile
-constexpr uint32_t kPrivBytes = 2 * 2 * kKeys * 128;  // f16 K and V tiles, two d-parts each
+constexpr uint32_t kPrivBytes = 2 * kKeys * 128;  // f16 V tile, two d-parts
 
 struct P8Params {
   const __nv_bfloat16* q;  // [B*Ld, Hq, D]
@@ -206,8 +207,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32, 1)
   const int mt = warp % p.MT;  // 16-row m-tile of that head's rows
   const int g = lane >> 2, c = lane & 3;
   const int BL = p.B * p.Ld;
-  const uint32_t kpriv = smem_u32(priv + warp * kPrivBytes);
-  const uint32_t vpriv = kpriv + kPrivBytes / 2;
+  const uint32_t vpriv = smem_u32(priv + warp * kPrivBytes);
   int stage = 0;
   uint32_t phase = 0;
 
@@ -257,37 +257,33 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32, 1)
         ok = false;
         break;
       }
-      {
-        // widen this head's K and V tile into the warp's private f16 tiles,
-        // then hand the ring slot back
-        const uint32_t k8 = smem_u32(smem + stage * stage_bytes) + hh * kHeadTile8;
-        const uint32_t v8 = k8 + kv_bytes;
-        const int key = lane >> 1, half = lane & 1;
-        widen_row(k8, kpriv, key, half);
-        widen_row(v8, vpriv, key, half);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[stage]);
-        if (++stage == p.nstage) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
+      const uint32_t k8 = smem_u32(smem + stage * stage_bytes) + hh * kHeadTile8;
+      // widen this head's V tile into the warp's private f16 tile (the PV
+      // operand needs it transposed, which ldmatrix.trans does on 16-bit data)
+      widen_row(k8 + kv_bytes, vpriv, lane >> 1, lane & 1);
 
-      // S = Q K^T over 16 keys: two n-tiles of 8 keys
+      // S = Q K^T over 16 keys: two n-tiles of 8 keys; the B fragments come
+      // straight from the e4m3 tile: key g, d = 16 ks + 2c (+1) and + 8 (+9)
       float sc[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-        const uint32_t key = nt * 8 + (lane & 7);
+        const uint32_t key = nt * 8 + g;
 #pragma unroll
-        for (int ks = 0; ks < KSTEPS; ks += 2) {
-          const uint32_t chunk = ks * 2 + (lane >> 3);
-          const uint32_t addr = kpriv + (chunk >> 3) * (kKeys * 128) + sw128(key, chunk & 7);
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4(addr, b0, b1, b2, b3);
-          mma_f16_16816(sc[nt], qa[ks], b0, b1);
-          mma_f16_16816(sc[nt], qa[ks + 1], b2, b3);
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          const uint32_t addr = k8 + sw128(key, ks) + 2 * c;
+          uint32_t x0, x1;
+          asm volatile("ld.shared.u16 %0, [%1];" : "=r"(x0) : "r"(addr));
+          asm volatile("ld.shared.u16 %0, [%1];" : "=r"(x1) : "r"(addr + 8));
+          mma_f16_16816(sc[nt], qa[ks], e4m3x2_to_f16x2(x0), e4m3x2_to_f16x2(x1));
         }
+      }
+      // the e4m3 tile is no longer needed: hand the ring slot back
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (++stage == p.nstage) {
+        stage = 0;
+        phase ^= 1;
       }
 
       // online softmax in the log2 domain; keys past the split end are masked
