@@ -65,13 +65,15 @@ def load(path: str | None = None):
     D = ctypes.c_double
     lib.oracle_prefill.argtypes = [P, P, P, I, I, I, I, D, P, P, P, I, P, I, P, P, I]
     lib.oracle_verify.argtypes = [P, P, P, P, P, P, I, I, I, I, I, D, P, I, P, P, I]
+    lib.oracle_prefill_bwd.argtypes = [P, P, P, P, I, I, I, I, D, P, P, P, I, P, P, P, I]
     lib.oracle_verify_shared.argtypes = [P, P, P, P, P, ctypes.c_int64, I, I, I, I, I, D, P, I,
                                          P, P, I]
     lib.oracle_verify_fp8.argtypes = [P, P, P, P, P, D, D, P, I, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_decode_e4m3.argtypes = [P, P, ctypes.c_int64]
     lib.oracle_sparse_latent.argtypes = [P, P, P, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_visibility.argtypes = [P, P, P, I, I, I, I, P]
-    for f in (lib.oracle_prefill, lib.oracle_verify, lib.oracle_verify_shared,
+    for f in (lib.oracle_prefill, lib.oracle_prefill_bwd, lib.oracle_verify,
+              lib.oracle_verify_shared,
               lib.oracle_verify_fp8, lib.oracle_decode_e4m3, lib.oracle_sparse_latent,
               lib.oracle_visibility):
         f.restype = I
@@ -144,6 +146,24 @@ def prefill(q, k, v, segments, scale: float, rows=None, nthreads: int | None = N
                             nthreads or default_threads())
     assert rc == 0, "oracle_prefill rejected its arguments"
     return o, lse
+
+
+def prefill_bwd(q, k, v, dout, segments, scale: float, nthreads: int | None = None, lib=None):
+    """Gradients (dq [T, Hq, d], dk, dv [T, Hkv, d], fp64) of the prefill
+    output O with upstream gradient dout [T, Hq, d]."""
+    lib = lib or load()
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(dout)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    start, lens, parent = segment_arrays(segments)
+    dq = np.zeros((T, Hq, d), dtype=np.float64)
+    dk = np.zeros((T, Hkv, d), dtype=np.float64)
+    dv = np.zeros((T, Hkv, d), dtype=np.float64)
+    rc = lib.oracle_prefill_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), T, Hq, Hkv, d, float(scale),
+                                _ptr(start), _ptr(lens), _ptr(parent), len(lens), _ptr(dq),
+                                _ptr(dk), _ptr(dv), nthreads or default_threads())
+    assert rc == 0, "oracle_prefill_bwd rejected its arguments"
+    return dq, dk, dv
 
 
 def verify(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr, Ld: int,

@@ -251,6 +251,118 @@ int oracle_prefill(const float *q, const float *k, const float *v, int T, int Hq
 }
 
 /* ------------------------------------------------------------------ */
+/* backward of the prefill: gradients of O = softmax(scale Q K^T) V      */
+/* ------------------------------------------------------------------ */
+
+/*
+ * "KV-0 redundancy prefix sharing attention mask design", design summary and
+ * test plan: the flat layout must give the same gradients as running every
+ * [prefix; s_i] on its own, so the prefix K/V collect the gradients of all
+ * suffixes that see them.  Written out from the definition of softmax
+ * attention for one query row q with visible keys k:
+ *   P_k = softmax_k(scale q.k_k), O = sum_k P_k v_k, D = dO . O,
+ *   dV_k += P_k dO, dP_k = dO . v_k, dS_k = P_k (dP_k - D),
+ *   dQ += scale sum_k dS_k k_k, dK_k += scale dS_k q.
+ * A query head h contributes to KV head h / (Hq / Hkv).
+ */
+typedef struct {
+    const float *q, *k, *v, *dout;
+    int T, Hq, Hkv, d;
+    double scale;
+    const int32_t *tok_seg, *parent;
+    double *dq, *dk, *dv;
+    int kvh0, kvh1;
+} bwd_ctx;
+
+static void *bwd_worker(void *p) {
+    bwd_ctx *c = (bwd_ctx *)p;
+    int G = c->Hq / c->Hkv, d = c->d, T = c->T;
+    double *z = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    int32_t *ks = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1));
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int kvh = c->kvh0; kvh < c->kvh1; ++kvh) {
+        for (int g = 0; g < G; ++g) {
+            int h = kvh * G + g;
+            for (int qi = 0; qi < T; ++qi) {
+                const float *qrow = c->q + ((size_t)qi * c->Hq + h) * d;
+                const float *dorow = c->dout + ((size_t)qi * c->Hq + h) * d;
+                int n = 0;
+                for (int kj = 0; kj < T; ++kj) {
+                    if (!visible(c->tok_seg, c->parent, qi, kj)) continue;
+                    const float *krow = c->k + ((size_t)kj * c->Hkv + kvh) * d;
+                    z[n] = c->scale * dot(qrow, krow, d);
+                    ks[n++] = kj;
+                }
+                if (n == 0) continue;
+                double m = -INFINITY, l = 0.0;
+                for (int i = 0; i < n; ++i) if (z[i] > m) m = z[i];
+                for (int i = 0; i < n; ++i) { z[i] = exp(z[i] - m); l += z[i]; }
+                for (int i = 0; i < n; ++i) z[i] /= l; /* z now holds P */
+                for (int e = 0; e < d; ++e) o[e] = 0.0;
+                for (int i = 0; i < n; ++i) {
+                    const float *vrow = c->v + ((size_t)ks[i] * c->Hkv + kvh) * d;
+                    for (int e = 0; e < d; ++e) o[e] += z[i] * (double)vrow[e];
+                }
+                double D = 0.0;
+                for (int e = 0; e < d; ++e) D += (double)dorow[e] * o[e];
+                double *dqrow = c->dq + ((size_t)qi * c->Hq + h) * d;
+                for (int i = 0; i < n; ++i) {
+                    const float *krow = c->k + ((size_t)ks[i] * c->Hkv + kvh) * d;
+                    const float *vrow = c->v + ((size_t)ks[i] * c->Hkv + kvh) * d;
+                    double dp = dot(dorow, vrow, d);
+                    double dsc = z[i] * (dp - D);
+                    double *dkrow = c->dk + ((size_t)ks[i] * c->Hkv + kvh) * d;
+                    double *dvrow = c->dv + ((size_t)ks[i] * c->Hkv + kvh) * d;
+                    for (int e = 0; e < d; ++e) {
+                        dqrow[e] += c->scale * dsc * (double)krow[e];
+                        dkrow[e] += c->scale * dsc * (double)qrow[e];
+                        dvrow[e] += z[i] * (double)dorow[e];
+                    }
+                }
+            }
+        }
+    }
+    free(z);
+    free(ks);
+    free(o);
+    return NULL;
+}
+
+/*
+ * q, dout [T, Hq, d]; k, v [T, Hkv, d] (fp32 holding the exact input values);
+ * segments as for oracle_prefill.  dq [T, Hq, d], dk, dv [T, Hkv, d] (fp64,
+ * written).  Threads split the KV heads, so no two threads write one output.
+ */
+int oracle_prefill_bwd(const float *q, const float *k, const float *v, const float *dout,
+                       int T, int Hq, int Hkv, int d, double scale,
+                       const int32_t *seg_start, const int32_t *seg_len,
+                       const int32_t *parent, int nseg, double *dq, double *dk, double *dv,
+                       int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || T < 0) return -1;
+    int32_t *tok_seg = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1));
+    if (!tok_seg) return -1;
+    token_segments(seg_start, seg_len, nseg, T, tok_seg);
+    memset(dq, 0, sizeof(double) * (size_t)T * Hq * d);
+    memset(dk, 0, sizeof(double) * (size_t)T * Hkv * d);
+    memset(dv, 0, sizeof(double) * (size_t)T * Hkv * d);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > Hkv) nthreads = Hkv;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    bwd_ctx *cs = (bwd_ctx *)malloc(sizeof(bwd_ctx) * (size_t)nthreads);
+    for (int i = 0; i < nthreads; ++i) {
+        bwd_ctx c = {q, k, v, dout, T, Hq, Hkv, d, scale, tok_seg, parent, dq, dk, dv,
+                     Hkv * i / nthreads, Hkv * (i + 1) / nthreads};
+        cs[i] = c;
+        pthread_create(&th[i], NULL, bwd_worker, &cs[i]);
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th);
+    free(cs);
+    free(tok_seg);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* speculative verify: cached prefix plus a causal draft block          */
 /* ------------------------------------------------------------------ */
 

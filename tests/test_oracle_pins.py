@@ -374,11 +374,78 @@ def pin_verify_fp8_cache(lib):
     return bool(ok)
 
 
+def pin_backward_finite_differences(lib):
+    """The backward is the derivative of the forward: central differences of
+    L = sum(O * G) through the fp64 forward oracle, every input element of a
+    small two-level tree (GQA 2:1), match dq, dk, dv."""
+    segs = [(5, -1), (3, 0), (4, 0), (2, 1)]
+    T, Hq, Hkv, d = 14, 2, 1, 3
+    q, k, v = _rand((T, Hq, d), 81), _rand((T, Hkv, d), 82), _rand((T, Hkv, d), 83)
+    G = _rand((T, Hq, d), 84).double().numpy()
+    scale = 0.7
+    dq, dk, dv = oracle.prefill_bwd(q, k, v, torch.from_numpy(G).float(), segs, scale, lib=lib)
+    # G is rounded to fp32 by the call; use the same values for the loss
+    G = torch.from_numpy(G).float().double().numpy()
+    eps = 1e-2
+
+    def loss(qq, kk, vv):
+        o, _ = oracle.prefill(qq, kk, vv, segs, scale, lib=lib)
+        return float((o * G).sum())
+
+    ok = True
+    for name, base, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        flat = base.float().numpy().reshape(-1)
+        for i in range(flat.size):
+            up, dn = flat.copy(), flat.copy()
+            up[i] += np.float32(eps)
+            dn[i] -= np.float32(eps)
+            args = {"q": q, "k": k, "v": v}
+            args[name] = torch.from_numpy(up.reshape(base.shape))
+            lu = loss(args["q"], args["k"], args["v"])
+            args[name] = torch.from_numpy(dn.reshape(base.shape))
+            ld = loss(args["q"], args["k"], args["v"])
+            # divide by the step the fp32 inputs actually took
+            fd = (lu - ld) / (float(up[i]) - float(dn[i]))
+            ok &= abs(fd - grad.reshape(-1)[i]) < 1e-4 * max(1.0, abs(fd))
+    return bool(ok)
+
+
+def pin_backward_gradient_equivalence(lib):
+    """[PS] test plan (gradient equivalence): the flat layout's gradients
+    equal those of running each [prefix; s_i] on its own with ordinary causal
+    attention (torch autograd in fp64), the prefix collecting the gradients of
+    every suffix; each copy carries 1/N of the prefix rows' upstream
+    gradient so that the summed losses equal the flat loss."""
+    P, N, S, Hq, Hkv, d = 9, 3, 5, 4, 2, 8
+    T = P + N * S
+    q, k, v = _rand((T, Hq, d), 91), _rand((T, Hkv, d), 92), _rand((T, Hkv, d), 93)
+    G = _rand((T, Hq, d), 94)
+    scale = 1 / math.sqrt(d)
+    dq, dk, dv = oracle.prefill_bwd(q, k, v, G, W.grpo_segments(P, N, S), scale, lib=lib)
+    qd = q.double().requires_grad_(True)
+    kd = k.double().requires_grad_(True)
+    vd = v.double().requires_grad_(True)
+    total = 0.0
+    for i in range(N):
+        sl = list(range(P)) + list(range(P + i * S, P + (i + 1) * S))
+        qi, ki, vi = qd[sl], _expand_kv(kd[sl], Hq), _expand_kv(vd[sl], Hq)
+        o = F.scaled_dot_product_attention(qi.permute(1, 0, 2)[None], ki.permute(1, 0, 2)[None],
+                                           vi.permute(1, 0, 2)[None], is_causal=True,
+                                           scale=scale)[0].permute(1, 0, 2)
+        w = G.double()[sl].clone()
+        w[:P] /= N
+        total = total + (o * w).sum()
+    total.backward()
+    return bool(np.allclose(dq, qd.grad.numpy(), atol=1e-12) and
+                np.allclose(dk, kd.grad.numpy(), atol=1e-12) and
+                np.allclose(dv, vd.grad.numpy(), atol=1e-12))
+
+
 PINS = [pin_golden_masks, pin_golden_tiny_attention, pin_equivalence_route,
         pin_sdpa_random_trees, pin_closed_forms, pin_special_cases,
         pin_brute_force_python, pin_verify_against_sdpa, pin_split_identity,
         pin_verify_shared_prefix, pin_e4m3_decoder, pin_verify_fp8_cache,
-        pin_sparse_latent]
+        pin_backward_finite_differences, pin_backward_gradient_equivalence, pin_sparse_latent]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
