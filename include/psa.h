@@ -76,10 +76,12 @@ typedef struct psa_segment {
 } psa_segment;
 
 /* A visibility rectangle over flat token indices: queries [q0, q1) see keys
- * [k0, k1); if causal, only where q - q0 >= k - k0 (top-left aligned). */
+ * [k0, k1); if causal == 1, only where q - q0 >= k - k0 (top-left aligned).
+ * causal == 2 appears only in transposed specs (psa_transpose_spec), where
+ * the rows are keys: row r sees column c iff c - c0 >= r - r0. */
 typedef struct psa_rect {
     int32_t q0, q1, k0, k1;
-    int32_t causal;
+    int32_t causal;  /* 0: full; 1: causal; 2: transposed causal (psa_transpose_spec) */
 } psa_rect;
 
 /* Segments of the flat GRPO layout [PS] design summary: one prefix of P
@@ -117,10 +119,20 @@ int psa_build_spec(const psa_segment *segs, int32_t nseg, psa_rect *out, int32_t
  *          flags: bit 0 / 1 = half A / B has visible pairs in the tile,
  *                 bit 2 / 3 = every pair of half A / B is visible
  *   rects  at 8 + 4*n_items + 8*n_kv: {q0, q1, k0, k1, causal} x n_rect
+ *          causal: 0 full, 1 causal (k - k0 <= q - q0), 2 transposed causal
+ *          (k - k0 >= q - q0; see psa_transpose_spec)
  * Returns PSA_ERR_CAPACITY (with *nout = needed length) if cap is short. */
 int psa_build_schedule(const psa_rect *rects, int32_t nrect, const int32_t *cu_seqlens,
                        int32_t ngroups, int32_t tile_m, int32_t tile_n, int32_t *out,
                        int64_t cap, int64_t *nout);
+
+/* The transpose of a spec, for schedules that walk keys as rows (the
+ * backward's dK / dV pass): rectangle r becomes {k0, k1, q0, q1} with
+ * causal 1 turned into 2 and 2 into 1, where causal == 2 marks a
+ * transposed causal rectangle (row r sees column c iff c - c0 >= r - r0).
+ * out may alias rects.  PSA_ERR_INVALID_ARG for a causal value outside
+ * 0..2. */
+int psa_transpose_spec(const psa_rect *rects, int32_t nrect, psa_rect *out);
 
 /* The block and tile sizes psa_prefill_fwd expects in its schedule:
  * tile_m query rows per block (two halves), tile_n keys per KV tile. */

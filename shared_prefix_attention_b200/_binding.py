@@ -32,7 +32,7 @@ EXPORTS = [
     "psa_prefill_fwd", "psa_verify_auto_splits", "psa_verify_workspace_size",
     "psa_verify_fwd", "psa_verify_fwd_noalloc", "psa_sparse_latent_fwd", "psa_read_status",
     "psa_wait_selftest", "psa_verify_shared_auto_splits", "psa_verify_shared_fwd",
-    "psa_verify_fp8_fwd",
+    "psa_verify_fp8_fwd", "psa_transpose_spec",
 ]
 
 
@@ -93,6 +93,7 @@ def lib():
         "psa_read_status": ([P, P, P], ctypes.c_int),
         "psa_wait_selftest": ([I32, P, P], ctypes.c_int),
         "psa_verify_shared_auto_splits": ([I32, I32, I32, I32, I64], I32),
+        "psa_transpose_spec": ([P, I32, P], ctypes.c_int),
         "psa_verify_fp8_fwd": ([P, P, P, P, P, I64, P, I64, P, F, F, P, P, I32, I32, I32, I32,
                                 I32, F, I32, P, P, SZ, P, P], ctypes.c_int),
         "psa_verify_shared_fwd": ([P, P, P, P, P, I64, P, P, I32, I32, I32, I32, I32, F, I32, P,
@@ -179,6 +180,14 @@ def build_schedule(rects: np.ndarray, cu_seqlens: Sequence[int], tile_m: int,
     out = np.zeros(n.value, dtype=np.int32)
     _check(lib().psa_build_schedule(_ptr(rects), len(rects), _ptr(cu), ng, tile_m, tile_n,
                                     _ptr(out), n.value, ctypes.byref(n)), "psa_build_schedule")
+    return out
+
+
+def transpose_spec(rects: np.ndarray) -> np.ndarray:
+    """Rectangles with rows and columns swapped (keys become rows)."""
+    rects = np.ascontiguousarray(rects, dtype=np.int32)
+    out = np.zeros_like(rects)
+    _check(lib().psa_transpose_spec(_ptr(rects), len(rects), _ptr(out)), "psa_transpose_spec")
     return out
 
 

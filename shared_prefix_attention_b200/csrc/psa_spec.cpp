@@ -24,9 +24,15 @@ int64_t visible_in_box(const psa_rect& r, int32_t qa, int32_t qb, int32_t ka, in
   if (!r.causal) return int64_t(q_hi - q_lo) * (k_hi - k_lo);
   int64_t n = 0;
   for (int32_t q = q_lo; q < q_hi; ++q) {
-    // causal: k - k0 <= q - q0
-    int32_t last = std::min<int32_t>(k_hi - 1, r.k0 + (q - r.q0));
-    if (last >= k_lo) n += last - k_lo + 1;
+    if (r.causal == 1) {
+      // causal: k - k0 <= q - q0
+      int32_t last = std::min<int32_t>(k_hi - 1, r.k0 + (q - r.q0));
+      if (last >= k_lo) n += last - k_lo + 1;
+    } else {
+      // transposed causal (keys as rows): k - k0 >= q - q0
+      int32_t first = std::max<int32_t>(k_lo, r.k0 + (q - r.q0));
+      if (first < k_hi) n += k_hi - first;
+    }
   }
   return n;
 }
@@ -79,6 +85,18 @@ extern "C" int psa_build_spec(const psa_segment* segs, int32_t nseg, psa_rect* o
   return PSA_OK;
 }
 
+extern "C" int psa_transpose_spec(const psa_rect* rects, int32_t nrect, psa_rect* out) {
+  if (nrect < 0 || (nrect > 0 && (!rects || !out))) return PSA_ERR_INVALID_ARG;
+  for (int32_t r = 0; r < nrect; ++r) {
+    const psa_rect x = rects[r];
+    if (x.causal < 0 || x.causal > 2) return PSA_ERR_INVALID_ARG;
+    // rows become keys and columns queries; a causal rectangle turns into
+    // its transpose and back
+    out[r] = psa_rect{x.k0, x.k1, x.q0, x.q1, x.causal == 0 ? 0 : 3 - x.causal};
+  }
+  return PSA_OK;
+}
+
 extern "C" int psa_build_schedule(const psa_rect* rects, int32_t nrect,
                                   const int32_t* cu_seqlens, int32_t ngroups, int32_t tile_m,
                                   int32_t tile_n, int32_t* out, int64_t cap, int64_t* nout) {
@@ -91,7 +109,8 @@ extern "C" int psa_build_schedule(const psa_rect* rects, int32_t nrect,
   const int32_t T = cu_seqlens[ngroups];
   for (int32_t r = 0; r < nrect; ++r) {
     const psa_rect& x = rects[r];
-    if (x.q0 < 0 || x.q1 > T || x.q0 >= x.q1 || x.k0 < 0 || x.k1 > T || x.k0 >= x.k1)
+    if (x.q0 < 0 || x.q1 > T || x.q0 >= x.q1 || x.k0 < 0 || x.k1 > T || x.k0 >= x.k1 ||
+        x.causal < 0 || x.causal > 2)
       return PSA_ERR_INVALID_ARG;
   }
   const int32_t half = tile_m / 2;

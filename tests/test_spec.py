@@ -23,10 +23,14 @@ def _expand(rects, T, row0=0, nrows=None):
         if a >= b:
             continue
         for q in range(a, b):
-            hi = min(k1, k0 + (q - q0) + 1) if causal else k1
-            if hi > k0:
-                assert not m[q - row0, k0:hi].any(), "rectangles overlap"
-                m[q - row0, k0:hi] = 1
+            lo, hi = k0, k1
+            if causal == 1:      # k - k0 <= q - q0
+                hi = min(k1, k0 + (q - q0) + 1)
+            elif causal == 2:    # transposed: k - k0 >= q - q0
+                lo = max(k0, k0 + (q - q0))
+            if hi > lo:
+                assert not m[q - row0, lo:hi].any(), "rectangles overlap"
+                m[q - row0, lo:hi] = 1
     return m
 
 
@@ -94,15 +98,21 @@ def _decode(sched):
     return items, kvs, rects, tm, tn, T, maxkv
 
 
-def _check_schedule(segs, cu, tm, tn):
+def _check_schedule(segs, cu, tm, tn, transpose=False):
     """Every Q block (two halves of tm/2 rows) lists exactly the KV tiles in
     which some half has a visible pair; per half the active / full flags
-    and the copied rectangles reproduce the visibility of the box."""
+    and the copied rectangles reproduce the visibility of the box.  With
+    transpose, the spec is transposed first and the rows are keys: the
+    schedule must then reproduce the transposed visibility."""
     rects = psa.build_spec(segs)
+    if transpose:
+        rects = psa.transpose_spec(rects)
     sched = psa.build_schedule(rects, cu, tm, tn)
     items, kvs, trects, tm2, tn2, T, maxkv = _decode(sched)
     assert (tm2, tn2, T) == (tm, tn, cu[-1])
     vis = oracle.visibility(segs).astype(bool)
+    if transpose:
+        vis = vis.T.copy()
     counts = [int(it[3]) for it in items]
     assert counts == sorted(counts, reverse=True)          # longest first
     assert maxkv == max(counts)
@@ -153,6 +163,21 @@ def _check_schedule(segs, cu, tm, tn):
 def test_schedule_tiles(P, N, S, groups, tm, tn):
     wl = W.PrefillWorkload("t", P=P, N=N, S=S, Hq=1, Hkv=1, d=64, groups=groups)
     _check_schedule(wl.segments(), wl.cu_seqlens(), tm, tn)
+
+
+@pytest.mark.parametrize("P,N,S,groups,tm,tn", [
+    (64, 4, 32, 1, 128, 64), (100, 3, 37, 2, 128, 64), (5, 7, 3, 1, 8, 4), (0, 4, 50, 1, 32, 16)])
+def test_transposed_schedule_tiles(P, N, S, groups, tm, tn):
+    """The key-major schedule of the backward's dK / dV pass (keys as rows)."""
+    wl = W.PrefillWorkload("t", P=P, N=N, S=S, Hq=1, Hkv=1, d=64, groups=groups)
+    _check_schedule(wl.segments(), wl.cu_seqlens(), tm, tn, transpose=True)
+
+
+def test_transpose_spec_round_trip():
+    rects = psa.build_spec(W.grpo_segments(10, 3, 4))
+    t = psa.transpose_spec(rects)
+    assert set(int(c) for c in t[:, 4]) <= {0, 2}
+    assert np.array_equal(psa.transpose_spec(t), rects)
 
 
 def test_schedule_random_trees():
