@@ -163,6 +163,46 @@ int psa_prefill_fwd(const void *q, const void *k, const void *v, void *o, float 
                     void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Backward of the prefill        [PS] design summary and test plan (the flat
+ * layout gives the gradients of running each [prefix; s_i] separately, the
+ * prefix K/V collecting the gradients of every suffix that sees them)
+ * --------------------------------------------------------------------- */
+
+/* Block and tile sizes of both backward schedules: tile_m rows per block
+ * (two halves), tile_n columns per tile.  The dQ pass uses
+ * psa_build_schedule(spec, ...) and the dK / dV pass
+ * psa_build_schedule(psa_transpose_spec(spec), ...) with these sizes. */
+int psa_prefill_bwd_tiles(int32_t head_dim, int32_t *tile_m, int32_t *tile_n);
+
+/* Workspace bytes psa_prefill_bwd needs: the log2-domain LSE and
+ * D = rowsum(dO * O) per (row, head), head-major. */
+size_t psa_prefill_bwd_workspace_size(int32_t T, int32_t Hq);
+
+/*
+ * Gradients of O = psa_prefill_fwd(q, k, v) for the upstream gradient dout.
+ *   q, dout    device [T, Hq, d] bf16
+ *   k, v       device [T, Hkv, d] bf16
+ *   o, lse     device, the forward's outputs for the same inputs and
+ *              schedule ([T, Hq, d] bf16 and [T, Hq] fp32)
+ *   dq         device [T, Hq, d] bf16 (written)
+ *   dk, dv     device [T, Hkv, d] bf16 (written; every row, zero where no
+ *              query sees the key)
+ *   dev_schedule     device copy of psa_build_schedule(spec, cu_seqlens, ngroups,
+ *                    tile_m, tile_n) with psa_prefill_bwd_tiles' sizes
+ *   dev_schedule_kv  device copy of the same for psa_transpose_spec(spec)
+ * dQ = scale dS K and dK = scale dS^T Q with dS = P (dO V^T - D); dV = P^T dO.
+ * d in {64, 128}; Hq % Hkv == 0.  No atomics: each output row is written
+ * once, by one CTA.  workspace: device, >= psa_prefill_bwd_workspace_size
+ * bytes, 256-B aligned.
+ */
+int psa_prefill_bwd(const void *q, const void *k, const void *v, const void *o,
+                    const float *lse, const void *dout, void *dq, void *dk, void *dv, int32_t T,
+                    int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
+                    const int32_t *dev_schedule, int64_t sched_len,
+                    const int32_t *dev_schedule_kv, int64_t sched_kv_len, void *workspace,
+                    size_t ws_bytes, int32_t *dev_status, void *stream);
+
+/* ------------------------------------------------------------------------
  * Speculative verify: split-KV over the cached prefix, then an LSE combine
  * that folds in the causal draft block.   [SKV] implementation item 1
  * --------------------------------------------------------------------- */

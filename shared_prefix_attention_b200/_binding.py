@@ -32,7 +32,8 @@ EXPORTS = [
     "psa_prefill_fwd", "psa_verify_auto_splits", "psa_verify_workspace_size",
     "psa_verify_fwd", "psa_verify_fwd_noalloc", "psa_sparse_latent_fwd", "psa_read_status",
     "psa_wait_selftest", "psa_verify_shared_auto_splits", "psa_verify_shared_fwd",
-    "psa_verify_fp8_fwd", "psa_transpose_spec",
+    "psa_verify_fp8_fwd", "psa_transpose_spec", "psa_prefill_bwd_tiles",
+    "psa_prefill_bwd_workspace_size", "psa_prefill_bwd",
 ]
 
 
@@ -94,6 +95,10 @@ def lib():
         "psa_wait_selftest": ([I32, P, P], ctypes.c_int),
         "psa_verify_shared_auto_splits": ([I32, I32, I32, I32, I64], I32),
         "psa_transpose_spec": ([P, I32, P], ctypes.c_int),
+        "psa_prefill_bwd_tiles": ([I32, P, P], ctypes.c_int),
+        "psa_prefill_bwd_workspace_size": ([I32, I32], SZ),
+        "psa_prefill_bwd": ([P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, F, P, I64, P, I64, P,
+                             SZ, P, P], ctypes.c_int),
         "psa_verify_fp8_fwd": ([P, P, P, P, P, I64, P, I64, P, F, F, P, P, I32, I32, I32, I32,
                                 I32, F, I32, P, P, SZ, P, P], ctypes.c_int),
         "psa_verify_shared_fwd": ([P, P, P, P, P, I64, P, P, I32, I32, I32, I32, I32, F, I32, P,
@@ -356,3 +361,42 @@ def verify_fp8(q_draft, k_draft, v_draft, k_cache8, v_cache8, k_scale: float, v_
                                   _stream(q_draft.device))
     _check(rc, "psa_verify_fp8_fwd")
     return out, lse
+
+
+def prefill_bwd_tiles(head_dim: int):
+    tm, tn = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib().psa_prefill_bwd_tiles(head_dim, ctypes.byref(tm), ctypes.byref(tn)),
+           "psa_prefill_bwd_tiles")
+    return tm.value, tn.value
+
+
+def plan_prefill_bwd(segments, cu_seqlens, head_dim: int, device="cuda"):
+    """The two backward schedules (row-major for dQ, key-major for dK / dV)
+    for a segment forest, uploaded to ``device``."""
+    tm, tn = prefill_bwd_tiles(head_dim)
+    spec = build_spec(segments)
+    sq = build_schedule(spec, cu_seqlens, tm, tn)
+    skv = build_schedule(transpose_spec(spec), cu_seqlens, tm, tn)
+    return torch.from_numpy(sq).to(device), torch.from_numpy(skv).to(device)
+
+
+def prefill_bwd(q, k, v, o, lse, dout, schedules, scale: float, dq=None, dk=None, dv=None,
+                workspace=None, status=None):
+    """Gradients (dq, dk, dv) of the prefill output for upstream gradient
+    ``dout``; ``schedules`` from :func:`plan_prefill_bwd`."""
+    sq, skv = schedules
+    _require_cuda(q, k, v, o, lse, dout, sq, skv)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(max(int(lib().psa_prefill_bwd_workspace_size(T, Hq)), 256),
+                                dtype=torch.uint8, device=q.device)
+    rc = lib().psa_prefill_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                               _ptr(dq), _ptr(dk), _ptr(dv), T, Hq, Hkv, d, float(scale),
+                               _ptr(sq), sq.numel(), _ptr(skv), skv.numel(), _ptr(workspace),
+                               workspace.numel(), _ptr(status), _stream(q.device))
+    _check(rc, "psa_prefill_bwd")
+    return dq, dk, dv

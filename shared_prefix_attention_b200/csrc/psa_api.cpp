@@ -332,6 +332,69 @@ extern "C" int psa_verify_shared_fwd(const void* q_draft, const void* k_draft,
   return launch_verify_shared(a);
 }
 
+// ------------------------------------------------------------------ backward
+
+extern "C" int psa_prefill_bwd_tiles(int32_t head_dim, int32_t* tile_m, int32_t* tile_n) {
+  if (!tile_m || !tile_n) return PSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PSA_ERR_UNSUPPORTED;
+  *tile_m = 128;  // two halves of 64 rows (keys in the transposed schedule)
+  *tile_n = 64;
+  return PSA_OK;
+}
+
+extern "C" size_t psa_prefill_bwd_workspace_size(int32_t T, int32_t Hq) {
+  if (T <= 0 || Hq <= 0) return 0;
+  const size_t tp = (size_t(T) + 3) / 4 * 4;
+  return 2 * ((tp * Hq * sizeof(float) + 255) / 256 * 256);
+}
+
+extern "C" int psa_prefill_bwd(const void* q, const void* k, const void* v, const void* o,
+                               const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                               int32_t T, int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
+                               const int32_t* dev_schedule, int64_t sched_len,
+                               const int32_t* dev_schedule_kv, int64_t sched_kv_len,
+                               void* workspace, size_t ws_bytes, int32_t* dev_status,
+                               void* stream) {
+  if (T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || !(scale > 0.f))
+    return PSA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return PSA_ERR_UNSUPPORTED;
+  if (T == 0) return PSA_OK;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !dev_schedule ||
+      !dev_schedule_kv || sched_len < 8 || sched_kv_len < 8)
+    return PSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return PSA_ERR_INVALID_ARG;
+  const size_t need = psa_prefill_bwd_workspace_size(T, Hq);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PSA_ERR_WORKSPACE;
+  BackwardArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.dout = dout;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.T = T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = head_dim;
+  a.scale = scale;
+  a.sched_q = dev_schedule;
+  a.sched_q_len = sched_len;
+  a.sched_kv = dev_schedule_kv;
+  a.sched_kv_len = sched_kv_len;
+  a.lse2_t = static_cast<float*>(workspace);
+  a.delta_t = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + need / 2);
+  a.status = dev_status;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_backward(a);
+}
+
 // ------------------------------------------------------------------ prefill
 
 extern "C" int psa_prefill_tiles(int32_t head_dim, int32_t* tile_m, int32_t* tile_n) {

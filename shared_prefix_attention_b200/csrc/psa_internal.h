@@ -91,6 +91,31 @@ struct PrefillArgs {
 };
 int launch_prefill(const PrefillArgs& a);
 
+// ---------------------------------------------------------------- backward
+
+struct BackwardArgs {
+  const void* q;     // bf16 [T, Hq, D]
+  const void* k;     // bf16 [T, Hkv, D]
+  const void* v;
+  const void* o;     // bf16 [T, Hq, D], the forward output
+  const float* lse;  // [T, Hq], natural log, the forward's
+  const void* dout;  // bf16 [T, Hq, D]
+  void* dq;          // bf16 [T, Hq, D] (written)
+  void* dk;          // bf16 [T, Hkv, D] (written)
+  void* dv;
+  int32_t T, Hq, Hkv, D;
+  float scale;
+  const int32_t* sched_q;   // psa_build_schedule(spec, ...), blocks of 128 rows, tiles of 64
+  int64_t sched_q_len;
+  const int32_t* sched_kv;  // psa_build_schedule(transposed spec, ...), same tile sizes
+  int64_t sched_kv_len;
+  float* lse2_t;            // workspace [Hq, Tp], Tp = T rounded up to a multiple of 4
+  float* delta_t;           // workspace [Hq, Tp]
+  int32_t* status;
+  cudaStream_t stream;
+};
+int launch_backward(const BackwardArgs& a);
+
 // ---------------------------------------------------------------- sparse latent
 
 struct SparseArgs {

@@ -1,0 +1,77 @@
+"""Backward of the prefill on the GPU against the fp64 oracle backward
+("KV-0 redundancy prefix sharing attention mask design": design summary and
+test plan -- the flat layout's gradients equal those of the separate
+[prefix; s_i] sequences, which pins the oracle).  Every call goes through the
+C ABI.
+
+Tolerance: the kernels round P and dS to bf16 for the tensor cores (relative
+error 2^-9 each) and read the forward's bf16 O for D = rowsum(dO * O); dS is
+a difference dP - D that cancels where P is large, so the gradients carry a
+few times the forward's relative error.  Bar: relative Frobenius error
+<= 2e-2 and max |err| <= 2e-2 * max |reference| per gradient."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import shared_prefix_attention_b200 as psa
+from shared_prefix_attention_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+REL_FRO = 2e-2
+MAX_ABS_REL = 2e-2
+
+
+def _grad_errors(got, ref):
+    g = got.float().cpu().numpy().astype(np.float64)
+    d = g - ref
+    return (float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-30)),
+            float(np.abs(d).max() / max(np.abs(ref).max(), 1e-30)))
+
+
+def _run(segs, cu, T, Hq, Hkv, d, seed=100):
+    gen = torch.Generator().manual_seed(seed)
+    draw = lambda shape: (torch.randn(shape, generator=gen) * 0.5).to(torch.bfloat16)
+    q, k, v = draw((T, Hq, d)), draw((T, Hkv, d)), draw((T, Hkv, d))
+    dout = draw((T, Hq, d))
+    scale = 1.0 / np.sqrt(d)
+    qg, kg, vg, dog = (t.cuda() for t in (q, k, v, dout))
+    sched = psa.plan_prefill(segs, cu, d, "cuda")
+    o, lse = psa.prefill(qg, kg, vg, sched, scale)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dk, dv = psa.prefill_bwd(qg, kg, vg, o, lse, dog, psa.plan_prefill_bwd(segs, cu, d),
+                                 scale, status=status)
+    torch.cuda.synchronize()
+    assert psa.read_status(status) == 0
+    rq, rk, rv = oracle.prefill_bwd(q, k, v, dout, segs, scale)
+    return (dq, dk, dv), (rq, rk, rv)
+
+
+def _check(got, ref, what):
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        fro, mx = _grad_errors(g, r)
+        assert np.isfinite(g.float().cpu().numpy()).all(), f"{what} {name}: non-finite"
+        assert fro <= REL_FRO and mx <= MAX_ABS_REL, f"{what} {name}: fro={fro:.3e} max={mx:.3e}"
+
+
+@pytest.mark.parametrize("P,N,S,Hq,Hkv,d,groups", [
+    (64, 4, 32, 2, 2, 128, 1),     # tile-aligned prefix, suffixes of half a tile
+    (100, 3, 37, 4, 2, 64, 1),     # ragged everywhere, GQA 2:1, d = 64
+    (128, 2, 64, 2, 1, 128, 2),    # two packed groups, MQA
+    (5, 7, 3, 2, 2, 128, 1),       # rows and keys far below one tile
+    (300, 2, 41, 2, 2, 128, 1),    # several KV blocks, partial diagonal tiles
+])
+def test_backward_parity_flat(P, N, S, Hq, Hkv, d, groups):
+    wl = W.PrefillWorkload("t", P=P, N=N, S=S, Hq=Hq, Hkv=Hkv, d=d, groups=groups)
+    got, ref = _run(wl.segments(), wl.cu_seqlens(), wl.T, Hq, Hkv, d)
+    _check(got, ref, f"P={P} N={N} S={S}")
+
+
+def test_backward_parity_random_trees():
+    g = torch.Generator().manual_seed(12)
+    for i in range(3):
+        segs = W.random_tree_segments(g, nseg=6, max_len=70, groups=1)
+        T = sum(s[0] for s in segs)
+        got, ref = _run(segs, [0, T], T, 2, 1, 128, seed=200 + i)
+        _check(got, ref, f"tree {i}")
