@@ -318,6 +318,39 @@ class SparseRunner(Runner):
                                lse=self.lse)
 
 
+class BackwardRunner(Runner):
+    """Prefill backward (dq, dk, dv) of the GRPO group; the forward outputs
+    are computed once outside the timed region."""
+    unit = "TFLOP/s"
+    bound = "tensor"
+    kernels_per_step = 3
+    kernel_file = "psa_backward.cu"
+
+    def __init__(self, wl: W.PrefillWorkload, dev):
+        import shared_prefix_attention_b200 as psa
+        self.psa, self.wl, self.dev = psa, wl, dev
+        self.name = wl.name.replace("grpo", "grpo-backward", 1)
+        self.q, self.k, self.v = wl.make(dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(wl.seed + 100)
+        self.dout = (torch.randn(self.q.shape, generator=g, device=dev) * wl.sigma).to(self.q.dtype)
+        sched = psa.plan_prefill(wl.segments(), wl.cu_seqlens(), wl.d, dev)
+        self.o, self.lse = psa.prefill(self.q, self.k, self.v, sched, wl.scale)
+        self.scheds = psa.plan_prefill_bwd(wl.segments(), wl.cu_seqlens(), wl.d, dev)
+        self.dq, self.dk, self.dv = (torch.empty_like(t) for t in (self.q, self.k, self.v))
+        n = int(psa.lib().psa_prefill_bwd_workspace_size(wl.T, wl.Hq))
+        self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+
+    def work(self):
+        # five products of the visible pairs (S, dP, dV, dQ, dK), 2 d FLOP each
+        return self.wl.flops() * 10.0 / 4.0
+
+    def step(self):
+        self.psa.prefill_bwd(self.q, self.k, self.v, self.o, self.lse, self.dout, self.scheds,
+                             self.wl.scale, dq=self.dq, dk=self.dk, dv=self.dv,
+                             workspace=self.ws)
+
+
 class VerifyFp8Runner(Runner):
     """Split-KV verify over an e4m3 prefix cache: HBM-bound on the cache bytes
     (one byte per element)."""
@@ -390,6 +423,7 @@ def make_runner(name: str, dev):
             "verify": lambda: VerifyRunner(W.VERIFY, dev),
             "verify-shared": lambda: SharedVerifyRunner(W.VERIFY_SHARED, dev),
             "verify-fp8": lambda: VerifyFp8Runner(W.VERIFY_FP8, dev),
+            "grpo-backward": lambda: BackwardRunner(W.GRPO, dev),
             "sparse": lambda: SparseRunner(W.SPARSE, dev)}[name]()
 
 
@@ -467,7 +501,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="grpo",
                     choices=["grpo", "tiny", "large", "verify", "verify8", "verify-shared",
-                             "verify-fp8", "sparse", "sparse4k"])
+                             "verify-fp8", "grpo-backward", "sparse", "sparse4k"])
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -518,7 +552,7 @@ def main():
 
     if not args.no_extras and args.workload == "grpo":
         extras = {}
-        for name in ("verify", "verify-fp8", "verify-shared", "large", "sparse"):
+        for name in ("verify", "verify-fp8", "verify-shared", "large", "grpo-backward", "sparse"):
             try:
                 r = make_runner(name, dev)
                 v, m, rf = measure(r, max(3, min(args.steps, 10)), 3, flush, dist_on, world,

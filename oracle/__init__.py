@@ -66,13 +66,15 @@ def load(path: str | None = None):
     lib.oracle_prefill.argtypes = [P, P, P, I, I, I, I, D, P, P, P, I, P, I, P, P, I]
     lib.oracle_verify.argtypes = [P, P, P, P, P, P, I, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_prefill_bwd.argtypes = [P, P, P, P, I, I, I, I, D, P, P, P, I, P, P, P, I]
+    lib.oracle_prefill_bwd_dq.argtypes = [P, P, P, P, I, I, I, I, D, P, P, P, I, P, I, P, I]
     lib.oracle_verify_shared.argtypes = [P, P, P, P, P, ctypes.c_int64, I, I, I, I, I, D, P, I,
                                          P, P, I]
     lib.oracle_verify_fp8.argtypes = [P, P, P, P, P, D, D, P, I, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_decode_e4m3.argtypes = [P, P, ctypes.c_int64]
     lib.oracle_sparse_latent.argtypes = [P, P, P, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_visibility.argtypes = [P, P, P, I, I, I, I, P]
-    for f in (lib.oracle_prefill, lib.oracle_prefill_bwd, lib.oracle_verify,
+    for f in (lib.oracle_prefill, lib.oracle_prefill_bwd, lib.oracle_prefill_bwd_dq,
+              lib.oracle_verify,
               lib.oracle_verify_shared,
               lib.oracle_verify_fp8, lib.oracle_decode_e4m3, lib.oracle_sparse_latent,
               lib.oracle_visibility):
@@ -164,6 +166,23 @@ def prefill_bwd(q, k, v, dout, segments, scale: float, nthreads: int | None = No
                                 _ptr(dk), _ptr(dv), nthreads or default_threads())
     assert rc == 0, "oracle_prefill_bwd rejected its arguments"
     return dq, dk, dv
+
+
+def prefill_bwd_dq(q, k, v, dout, segments, scale: float, rows, nthreads: int | None = None,
+                   lib=None):
+    """dq [nrows, Hq, d] (fp64) of the selected flat rows only."""
+    lib = lib or load()
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(dout)
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    start, lens, parent = segment_arrays(segments)
+    rows = _i32(rows)
+    dq = np.zeros((len(rows), Hq, d), dtype=np.float64)
+    rc = lib.oracle_prefill_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(do), T, Hq, Hkv, d,
+                                   float(scale), _ptr(start), _ptr(lens), _ptr(parent), len(lens),
+                                   _ptr(rows), len(rows), _ptr(dq), nthreads or default_threads())
+    assert rc == 0, "oracle_prefill_bwd_dq rejected its arguments"
+    return dq
 
 
 def verify(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr, Ld: int,

@@ -362,6 +362,70 @@ int oracle_prefill_bwd(const float *q, const float *k, const float *v, const flo
     return 0;
 }
 
+/*
+ * dq of selected rows only (dq of a row depends on that row's softmax
+ * alone): dq[r] = scale sum_k P_k (dO . v_k - dO . O) k_k for row rows[r].
+ * dq [nrows, Hq, d] (fp64, written).
+ */
+typedef struct {
+    const float *q, *k, *v, *dout;
+    int T, Hq, Hkv, d;
+    double scale;
+    const int32_t *tok_seg, *parent, *rows;
+    double *dq;
+} bwdq_ctx;
+
+static void bwdq_row(void *p, int r, double *z, const float **vr, double *o) {
+    bwdq_ctx *c = (bwdq_ctx *)p;
+    int qi = c->rows[r], d = c->d;
+    for (int h = 0; h < c->Hq; ++h) {
+        int kvh = kv_head_of(h, c->Hq, c->Hkv);
+        const float *qrow = c->q + ((size_t)qi * c->Hq + h) * d;
+        const float *dorow = c->dout + ((size_t)qi * c->Hq + h) * d;
+        double *dqrow = c->dq + ((size_t)r * c->Hq + h) * d;
+        for (int e = 0; e < d; ++e) dqrow[e] = 0.0;
+        int n = 0;
+        for (int kj = 0; kj < c->T; ++kj) {
+            if (!visible(c->tok_seg, c->parent, qi, kj)) continue;
+            z[n] = c->scale * dot(qrow, c->k + ((size_t)kj * c->Hkv + kvh) * d, d);
+            vr[n++] = c->k + ((size_t)kj * c->Hkv + kvh) * d; /* the key row, for dq */
+        }
+        if (n == 0) continue;
+        double m = -INFINITY, l = 0.0;
+        for (int i = 0; i < n; ++i) if (z[i] > m) m = z[i];
+        for (int i = 0; i < n; ++i) { z[i] = exp(z[i] - m); l += z[i]; }
+        for (int e = 0; e < d; ++e) o[e] = 0.0;
+        for (int i = 0; i < n; ++i) {
+            size_t kj = (size_t)(vr[i] - c->k) / ((size_t)c->Hkv * d);
+            const float *vrow = c->v + (kj * c->Hkv + kvh) * d;
+            for (int e = 0; e < d; ++e) o[e] += z[i] / l * (double)vrow[e];
+        }
+        double D = 0.0;
+        for (int e = 0; e < d; ++e) D += (double)dorow[e] * o[e];
+        for (int i = 0; i < n; ++i) {
+            size_t kj = (size_t)(vr[i] - c->k) / ((size_t)c->Hkv * d);
+            const float *vrow = c->v + (kj * c->Hkv + kvh) * d;
+            double dsc = z[i] / l * (dot(dorow, vrow, d) - D);
+            for (int e = 0; e < d; ++e) dqrow[e] += c->scale * dsc * (double)vr[i][e];
+        }
+    }
+}
+
+int oracle_prefill_bwd_dq(const float *q, const float *k, const float *v, const float *dout,
+                          int T, int Hq, int Hkv, int d, double scale,
+                          const int32_t *seg_start, const int32_t *seg_len,
+                          const int32_t *parent, int nseg, const int32_t *rows, int nrows,
+                          double *dq, int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || T < 0) return -1;
+    int32_t *tok_seg = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1));
+    if (!tok_seg) return -1;
+    token_segments(seg_start, seg_len, nseg, T, tok_seg);
+    bwdq_ctx c = {q, k, v, dout, T, Hq, Hkv, d, scale, tok_seg, parent, rows, dq};
+    run_rows(bwdq_row, &c, nrows, T, d, nthreads);
+    free(tok_seg);
+    return 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* speculative verify: cached prefix plus a causal draft block          */
 /* ------------------------------------------------------------------ */

@@ -228,6 +228,14 @@ __device__ __forceinline__ void store_rows(__nv_bfloat16* base, int H, int head,
   }
 }
 
+// Unit of this CTA in round r.  Units are listed longest first; odd rounds
+// hand them out in reverse CTA order, so the CTAs that got the longest units
+// of one round get the shortest of the next.
+__device__ __forceinline__ int snake_unit(int r) {
+  const int lane_in_round = (r & 1) ? int(gridDim.x) - 1 - int(blockIdx.x) : int(blockIdx.x);
+  return r * int(gridDim.x) + lane_in_round;
+}
+
 // ---------------------------------------------------------------- dq pass
 
 // The ring is fed by lane 0 of warp 0 between its own tiles (no separate
@@ -243,9 +251,9 @@ struct DqCfg {
   static constexpr uint32_t SMEM = 1024 + OFF_BAR + 2 * kStages * 8 + 16;
 };
 
-// Walks the (unit, KV tile) sequence of one CTA for the dq pass.
+// Walks the (round, KV tile) sequence of one CTA for the dq pass.
 struct DqCursor {
-  int u, j;
+  int r, j;
 };
 
 template <int D>
@@ -255,15 +263,16 @@ __device__ __forceinline__ bool dq_issue(const BwdParams& p, const int4* items,
                                          uint64_t* empty, const CUtensorMap* tk,
                                          const CUtensorMap* tv, int* abort_flag) {
   using C = DqCfg<D>;
-  while (cur.u < units) {
-    const int4 it = __ldg(items + cur.u / p.Hq);
+  int u = snake_unit(cur.r);
+  while (u < units) {
+    const int4 it = __ldg(items + u / p.Hq);
     if (cur.j < it.w) break;
-    cur.u += gridDim.x;
+    u = snake_unit(++cur.r);
     cur.j = 0;
   }
-  if (cur.u >= units) return true;  // nothing left to load
-  const int4 it = __ldg(items + cur.u / p.Hq);
-  const int kvh = (cur.u % p.Hq) / p.G;
+  if (u >= units) return true;  // nothing left to load
+  const int4 it = __ldg(items + u / p.Hq);
+  const int kvh = (u % p.Hq) / p.G;
   const int k0 = __ldg(kvs + 8 * (it.z + cur.j));
   const int s = n % kStages;
   if (!mbar_wait(empty + s, ((n / kStages) & 1) ^ 1, abort_flag, p.status)) return false;
@@ -310,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   const bool producer = warp == 0 && lane == 0;
-  DqCursor cur{int(blockIdx.x), 0};
+  DqCursor cur{0, 0};
   uint32_t issued = 0;
   bool ok = true;
   if (producer) {
@@ -320,14 +329,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const DqCursor before = cur;
       ok = dq_issue<D>(p, items, kvs, units, cur, issued, smem, full, empty, &tmap_k, &tmap_v,
                        &abort_flag);
-      if (ok && (cur.u != before.u || cur.j != before.j)) ++issued;
+      if (ok && (cur.r != before.r || cur.j != before.j)) ++issued;
     }
   }
 
   const int x = warp >> 2;  // half of the row block
   const int g = lane >> 2, c = lane & 3;
   uint32_t n = 0;
-  for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+  for (int rnd = 0; ok; ++rnd) {
+    const int u = snake_unit(rnd);
+    if (u >= units) break;
     const int4 it = __ldg(items + u / p.Hq);
     const int h = u % p.Hq;
     const int r0 = it.x + x * BR + (warp & 3) * 16;  // this warp's 16 rows
@@ -385,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const DqCursor before = cur;
         ok = dq_issue<D>(p, items, kvs, units, cur, issued, smem, full, empty, &tmap_k, &tmap_v,
                          &abort_flag);
-        if (ok && (cur.u != before.u || cur.j != before.j)) ++issued;
+        if (ok && (cur.r != before.r || cur.j != before.j)) ++issued;
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
     }
@@ -419,9 +430,9 @@ struct KvCfg {
   static constexpr uint32_t SMEM = 1024 + OFF_BAR + (2 * kStages + 2) * 8 + 16;
 };
 
-// Walks the (unit, query head, query tile) sequence of one CTA.
+// Walks the (round, query head, query tile) sequence of one CTA.
 struct KvCursor {
-  int u, gq, j;
+  int r, gq, j;
 };
 
 struct KvMaps {
@@ -434,18 +445,19 @@ __device__ __forceinline__ bool kv_issue(const BwdParams& p, const int4* items,
                                          uint32_t n, uint8_t* smem, uint64_t* full,
                                          uint64_t* empty, const KvMaps& m, int* abort_flag) {
   using C = KvCfg<D>;
-  while (cur.u < units) {
-    const int4 it = __ldg(items + cur.u / p.Hkv);
+  int u = snake_unit(cur.r);
+  while (u < units) {
+    const int4 it = __ldg(items + u / p.Hkv);
     if (cur.j < it.w) break;
     cur.j = 0;
     if (++cur.gq == p.G) {
       cur.gq = 0;
-      cur.u += gridDim.x;
+      u = snake_unit(++cur.r);
     }
   }
-  if (cur.u >= units) return true;
-  const int4 it = __ldg(items + cur.u / p.Hkv);
-  const int h = (cur.u % p.Hkv) * p.G + cur.gq;
+  if (u >= units) return true;
+  const int4 it = __ldg(items + u / p.Hkv);
+  const int h = (u % p.Hkv) * p.G + cur.gq;
   const int q0 = __ldg(qts + 8 * (it.z + cur.j));
   const int s = n % kStages;
   if (!mbar_wait(empty + s, ((n / kStages) & 1) ^ 1, abort_flag, p.status)) return false;
@@ -503,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   const bool producer = warp == 0 && lane == 0;
   const KvMaps maps{&tmap_q, &tmap_do, &tmap_lse, &tmap_delta};
-  KvCursor cur{int(blockIdx.x), 0, 0};
+  KvCursor cur{0, 0, 0};
   uint32_t issued = 0;
   bool ok = true;
   // the K and V block of unit u (the previous unit must have released it)
@@ -525,13 +537,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const KvCursor before = cur;
     const bool r = kv_issue<D>(p, items, qts, units, cur, issued, smem, full, empty, maps,
                                &abort_flag);
-    if (r && (cur.u != before.u || cur.gq != before.gq || cur.j != before.j)) ++issued;
+    if (r && (cur.r != before.r || cur.gq != before.gq || cur.j != before.j)) ++issued;
     return r;
   };
   if (producer) {
     tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_do);
-    ok = load_block(blockIdx.x, 0);
+    ok = load_block(snake_unit(0), 0);
     for (int i = 0; i < kStages && ok; ++i) ok = issue();
   }
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -540,7 +552,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = lane >> 2, c = lane & 3;
   const uint32_t kblk = smem_u32(smem + C::OFF_KV), vblk = kblk + C::BLOCK;
   uint32_t n = 0, uc = 0;
-  for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++uc) {
+  for (int rnd = 0; ok; ++rnd, ++uc) {
+    const int u = snake_unit(rnd);
+    if (u >= units) break;
     const int4 it = __ldg(items + u / p.Hkv);
     const int kvh = u % p.Hkv;
     const int kl0 = x * BR + (warp & 3) * 16;  // this warp's 16 keys within the block
@@ -605,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_arrive(kv_empty);
     store_rows<D>(p.dk, p.Hkv, kvh, key0, kend, dka, p.scale);
     store_rows<D>(p.dv, p.Hkv, kvh, key0, kend, dva, 1.f);
-    if (producer) ok = load_block(u + gridDim.x, uc + 1);
+    if (producer) ok = load_block(snake_unit(rnd + 1), uc + 1);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
   }
   if (!ok && producer) {

@@ -75,3 +75,33 @@ def test_backward_parity_random_trees():
         T = sum(s[0] for s in segs)
         got, ref = _run(segs, [0, T], T, 2, 1, 128, seed=200 + i)
         _check(got, ref, f"tree {i}")
+
+
+def test_backward_full_size_grpo():
+    """The GRPO group (P=2048, N=8, S=512, 16 heads, d=128): dq on sampled
+    rows against the oracle, and two identities that hold at any size and
+    involve every key: sum_k dV[k] = sum over the group's query heads and
+    rows of dO (each row's P sums to one), and sum_k dK[k] = 0 (each row's
+    dS sums to zero)."""
+    wl = W.GRPO
+    q, k, v = (t.cuda() for t in wl.make("cpu"))
+    gen = torch.Generator().manual_seed(300)
+    dout = (torch.randn((wl.T, wl.Hq, wl.d), generator=gen) * 0.5).to(torch.bfloat16)
+    dog = dout.cuda()
+    sched = psa.plan_prefill(wl.segments(), wl.cu_seqlens(), wl.d, "cuda")
+    o, lse = psa.prefill(q, k, v, sched, wl.scale)
+    dq, dk, dv = psa.prefill_bwd(q, k, v, o, lse, dog,
+                                 psa.plan_prefill_bwd(wl.segments(), wl.cu_seqlens(), wl.d),
+                                 wl.scale)
+    torch.cuda.synchronize()
+    rows = np.array([0, 1, 127, 128, 2047, 2048, 2100, 2559, 2560, 4000, wl.T - 1],
+                    dtype=np.int32)
+    rq = oracle.prefill_bwd_dq(q.cpu(), k.cpu(), v.cpu(), dout, wl.segments(), wl.scale, rows)
+    fro, mx = _grad_errors(dq[torch.as_tensor(rows).long().cuda()], rq)
+    assert fro <= REL_FRO and mx <= MAX_ABS_REL, f"dq rows: fro={fro:.3e} max={mx:.3e}"
+    G = wl.Hq // wl.Hkv
+    sv = dv.double().sum(0)                                   # [Hkv, d]
+    want = dog.double().sum(0).view(wl.Hkv, G, wl.d).sum(1)   # [Hkv, d]
+    assert (sv - want).norm() <= REL_FRO * want.norm()
+    sk = dk.double().sum(0)
+    assert sk.norm() <= 0.05 * dk.double().norm()

@@ -436,9 +436,14 @@ def pin_backward_gradient_equivalence(lib):
         w[:P] /= N
         total = total + (o * w).sum()
     total.backward()
-    return bool(np.allclose(dq, qd.grad.numpy(), atol=1e-12) and
-                np.allclose(dk, kd.grad.numpy(), atol=1e-12) and
-                np.allclose(dv, vd.grad.numpy(), atol=1e-12))
+    ok = (np.allclose(dq, qd.grad.numpy(), atol=1e-12) and
+          np.allclose(dk, kd.grad.numpy(), atol=1e-12) and
+          np.allclose(dv, vd.grad.numpy(), atol=1e-12))
+    # the row-sampled dq agrees with the full backward
+    rows = np.array([0, P - 1, P, T - 1, P + S + 2], dtype=np.int32)
+    dqs = oracle.prefill_bwd_dq(q, k, v, G, W.grpo_segments(P, N, S), scale, rows, lib=lib)
+    ok &= np.allclose(dqs, dq[rows], atol=1e-12)
+    return bool(ok)
 
 
 PINS = [pin_golden_masks, pin_golden_tiny_attention, pin_equivalence_route,
