@@ -67,6 +67,7 @@ def load(path: str | None = None):
     lib.oracle_verify.argtypes = [P, P, P, P, P, P, I, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_prefill_bwd.argtypes = [P, P, P, P, I, I, I, I, D, P, P, P, I, P, P, P, I]
     lib.oracle_prefill_bwd_dq.argtypes = [P, P, P, P, I, I, I, I, D, P, P, P, I, P, I, P, I]
+    lib.oracle_verify_tree.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_verify_shared.argtypes = [P, P, P, P, P, ctypes.c_int64, I, I, I, I, I, D, P, I,
                                          P, P, I]
     lib.oracle_verify_fp8.argtypes = [P, P, P, P, P, D, D, P, I, I, I, I, I, D, P, I, P, P, I]
@@ -74,7 +75,7 @@ def load(path: str | None = None):
     lib.oracle_sparse_latent.argtypes = [P, P, P, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_visibility.argtypes = [P, P, P, I, I, I, I, P]
     for f in (lib.oracle_prefill, lib.oracle_prefill_bwd, lib.oracle_prefill_bwd_dq,
-              lib.oracle_verify,
+              lib.oracle_verify, lib.oracle_verify_tree,
               lib.oracle_verify_shared,
               lib.oracle_verify_fp8, lib.oracle_decode_e4m3, lib.oracle_sparse_latent,
               lib.oracle_visibility):
@@ -203,6 +204,30 @@ def verify(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr, Ld: int,
                            B, Ld, Hq, Hkv, d, float(scale), _ptr(rows), len(rows),
                            _ptr(o), _ptr(lse), nthreads or default_threads())
     assert rc == 0, "oracle_verify rejected its arguments"
+    return o, lse
+
+
+def verify_tree(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr, draft_mask, Ld: int,
+                scale: float, rows=None, nthreads: int | None = None, lib=None):
+    """As verify, with the draft block given by draft_mask [B*Ld, Ld] (row
+    b*Ld + j lists the drafts of request b that draft j sees)."""
+    lib = lib or load()
+    qd, kd, vd = _f32(q_draft), _f32(k_draft), _f32(v_draft)
+    kc, vc = _f32(k_cache), _f32(v_cache)
+    dm = _u8(draft_mask)
+    indptr = np.ascontiguousarray(np.asarray(
+        kv_indptr.cpu().numpy() if hasattr(kv_indptr, "cpu") else kv_indptr, dtype=np.int64))
+    BL, Hq, d = qd.shape
+    Hkv = kd.shape[1]
+    B = BL // Ld
+    assert dm.shape == (BL, Ld)
+    rows = np.arange(BL, dtype=np.int32) if rows is None else _i32(rows)
+    o = np.zeros((len(rows), Hq, d), dtype=np.float64)
+    lse = np.zeros((len(rows), Hq), dtype=np.float64)
+    rc = lib.oracle_verify_tree(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kc), _ptr(vc), _ptr(indptr),
+                                _ptr(dm), B, Ld, Hq, Hkv, d, float(scale), _ptr(rows), len(rows),
+                                _ptr(o), _ptr(lse), nthreads or default_threads())
+    assert rc == 0, "oracle_verify_tree rejected its arguments"
     return o, lse
 
 

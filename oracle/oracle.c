@@ -438,6 +438,7 @@ typedef struct {
     double scale;
     const int32_t *rows;
     double *o, *lse;
+    const uint8_t *dmask;  /* NULL: causal draft block; else [B*Ld, Ld], draft j sees i */
 } verify_ctx;
 
 static void verify_row(void *p, int r, double *z, const float **vr, double *o) {
@@ -459,7 +460,9 @@ static void verify_row(void *p, int r, double *z, const float **vr, double *o) {
 #if ORACLE_MUTANT == 6
         for (int i = 0; i < c->Ld; ++i) {  /* planted: the draft block is not causal */
 #else
-        for (int i = 0; i <= j; ++i) {     /* drafts 0..j: the causal draft block */
+        for (int i = 0; i < c->Ld; ++i) {
+            /* drafts 0..j (the causal draft block), or the tree mask's row j */
+            if (c->dmask ? !c->dmask[(size_t)row * c->Ld + i] : i > j) continue;
 #endif
             size_t dr = (size_t)b * c->Ld + i;
             const float *krow = c->kd + (dr * c->Hkv + kvh) * c->d;
@@ -487,7 +490,28 @@ int oracle_verify(const float *qd, const float *kd, const float *vd,
     int64_t maxlen = 0;
     for (int b = 0; b < B; ++b)
         if (indptr[b + 1] - indptr[b] > maxlen) maxlen = indptr[b + 1] - indptr[b];
-    verify_ctx c = {qd, kd, vd, kc, vc, indptr, 0, Ld, Hq, Hkv, d, scale, rows, o, lse};
+    verify_ctx c = {qd, kd, vd, kc, vc, indptr, 0, Ld, Hq, Hkv, d, scale, rows, o, lse, NULL};
+    run_rows(verify_row, &c, nrows, (int)maxlen + Ld, d, nthreads);
+    return 0;
+}
+
+/*
+ * Tree verify: "Split-KV flash-decode attention for EAGLE target-verify"
+ * (can_handle: topk > 1 brings a custom draft mask; the prefix is skipped by
+ * the custom mask, so every draft still sees the whole cached prefix).
+ * dmask [B*Ld, Ld] uint8: draft j of request b sees draft i of b iff
+ * dmask[(b*Ld + j)*Ld + i] != 0.  Otherwise as oracle_verify.
+ */
+int oracle_verify_tree(const float *qd, const float *kd, const float *vd,
+                       const float *kc, const float *vc, const int64_t *indptr,
+                       const uint8_t *dmask, int B, int Ld, int Hq, int Hkv, int d,
+                       double scale, const int32_t *rows, int nrows, double *o,
+                       double *lse, int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || B < 0 || Ld <= 0 || !dmask) return -1;
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b)
+        if (indptr[b + 1] - indptr[b] > maxlen) maxlen = indptr[b + 1] - indptr[b];
+    verify_ctx c = {qd, kd, vd, kc, vc, indptr, 0, Ld, Hq, Hkv, d, scale, rows, o, lse, dmask};
     run_rows(verify_row, &c, nrows, (int)maxlen + Ld, d, nthreads);
     return 0;
 }
@@ -507,7 +531,7 @@ int oracle_verify_shared(const float *qd, const float *kd, const float *vd,
                          const int32_t *rows, int nrows, double *o, double *lse,
                          int nthreads) {
     if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || B < 0 || Ld <= 0 || L < 0) return -1;
-    verify_ctx c = {qd, kd, vd, kp, vp, NULL, L, Ld, Hq, Hkv, d, scale, rows, o, lse};
+    verify_ctx c = {qd, kd, vd, kp, vp, NULL, L, Ld, Hq, Hkv, d, scale, rows, o, lse, NULL};
     run_rows(verify_row, &c, nrows, (int)L + Ld, d, nthreads);
     return 0;
 }

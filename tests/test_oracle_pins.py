@@ -231,6 +231,34 @@ def pin_verify_against_sdpa(lib):
     return bool(ok)
 
 
+def pin_verify_tree_mask(lib):
+    """[SKV] can_handle: EAGLE trees (topk > 1) bring a custom draft mask while
+    the prefix stays fully visible.  Checked against SDPA with the explicit
+    mask; the lower-triangular mask reproduces the causal verify exactly."""
+    q, kd, vd, kc, vc, indptr, Ld = _verify_case(seed=61, Ld=4)
+    B, Hq, d = len(indptr) - 1, q.shape[1], q.shape[2]
+    scale = 1 / math.sqrt(d)
+    # a depth-2 tree per request: 0 -> {1, 2}, 1 -> 3 (each draft sees its ancestors and itself)
+    tree = np.array([[1, 0, 0, 0], [1, 1, 0, 0], [1, 0, 1, 0], [1, 1, 0, 1]], dtype=np.uint8)
+    dm = np.tile(tree, (B, 1))
+    o, _ = oracle.verify_tree(q, kd, vd, kc, vc, indptr, dm, Ld, scale, lib=lib)
+    ok = True
+    for b in range(B):
+        p0, p1 = int(indptr[b]), int(indptr[b + 1])
+        ks = torch.cat([kc[p0:p1], kd[b * Ld:(b + 1) * Ld]])
+        vs = torch.cat([vc[p0:p1], vd[b * Ld:(b + 1) * Ld]])
+        L = p1 - p0
+        mask = torch.ones((Ld, L + Ld), dtype=torch.bool)
+        mask[:, L:] = torch.from_numpy(tree.astype(bool))
+        ref = _sdpa(q[b * Ld:(b + 1) * Ld], _expand_kv(ks, Hq), _expand_kv(vs, Hq), mask, scale)
+        ok &= np.allclose(o[b * Ld:(b + 1) * Ld], ref, atol=1e-12)
+    causal = np.tile(np.tril(np.ones((Ld, Ld), dtype=np.uint8)), (B, 1))
+    o1, l1 = oracle.verify_tree(q, kd, vd, kc, vc, indptr, causal, Ld, scale, lib=lib)
+    o2, l2 = oracle.verify(q, kd, vd, kc, vc, indptr, Ld, scale, lib=lib)
+    ok &= np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    return bool(ok)
+
+
 def _split_combine(q, kd, vd, kc, vc, indptr, Ld, scale, nsplit):
     """Split-KV + LSE combine written out per [SKV] implementation item 1:
     stage 1 gives each prefix chunk a normalised partial O and its LSE
@@ -449,7 +477,7 @@ def pin_backward_gradient_equivalence(lib):
 PINS = [pin_golden_masks, pin_golden_tiny_attention, pin_equivalence_route,
         pin_sdpa_random_trees, pin_closed_forms, pin_special_cases,
         pin_brute_force_python, pin_verify_against_sdpa, pin_split_identity,
-        pin_verify_shared_prefix, pin_e4m3_decoder, pin_verify_fp8_cache,
+        pin_verify_tree_mask, pin_verify_shared_prefix, pin_e4m3_decoder, pin_verify_fp8_cache,
         pin_backward_finite_differences, pin_backward_gradient_equivalence, pin_sparse_latent]
 
 
