@@ -260,6 +260,27 @@ int psa_verify_fwd(const void *q_draft, const void *k_draft, const void *v_draft
                    float scale, int32_t nsplit, const psa_verify_features *features,
                    void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/*
+ * Tree verify: psa_verify_fwd with the draft block given by a custom mask
+ * instead of the causal chain ([SKV] key code, can_handle: EAGLE trees with
+ * topk > 1 bring a custom mask; the prefix is not masked, so every draft
+ * still sees the whole cached prefix).
+ *   dev_draft_mask  device uint8 [B*Ld, Ld]: draft j of request b sees draft
+ *                   i of b iff dev_draft_mask[(b*Ld + j)*Ld + i] != 0
+ *                   (required when B > 0: PSA_ERR_INVALID_ARG otherwise)
+ * features->has_custom_mask may be set here; every other argument, layout,
+ * gate and status is that of psa_verify_fwd.  A draft row that sees no key
+ * (empty prefix and an empty mask row) gets O = 0 and LSE = -inf.
+ */
+int psa_verify_tree_fwd(const void *q_draft, const void *k_draft, const void *v_draft,
+                        const void *k_cache, const void *v_cache, int64_t n_cache_tokens,
+                        const int32_t *dev_kv_indptr, int64_t max_prefix_len,
+                        const int32_t *kv_indices, const uint8_t *dev_draft_mask, void *o,
+                        float *lse, int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv,
+                        int32_t head_dim, float scale, int32_t nsplit,
+                        const psa_verify_features *features, void *workspace, size_t ws_bytes,
+                        int32_t *dev_status, void *stream);
+
 /* Size of the library's fixed device scratch used by psa_verify_fwd_noalloc:
  * 16 MiB, held by every GPU that loads the library until the process exits. */
 #define PSA_VERIFY_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -33,7 +33,7 @@ EXPORTS = [
     "psa_verify_fwd", "psa_verify_fwd_noalloc", "psa_sparse_latent_fwd", "psa_read_status",
     "psa_wait_selftest", "psa_verify_shared_auto_splits", "psa_verify_shared_fwd",
     "psa_verify_fp8_fwd", "psa_transpose_spec", "psa_prefill_bwd_tiles",
-    "psa_prefill_bwd_workspace_size", "psa_prefill_bwd",
+    "psa_prefill_bwd_workspace_size", "psa_prefill_bwd", "psa_verify_tree_fwd",
 ]
 
 
@@ -96,6 +96,8 @@ def lib():
         "psa_verify_shared_auto_splits": ([I32, I32, I32, I32, I64], I32),
         "psa_transpose_spec": ([P, I32, P], ctypes.c_int),
         "psa_prefill_bwd_tiles": ([I32, P, P], ctypes.c_int),
+        "psa_verify_tree_fwd": ([P, P, P, P, P, I64, P, I64, P, P, P, P, I32, I32, I32, I32, I32,
+                                 F, I32, P, P, SZ, P, P], ctypes.c_int),
         "psa_prefill_bwd_workspace_size": ([I32, I32], SZ),
         "psa_prefill_bwd": ([P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, F, P, I64, P, I64, P,
                              SZ, P, P], ctypes.c_int),
@@ -400,3 +402,28 @@ def prefill_bwd(q, k, v, o, lse, dout, schedules, scale: float, dq=None, dk=None
                                workspace.numel(), _ptr(status), _stream(q.device))
     _check(rc, "psa_prefill_bwd")
     return dq, dk, dv
+
+
+def verify_tree(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr: torch.Tensor,
+                max_prefix_len: int, draft_mask: torch.Tensor, scale: float, Ld: int,
+                nsplit: int = 0, out=None, lse=None, workspace=None, status=None):
+    """Split-KV verify with a custom draft mask (device uint8 [B*Ld, Ld])."""
+    _require_cuda(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr, draft_mask)
+    BL, Hq, d = q_draft.shape
+    Hkv = k_draft.shape[1]
+    B = BL // Ld
+    ns = nsplit or verify_auto_splits(B, max_prefix_len, Hkv, d)
+    out = torch.empty_like(q_draft) if out is None else out
+    lse = torch.empty((BL, Hq), dtype=torch.float32, device=q_draft.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(max(verify_workspace_size(B, Ld, Hq, d, ns), 256),
+                                dtype=torch.uint8, device=q_draft.device)
+    feat = VerifyFeatures(1, 1, -1, 0, 0.0, -1, 0)
+    rc = lib().psa_verify_tree_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft), _ptr(k_cache),
+                                   _ptr(v_cache), k_cache.shape[0], _ptr(kv_indptr),
+                                   int(max_prefix_len), None, _ptr(draft_mask), _ptr(out),
+                                   _ptr(lse), B, Ld, Hq, Hkv, d, float(scale), ns,
+                                   ctypes.byref(feat), _ptr(workspace), workspace.numel(),
+                                   _ptr(status), _stream(q_draft.device))
+    _check(rc, "psa_verify_tree_fwd")
+    return out, lse

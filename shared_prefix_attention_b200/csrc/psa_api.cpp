@@ -134,17 +134,19 @@ extern "C" size_t psa_verify_workspace_size(int32_t B, int32_t Ld, int32_t Hq,
   return o_bytes + l_bytes;
 }
 
-extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const void* v_draft,
+static int verify_common(const void* q_draft, const void* k_draft, const void* v_draft,
                               const void* k_cache, const void* v_cache, int64_t n_cache_tokens,
                               const int32_t* dev_kv_indptr, int64_t max_prefix_len,
                               const int32_t* kv_indices, void* o, float* lse, int32_t B,
                               int32_t Ld, int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
                               int32_t nsplit, const psa_verify_features* features,
                               void* workspace, size_t ws_bytes, int32_t* dev_status,
-                              void* stream) {
-  // The split-KV path's gating ("can_handle"): everything else is refused.
+                              void* stream, const uint8_t* dmask) {
+  // The split-KV path's gating ("can_handle"): everything else is refused;
+  // a custom draft mask only through the tree entry, which passes dmask.
   if (features) {
-    if (features->has_custom_mask || !features->is_causal || features->sliding_window > 0 ||
+    if ((features->has_custom_mask && !dmask) || !features->is_causal ||
+        features->sliding_window > 0 ||
         features->has_sinks || features->logit_cap != 0.f ||
         features->xai_temperature_len > 0 || features->ragged_extend)
       return PSA_ERR_UNSUPPORTED;
@@ -193,7 +195,38 @@ extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const vo
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + o_bytes);
   a.status = dev_status;
   a.stream = static_cast<cudaStream_t>(stream);
+  a.dmask = dmask;
   return launch_verify(a);
+}
+
+extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const void* v_draft,
+                              const void* k_cache, const void* v_cache, int64_t n_cache_tokens,
+                              const int32_t* dev_kv_indptr, int64_t max_prefix_len,
+                              const int32_t* kv_indices, void* o, float* lse, int32_t B,
+                              int32_t Ld, int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
+                              int32_t nsplit, const psa_verify_features* features,
+                              void* workspace, size_t ws_bytes, int32_t* dev_status,
+                              void* stream) {
+  return verify_common(q_draft, k_draft, v_draft, k_cache, v_cache, n_cache_tokens,
+                       dev_kv_indptr, max_prefix_len, kv_indices, o, lse, B, Ld, Hq, Hkv,
+                       head_dim, scale, nsplit, features, workspace, ws_bytes, dev_status, stream,
+                       nullptr);
+}
+
+extern "C" int psa_verify_tree_fwd(const void* q_draft, const void* k_draft, const void* v_draft,
+                                   const void* k_cache, const void* v_cache,
+                                   int64_t n_cache_tokens, const int32_t* dev_kv_indptr,
+                                   int64_t max_prefix_len, const int32_t* kv_indices,
+                                   const uint8_t* dev_draft_mask, void* o, float* lse, int32_t B,
+                                   int32_t Ld, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                                   float scale, int32_t nsplit,
+                                   const psa_verify_features* features, void* workspace,
+                                   size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (B > 0 && !dev_draft_mask) return PSA_ERR_INVALID_ARG;
+  return verify_common(q_draft, k_draft, v_draft, k_cache, v_cache, n_cache_tokens,
+                       dev_kv_indptr, max_prefix_len, kv_indices, o, lse, B, Ld, Hq, Hkv,
+                       head_dim, scale, nsplit, features, workspace, ws_bytes, dev_status, stream,
+                       dev_draft_mask);
 }
 
 extern "C" int psa_verify_fp8_fwd(const void* q_draft, const void* k_draft, const void* v_draft,

@@ -39,6 +39,7 @@ struct VerifyArgs {
   float* part_lse;  // [nsplit][B*Ld][Hq], log2 domain
   int32_t* status;
   cudaStream_t stream;
+  const uint8_t* dmask = nullptr;  // tree verify: [B*Ld, Ld] draft mask (device)
 };
 
 // KV heads per CTA, 16-row m-tiles per CTA and row blocks per KV head;

@@ -329,6 +329,7 @@ struct Stage2Params {
   const float* part_lse;
   __nv_bfloat16* o;
   float* lse;
+  const uint8_t* dmask;  // nullable: causal draft block; else [B*Ld, Ld] tree mask
   int32_t B, Ld, Hq, Hkv, G, nsplit;
   float scale_log2;
 };
@@ -361,13 +362,25 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
     for (int off = 16; off > 0; off >>= 1) sdot += __shfl_xor_sync(0xffffffffu, sdot, off);
     return sdot * p.scale_log2;
   };
+  // the draft block: drafts 0..j, or the tree mask's row (the same for every head)
+  const uint8_t* mrow = p.dmask ? p.dmask + size_t(row) * p.Ld : nullptr;
+  auto sees = [&](int i) { return mrow ? __ldg(mrow + i) != 0 : i <= j; };
+  const int nd = mrow ? p.Ld : j + 1;
   float M = -INFINITY;
-  const int nd = j + 1;
-  for (int i = 0; i < nd; ++i) M = fmaxf(M, draft_logit(i));
+  for (int i = 0; i < nd; ++i)
+    if (sees(i)) M = fmaxf(M, draft_logit(i));
   for (int s = lane; s < p.nsplit; s += 32)
     M = fmaxf(M, p.part_lse[(size_t(s) * BL + row) * p.Hq + qh]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (M == -INFINITY) {
+    // no visible key (an empty prefix and an empty tree-mask row)
+    __nv_bfloat16* op = p.o + (size_t(row) * p.Hq + qh) * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) op[e] = __float2bfloat16(0.f);
+    if (p.lse && lane == 0) p.lse[size_t(row) * p.Hq + qh] = -INFINITY;
+    return;
+  }
 
   float acc[E];
 #pragma unroll
@@ -388,18 +401,20 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
     wsum += w;
   }
   for (int i = 0; i < nd; ++i) {
+    if (!sees(i)) continue;
     const float w = fast_exp2(draft_logit(i) - M);
     const __nv_bfloat16* vp = p.vd + (size_t(b * p.Ld + i) * p.Hkv + kvh) * D + lane * E;
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] += w * __bfloat162float(vp[e]);
     wsum += w;
   }
-  const float inv = 1.f / wsum;
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;  // no visible key at all: O = 0
   __nv_bfloat16* op = p.o + (size_t(row) * p.Hq + qh) * D + lane * E;
 #pragma unroll
   for (int e = 0; e < E; e += 2)
     *reinterpret_cast<__nv_bfloat162*>(op + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
-  if (p.lse && lane == 0) p.lse[size_t(row) * p.Hq + qh] = (M + __log2f(wsum)) * kLn2;
+  if (p.lse && lane == 0)
+    p.lse[size_t(row) * p.Hq + qh] = wsum > 0.f ? (M + __log2f(wsum)) * kLn2 : -INFINITY;
 }
 
 template <int D>
@@ -478,6 +493,7 @@ int launch_combine_d(const VerifyArgs& a) {
   p2.part_lse = a.part_lse;
   p2.o = static_cast<__nv_bfloat16*>(a.o);
   p2.lse = a.lse;
+  p2.dmask = a.dmask;
   p2.B = a.B;
   p2.Ld = a.Ld;
   p2.Hq = a.Hq;

@@ -118,6 +118,20 @@ def test_verify_shared_auto_splits():
     assert psa.verify_shared_auto_splits(1, 1, 1, 1, 1 << 20) <= 256
 
 
+def test_verify_tree_needs_a_mask():
+    P = ctypes.c_void_p
+    f = psa.VerifyFeatures(1, 1, -1, 0, 0.0, -1, 0)
+    rc = psa.lib().psa_verify_tree_fwd(P(16), P(16), P(16), P(16), P(16), 64, P(16), 64, None,
+                                       None, P(16), None, 1, 4, 8, 2, 128, 0.1, 1,
+                                       ctypes.byref(f), None, 0, None, None)
+    assert rc == psa.PSA_ERR_INVALID_ARG
+    # with a mask the custom-mask feature passes the gate (then the workspace is missing)
+    rc = psa.lib().psa_verify_tree_fwd(P(16), P(16), P(16), P(16), P(16), 64, P(16), 64, None,
+                                       P(16), P(16), None, 1, 4, 8, 2, 128, 0.1, 1,
+                                       ctypes.byref(f), None, 0, None, None)
+    assert rc == psa.PSA_ERR_WORKSPACE
+
+
 def test_verify_fp8_host_validation():
     P = ctypes.c_void_p
 
