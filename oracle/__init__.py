@@ -68,6 +68,7 @@ def load(path: str | None = None):
     lib.oracle_prefill_bwd.argtypes = [P, P, P, P, I, I, I, I, D, P, P, P, I, P, P, P, I]
     lib.oracle_prefill_bwd_dq.argtypes = [P, P, P, P, I, I, I, I, D, P, P, P, I, P, I, P, I]
     lib.oracle_verify_tree.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, D, P, I, P, P, I]
+    lib.oracle_verify_extend.argtypes = [P] * 10 + [I, I, I, I, D, P, I, P, P, I]
     lib.oracle_verify_shared.argtypes = [P, P, P, P, P, ctypes.c_int64, I, I, I, I, I, D, P, I,
                                          P, P, I]
     lib.oracle_verify_fp8.argtypes = [P, P, P, P, P, D, D, P, I, I, I, I, I, D, P, I, P, P, I]
@@ -75,7 +76,7 @@ def load(path: str | None = None):
     lib.oracle_sparse_latent.argtypes = [P, P, P, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_visibility.argtypes = [P, P, P, I, I, I, I, P]
     for f in (lib.oracle_prefill, lib.oracle_prefill_bwd, lib.oracle_prefill_bwd_dq,
-              lib.oracle_verify, lib.oracle_verify_tree,
+              lib.oracle_verify, lib.oracle_verify_tree, lib.oracle_verify_extend,
               lib.oracle_verify_shared,
               lib.oracle_verify_fp8, lib.oracle_decode_e4m3, lib.oracle_sparse_latent,
               lib.oracle_visibility):
@@ -228,6 +229,43 @@ def verify_tree(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr, draft_ma
                                 _ptr(dm), B, Ld, Hq, Hkv, d, float(scale), _ptr(rows), len(rows),
                                 _ptr(o), _ptr(lse), nthreads or default_threads())
     assert rc == 0, "oracle_verify_tree rejected its arguments"
+    return o, lse
+
+
+def _i64(x):
+    return np.ascontiguousarray(np.asarray(x.cpu().numpy() if hasattr(x, "cpu") else x,
+                                           dtype=np.int64))
+
+
+def verify_extend(q_draft, k_draft, v_draft, k_cache, v_cache, qo_indptr, kv_indptr, scale: float,
+                  kv_indices=None, draft_mask=None, mask_indptr=None, rows=None,
+                  nthreads: int | None = None, lib=None):
+    """Verify in the extend form: ragged draft counts (qo_indptr), a paged
+    prefix (kv_indices: prefix position t is cache row kv_indices[t]) and an
+    optional per-request draft mask (request b's Lb x Lb block starts at
+    draft_mask[mask_indptr[b]], flat uint8).  O [nrows, Hq, d], LSE [nrows, Hq]."""
+    lib = lib or load()
+    qd, kd, vd = _f32(q_draft), _f32(k_draft), _f32(v_draft)
+    kc, vc = _f32(k_cache), _f32(v_cache)
+    qo, kvp = _i64(qo_indptr), _i64(kv_indptr)
+    B = len(qo) - 1
+    assert len(kvp) == B + 1
+    idx = None if kv_indices is None else _i32(kv_indices)
+    dm = None if draft_mask is None else _u8(draft_mask).reshape(-1)
+    mi = None if mask_indptr is None else _i64(mask_indptr)
+    NR, Hq, d = qd.shape
+    Hkv = kd.shape[1]
+    assert qo[-1] == NR
+    rows = np.arange(NR, dtype=np.int32) if rows is None else _i32(rows)
+    o = np.zeros((len(rows), Hq, d), dtype=np.float64)
+    lse = np.zeros((len(rows), Hq), dtype=np.float64)
+    nul = ctypes.c_void_p(0)
+    rc = lib.oracle_verify_extend(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kc), _ptr(vc), _ptr(qo),
+                                  _ptr(kvp), nul if idx is None else _ptr(idx),
+                                  nul if dm is None else _ptr(dm), nul if mi is None else _ptr(mi),
+                                  B, Hq, Hkv, d, float(scale), _ptr(rows), len(rows), _ptr(o),
+                                  _ptr(lse), nthreads or default_threads())
+    assert rc == 0, "oracle_verify_extend rejected its arguments"
     return o, lse
 
 

@@ -439,12 +439,36 @@ typedef struct {
     const int32_t *rows;
     double *o, *lse;
     const uint8_t *dmask;  /* NULL: causal draft block; else [B*Ld, Ld], draft j sees i */
+    /* extend form (all three NULL for the uniform, contiguous case):
+     * qo_indptr   request b's draft rows are [qo_indptr[b], qo_indptr[b+1])
+     * kv_indices  prefix position t of the flat kv_indptr range is cache row
+     *             kv_indices[t] (a page table with one token per page)
+     * mask_indptr request b's draft mask starts at dmask[mask_indptr[b]] */
+    const int64_t *qo_indptr;
+    const int32_t *kv_indices;
+    const int64_t *mask_indptr;
 } verify_ctx;
 
 static void verify_row(void *p, int r, double *z, const float **vr, double *o) {
     verify_ctx *c = (verify_ctx *)p;
-    int row = c->rows[r]; /* row = b * Ld + j */
-    int b = row / c->Ld, j = row % c->Ld;
+    int row = c->rows[r]; /* flat draft row: request b, draft j */
+    int b, j, Lb;
+    int64_t q0;
+    if (c->qo_indptr) {
+        b = 0;
+        while (row >= c->qo_indptr[b + 1]) ++b;
+        q0 = c->qo_indptr[b];
+        Lb = (int)(c->qo_indptr[b + 1] - q0);
+    } else {
+        b = row / c->Ld;
+        q0 = (int64_t)b * c->Ld;
+        Lb = c->Ld;
+    }
+    j = (int)(row - q0);
+    /* request b's mask is Lb x Lb, row-major, draft j's row first at mrow */
+    const uint8_t *mrow = NULL;
+    if (c->dmask)
+        mrow = c->dmask + (c->mask_indptr ? c->mask_indptr[b] : q0 * Lb) + (int64_t)j * Lb;
     int64_t p0 = c->indptr ? c->indptr[b] : 0;
     int64_t p1 = c->indptr ? c->indptr[b + 1] : c->shared_len;
     for (int h = 0; h < c->Hq; ++h) {
@@ -452,19 +476,24 @@ static void verify_row(void *p, int r, double *z, const float **vr, double *o) {
         const float *qrow = c->qd + ((size_t)row * c->Hq + h) * c->d;
         int n = 0;
         for (int64_t t = p0; t < p1; ++t) { /* the whole cached prefix */
-            const float *krow = c->kc + ((size_t)t * c->Hkv + kvh) * c->d;
+#if ORACLE_MUTANT == 7
+            int64_t slot = t;  /* planted: the page table is ignored */
+#else
+            int64_t slot = c->kv_indices ? c->kv_indices[t] : t;
+#endif
+            const float *krow = c->kc + ((size_t)slot * c->Hkv + kvh) * c->d;
             z[n] = apply_scale(dot(qrow, krow, c->d), c->scale);
-            vr[n] = c->vc + ((size_t)t * c->Hkv + kvh) * c->d;
+            vr[n] = c->vc + ((size_t)slot * c->Hkv + kvh) * c->d;
             ++n;
         }
 #if ORACLE_MUTANT == 6
-        for (int i = 0; i < c->Ld; ++i) {  /* planted: the draft block is not causal */
+        for (int i = 0; i < Lb; ++i) {  /* planted: the draft block is not causal */
 #else
-        for (int i = 0; i < c->Ld; ++i) {
+        for (int i = 0; i < Lb; ++i) {
             /* drafts 0..j (the causal draft block), or the tree mask's row j */
-            if (c->dmask ? !c->dmask[(size_t)row * c->Ld + i] : i > j) continue;
+            if (mrow ? !mrow[i] : i > j) continue;
 #endif
-            size_t dr = (size_t)b * c->Ld + i;
+            size_t dr = (size_t)q0 + i;
             const float *krow = c->kd + (dr * c->Hkv + kvh) * c->d;
             z[n] = apply_scale(dot(qrow, krow, c->d), c->scale);
             vr[n] = c->vd + (dr * c->Hkv + kvh) * c->d;
@@ -490,7 +519,8 @@ int oracle_verify(const float *qd, const float *kd, const float *vd,
     int64_t maxlen = 0;
     for (int b = 0; b < B; ++b)
         if (indptr[b + 1] - indptr[b] > maxlen) maxlen = indptr[b + 1] - indptr[b];
-    verify_ctx c = {qd, kd, vd, kc, vc, indptr, 0, Ld, Hq, Hkv, d, scale, rows, o, lse, NULL};
+    verify_ctx c = {qd, kd, vd, kc, vc, indptr, 0, Ld, Hq, Hkv, d, scale, rows, o, lse, NULL,
+                     NULL, NULL, NULL};
     run_rows(verify_row, &c, nrows, (int)maxlen + Ld, d, nthreads);
     return 0;
 }
@@ -511,8 +541,44 @@ int oracle_verify_tree(const float *qd, const float *kd, const float *vd,
     int64_t maxlen = 0;
     for (int b = 0; b < B; ++b)
         if (indptr[b + 1] - indptr[b] > maxlen) maxlen = indptr[b + 1] - indptr[b];
-    verify_ctx c = {qd, kd, vd, kc, vc, indptr, 0, Ld, Hq, Hkv, d, scale, rows, o, lse, dmask};
+    verify_ctx c = {qd, kd, vd, kc, vc, indptr, 0, Ld, Hq, Hkv, d, scale, rows, o, lse, dmask,
+                     NULL, NULL, NULL};
     run_rows(verify_row, &c, nrows, (int)maxlen + Ld, d, nthreads);
+    return 0;
+}
+
+/*
+ * Verify in the general extend form of "Split-KV flash-decode attention for
+ * EAGLE target-verify" (the verify entry's signature: qo_indptr, kv_indptr,
+ * kv_indices, custom_mask, mask_indptr; can_handle names ragged extend and
+ * the custom mask as the cases its split path leaves out).
+ *   qo_indptr [B+1]   request b's draft rows are [qo_indptr[b], qo_indptr[b+1])
+ *                     of q/k/v_draft; Lb = their count (0 allowed)
+ *   kv_indptr [B+1]   request b's prefix positions are [kv_indptr[b], kv_indptr[b+1])
+ *   kv_indices        NULL, or prefix position t is cache row kv_indices[t]
+ *   dmask             NULL: causal draft block; else request b's Lb x Lb mask
+ *                     starts at dmask[mask_indptr[b]], draft j sees draft i
+ *                     iff its (j, i) byte is non-zero
+ * Every draft row sees its whole prefix.  rows: flat draft rows to evaluate.
+ */
+int oracle_verify_extend(const float *qd, const float *kd, const float *vd,
+                         const float *kc, const float *vc, const int64_t *qo_indptr,
+                         const int64_t *kv_indptr, const int32_t *kv_indices,
+                         const uint8_t *dmask, const int64_t *mask_indptr, int B, int Hq,
+                         int Hkv, int d, double scale, const int32_t *rows, int nrows,
+                         double *o, double *lse, int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || B < 0 || !qo_indptr || !kv_indptr) return -1;
+    if (dmask && !mask_indptr) return -1;
+    int64_t maxlen = 0, maxld = 1;
+    for (int b = 0; b < B; ++b) {
+        if (kv_indptr[b + 1] - kv_indptr[b] > maxlen) maxlen = kv_indptr[b + 1] - kv_indptr[b];
+        if (qo_indptr[b + 1] - qo_indptr[b] > maxld) maxld = qo_indptr[b + 1] - qo_indptr[b];
+    }
+    for (int r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= qo_indptr[B]) return -1;
+    verify_ctx c = {qd, kd, vd, kc, vc, kv_indptr, 0, 1, Hq, Hkv, d, scale, rows, o, lse, dmask,
+                    qo_indptr, kv_indices, mask_indptr};
+    run_rows(verify_row, &c, nrows, (int)(maxlen + maxld), d, nthreads);
     return 0;
 }
 
@@ -531,7 +597,8 @@ int oracle_verify_shared(const float *qd, const float *kd, const float *vd,
                          const int32_t *rows, int nrows, double *o, double *lse,
                          int nthreads) {
     if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || B < 0 || Ld <= 0 || L < 0) return -1;
-    verify_ctx c = {qd, kd, vd, kp, vp, NULL, L, Ld, Hq, Hkv, d, scale, rows, o, lse, NULL};
+    verify_ctx c = {qd, kd, vd, kp, vp, NULL, L, Ld, Hq, Hkv, d, scale, rows, o, lse, NULL,
+                     NULL, NULL, NULL};
     run_rows(verify_row, &c, nrows, (int)L + Ld, d, nthreads);
     return 0;
 }

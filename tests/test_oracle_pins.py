@@ -259,6 +259,69 @@ def pin_verify_tree_mask(lib):
     return bool(ok)
 
 
+def _random_tree(n, rng):
+    """Ancestor mask of a random tree over n drafts in topological order."""
+    parent = [-1] + [int(rng.integers(-1, j)) for j in range(1, n)]
+    m = np.zeros((n, n), dtype=np.uint8)
+    for j in range(n):
+        a = j
+        while a >= 0:
+            m[j, a] = 1
+            a = parent[a]
+    return m
+
+
+def pin_verify_extend_form(lib):
+    """[SKV] the verify entry's signature (qo_indptr, kv_indptr, kv_indices,
+    custom_mask, mask_indptr) and can_handle (ragged extend and custom masks
+    left out of the split path): ragged draft counts, a prefix read through a
+    token-granular page table, per-request tree masks.  Checked against SDPA
+    on keys gathered with numpy fancy indexing; with a uniform draft count
+    and the identity table it reproduces the contiguous verify exactly."""
+    rng = np.random.default_rng(71)
+    Hq, Hkv, d = 4, 2, 16
+    scale = 1 / math.sqrt(d)
+    Lds = [3, 0, 5, 1]
+    lens = [29, 11, 0, 40]
+    B = len(Lds)
+    qo = np.concatenate([[0], np.cumsum(Lds)]).astype(np.int64)
+    kvp = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    nslots = 120
+    table = rng.permutation(nslots)[:int(kvp[-1])].astype(np.int32)
+    NR = int(qo[-1])
+    q = _rand((NR, Hq, d), 72)
+    kd, vd = _rand((NR, Hkv, d), 73), _rand((NR, Hkv, d), 74)
+    kc, vc = _rand((nslots, Hkv, d), 75), _rand((nslots, Hkv, d), 76)
+    masks = [_random_tree(n, rng) for n in Lds]
+    mi = np.concatenate([[0], np.cumsum([n * n for n in Lds])]).astype(np.int64)
+    flat = np.concatenate([m.reshape(-1) for m in masks]).astype(np.uint8)
+    ok = True
+    for dm, mask_of in ((flat, lambda b: masks[b]), (None, lambda b: np.tril(np.ones((Lds[b],) * 2)))):
+        o, lse = oracle.verify_extend(q, kd, vd, kc, vc, qo, kvp, scale, kv_indices=table,
+                                      draft_mask=dm, mask_indptr=None if dm is None else mi,
+                                      lib=lib)
+        for b in range(B):
+            if Lds[b] == 0:
+                continue
+            sl = slice(int(qo[b]), int(qo[b + 1]))
+            slots = torch.from_numpy(table[kvp[b]:kvp[b + 1]].astype(np.int64))
+            ks = torch.cat([kc[slots], kd[sl]])
+            vs = torch.cat([vc[slots], vd[sl]])
+            mask = torch.ones((Lds[b], lens[b] + Lds[b]), dtype=torch.bool)
+            mask[:, lens[b]:] = torch.from_numpy(mask_of(b).astype(bool))
+            ref = _sdpa(q[sl], _expand_kv(ks, Hq), _expand_kv(vs, Hq), mask, scale)
+            ok &= np.allclose(o[sl], ref, atol=1e-12)
+    # uniform draft count, identity table: the contiguous verify
+    q2, kd2, vd2, kc2, vc2, indptr, Ld = _verify_case(seed=77)
+    B2 = len(indptr) - 1
+    qo2 = np.arange(B2 + 1, dtype=np.int64) * Ld
+    o1, l1 = oracle.verify_extend(q2, kd2, vd2, kc2, vc2, qo2, indptr, 0.3,
+                                  kv_indices=np.arange(int(indptr[-1]), dtype=np.int32), lib=lib)
+    o2, l2 = oracle.verify(q2, kd2, vd2, kc2, vc2, indptr, Ld, 0.3, lib=lib)
+    ok &= np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    return bool(ok)
+
+
 def _split_combine(q, kd, vd, kc, vc, indptr, Ld, scale, nsplit):
     """Split-KV + LSE combine written out per [SKV] implementation item 1:
     stage 1 gives each prefix chunk a normalised partial O and its LSE
@@ -477,7 +540,7 @@ def pin_backward_gradient_equivalence(lib):
 PINS = [pin_golden_masks, pin_golden_tiny_attention, pin_equivalence_route,
         pin_sdpa_random_trees, pin_closed_forms, pin_special_cases,
         pin_brute_force_python, pin_verify_against_sdpa, pin_split_identity,
-        pin_verify_tree_mask, pin_verify_shared_prefix, pin_e4m3_decoder, pin_verify_fp8_cache,
+        pin_verify_tree_mask, pin_verify_extend_form, pin_verify_shared_prefix, pin_e4m3_decoder, pin_verify_fp8_cache,
         pin_backward_finite_differences, pin_backward_gradient_equivalence, pin_sparse_latent]
 
 
@@ -489,8 +552,9 @@ def test_oracle_pin(pin):
 # Planted mistakes (compile-time switches in oracle.c), each of which some
 # pin above must catch: 1 drops the scale, 2 makes causality strict,
 # 3 interleaves GQA heads, 4 hides the prefix from suffixes, 5 drops the
-# row maximum from the LSE, 6 makes the draft block non-causal.
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6])
+# row maximum from the LSE, 6 makes the draft block non-causal, 7 ignores
+# the verify's page table.
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7])
 def test_planted_mistake_is_caught(mutant, tmp_path):
     path = oracle.build(mutant=mutant, out=str(tmp_path / f"liboracle_m{mutant}.so"))
     lib = oracle.load(path)
