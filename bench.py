@@ -408,6 +408,63 @@ class SharedVerifyRunner(Runner):
                                nsplit=self.ns, out=self.o, lse=self.lse, workspace=self.ws)
 
 
+class ExtendVerifyRunner(Runner):
+    """Verify in the extend form: ragged drafts in trees, each prefix read
+    through a token-granular page table (gathered with 16-byte copies)."""
+    unit = "GB/s"
+    bound = "hbm"
+    kernels_per_step = 2
+    kernel_file = "psa_verify.cu"
+
+    def __init__(self, wl: W.ExtendVerifyWorkload, dev):
+        import shared_prefix_attention_b200 as psa
+        self.psa, self.wl, self.dev = psa, wl, dev
+        self.name = wl.name
+        q, kd, vd, kp, vp, idx, mask = wl.make("cpu")
+        self.q, self.kd, self.vd, self.kp, self.vp, self.idx = (
+            t.to(dev) for t in (q, kd, vd, kp, vp, idx))
+        self.mask = None if mask is None else mask.to(dev)
+        i32 = lambda xs: torch.tensor(xs, dtype=torch.int32, device=dev)  # noqa: E731
+        self.qo, self.kvp, self.mi = i32(wl.qo_indptr()), i32(wl.kv_indptr()), i32(wl.mask_indptr())
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=dev)
+        n = psa.verify_workspace_size(1, wl.n_rows, wl.Hq, wl.d, wl.nsplit)
+        self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+
+    def work(self):
+        return float(self.wl.prefix_kv_bytes())
+
+    def step(self):
+        wl = self.wl
+        self.psa.verify_extend(self.q, self.kd, self.vd, self.kp, self.vp, self.qo,
+                               wl.max_draft_len, self.kvp, wl.max_prefix_len, wl.scale,
+                               kv_indices=self.idx, draft_mask=self.mask,
+                               mask_indptr=None if self.mask is None else self.mi,
+                               nsplit=wl.nsplit, out=self.o, lse=self.lse, workspace=self.ws)
+
+    def oracle_sample(self, budget_s: float):
+        import numpy as np
+        import oracle
+        wl = self.wl
+        qo, kvp = wl.qo_indptr(), wl.kv_indptr()
+        host = [t.cpu() for t in (self.q, self.kd, self.vd, self.kp, self.vp, self.idx)]
+        mask = None if self.mask is None else self.mask.cpu()
+        t0 = time.perf_counter()
+        done, n, b = 0.0, 0, 0
+        per_tok = wl.Hkv * wl.d * 2 * 2  # prefix K and V bytes per token
+        while time.perf_counter() - t0 < budget_s and b < wl.B:
+            rows = np.arange(qo[b], qo[b + 1], dtype=np.int32)
+            if len(rows):
+                oracle.verify_extend(*host[:5], qo, kvp, wl.scale, kv_indices=host[5],
+                                     draft_mask=mask,
+                                     mask_indptr=None if mask is None else wl.mask_indptr(),
+                                     rows=rows)
+            done += per_tok * wl.prefix_lens[b]
+            n += 1
+            b += 1
+        return done, time.perf_counter() - t0, f"{n} whole requests"
+
+
 VERIFY_SMALL = W.VerifyWorkload("verify B=8 L=16384 drafts=4 H=32/8 d=128 splits=32 bf16", B=8,
                                 L=16384, Ld=4, Hq=32, Hkv=8, d=128, nsplit=32, seed=4)
 SPARSE_SMALL = W.SparseLatentWorkload("sparse T=4096 H=64 dl=512 topk=2048 bf16", T=4096, H=64,
@@ -423,6 +480,7 @@ def make_runner(name: str, dev):
             "verify": lambda: VerifyRunner(W.VERIFY, dev),
             "verify-shared": lambda: SharedVerifyRunner(W.VERIFY_SHARED, dev),
             "verify-fp8": lambda: VerifyFp8Runner(W.VERIFY_FP8, dev),
+            "verify-extend": lambda: ExtendVerifyRunner(W.VERIFY_PAGED, dev),
             "grpo-backward": lambda: BackwardRunner(W.GRPO, dev),
             "sparse": lambda: SparseRunner(W.SPARSE, dev)}[name]()
 
@@ -501,7 +559,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="grpo",
                     choices=["grpo", "tiny", "large", "verify", "verify8", "verify-shared",
-                             "verify-fp8", "grpo-backward", "sparse", "sparse4k"])
+                             "verify-fp8", "verify-extend", "grpo-backward", "sparse",
+                             "sparse4k"])
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -552,7 +611,8 @@ def main():
 
     if not args.no_extras and args.workload == "grpo":
         extras = {}
-        for name in ("verify", "verify-fp8", "verify-shared", "large", "grpo-backward", "sparse"):
+        for name in ("verify", "verify-fp8", "verify-extend", "verify-shared", "large",
+                     "grpo-backward", "sparse"):
             try:
                 r = make_runner(name, dev)
                 v, m, rf = measure(r, max(3, min(args.steps, 10)), 3, flush, dist_on, world,

@@ -236,14 +236,18 @@ size_t psa_verify_workspace_size(int32_t B, int32_t Ld, int32_t Hq, int32_t head
 /*
  *   q_draft          device [B*Ld, Hq, d] bf16   draft-token queries, request-major
  *   k_draft, v_draft device [B*Ld, Hkv, d] bf16  draft-token keys/values
- *   k_cache, v_cache device [Ntok, Hkv, d] bf16  cached prefix, one contiguous
- *                                                token range per request
+ *   k_cache, v_cache device [Ntok, Hkv, d] bf16  the KV cache (token rows)
  *   n_cache_tokens   host value Ntok (rows of k_cache / v_cache)
- *   dev_kv_indptr    device int32 [B+1]         request b's prefix is cache tokens
+ *   dev_kv_indptr    device int32 [B+1]         request b's prefix positions are
  *                                                [indptr[b], indptr[b+1])
  *   max_prefix_len   host value >= every prefix length (no device sync is made)
- *   kv_indices       must be NULL (paged caches are not implemented:
- *                    PSA_ERR_UNSUPPORTED)
+ *   kv_indices       NULL: prefix position t is cache row t (one contiguous
+ *                    range per request, streamed with TMA tiles); else device
+ *                    int32 [indptr[B]], a page table with one token per page:
+ *                    position t is cache row kv_indices[t] ([SKV] the verify
+ *                    entry's kv_indptr / kv_indices pair).  Rows are gathered
+ *                    with 16-byte copies; a row outside [0, Ntok) reads as
+ *                    zeros and sets PSA_ERR_INVALID_ARG in dev_status.
  *   o                device [B*Ld, Hq, d] bf16   (written)
  *   lse              device [B*Ld, Hq] fp32      (written; nullable)
  * Draft j of request b sees the whole prefix of b plus drafts 0..j.
@@ -280,6 +284,43 @@ int psa_verify_tree_fwd(const void *q_draft, const void *k_draft, const void *v_
                         int32_t head_dim, float scale, int32_t nsplit,
                         const psa_verify_features *features, void *workspace, size_t ws_bytes,
                         int32_t *dev_status, void *stream);
+
+/*
+ * Verify in the general extend form ([SKV] the verify entry's signature:
+ * qo_indptr, kv_indptr, kv_indices, custom_mask, mask_indptr; can_handle
+ * names ragged extend and custom masks as what its split path leaves out):
+ * per-request draft counts, an optional page table and optional tree masks.
+ *   q_draft          device [n_rows, Hq, d] bf16   draft rows, request-major
+ *   k_draft, v_draft device [n_rows, Hkv, d] bf16
+ *   dev_qo_indptr    device int32 [B+1]: request b's drafts are rows
+ *                    [qo_indptr[b], qo_indptr[b+1]); qo_indptr[B] == n_rows
+ *   n_rows           host value, the total draft rows
+ *   max_draft_len    host value >= every draft count (the m-tile plan uses
+ *                    it: max_draft_len * Hq / Hkv <= 128).  A count above it
+ *                    or a decreasing qo_indptr sets PSA_ERR_INVALID_ARG in
+ *                    dev_status; those rows are not written.
+ *   dev_kv_indptr, max_prefix_len, dev_kv_indices: as psa_verify_fwd
+ *   dev_draft_mask   NULL: each request's draft block is causal; else device
+ *                    uint8, request b's Lb x Lb block (row-major, Lb its draft
+ *                    count) starting at dev_draft_mask[mask_indptr[b]]: draft
+ *                    j sees draft i iff its (j, i) byte is non-zero
+ *   dev_mask_indptr  device int32 [B+1] (required with a mask)
+ *   o, lse           device [n_rows, Hq, d] bf16 / [n_rows, Hq] fp32
+ * features->ragged_extend and ->has_custom_mask may be set here.  The
+ * workspace holds the partials of n_rows rows:
+ * psa_verify_workspace_size(1, n_rows, Hq, d, nsplit) bytes.  Every draft row
+ * sees its request's whole prefix; a row that sees no key gets O = 0 and
+ * LSE = -inf.  Other arguments and statuses as psa_verify_fwd.
+ */
+int psa_verify_extend_fwd(const void *q_draft, const void *k_draft, const void *v_draft,
+                          const void *k_cache, const void *v_cache, int64_t n_cache_tokens,
+                          const int32_t *dev_qo_indptr, int32_t n_rows, int32_t max_draft_len,
+                          const int32_t *dev_kv_indptr, int64_t max_prefix_len,
+                          const int32_t *dev_kv_indices, const uint8_t *dev_draft_mask,
+                          const int32_t *dev_mask_indptr, void *o, float *lse, int32_t B,
+                          int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
+                          int32_t nsplit, const psa_verify_features *features,
+                          void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
 
 /* Size of the library's fixed device scratch used by psa_verify_fwd_noalloc:
  * 16 MiB, held by every GPU that loads the library until the process exits. */

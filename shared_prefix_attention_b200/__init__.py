@@ -10,7 +10,7 @@ from ._binding import (  # noqa: F401
     lib, plan_prefill, prefill, prefill_tiles, read_status, sparse_latent, spec_flat,
     status_string, verify, verify_auto_splits, verify_noalloc, verify_workspace_size,
     wait_selftest, verify_shared, verify_shared_auto_splits, verify_fp8, transpose_spec,
-    prefill_bwd, plan_prefill_bwd, prefill_bwd_tiles, verify_tree,
+    prefill_bwd, plan_prefill_bwd, prefill_bwd_tiles, verify_tree, verify_extend,
     PSA_OK, PSA_ERR_INVALID_ARG, PSA_ERR_UNSUPPORTED, PSA_ERR_WORKSPACE, PSA_ERR_CUDA,
     PSA_ERR_TIMEOUT, PSA_ERR_CAPACITY, PSA_BF16, PSA_F32,
 )

@@ -34,6 +34,7 @@ EXPORTS = [
     "psa_wait_selftest", "psa_verify_shared_auto_splits", "psa_verify_shared_fwd",
     "psa_verify_fp8_fwd", "psa_transpose_spec", "psa_prefill_bwd_tiles",
     "psa_prefill_bwd_workspace_size", "psa_prefill_bwd", "psa_verify_tree_fwd",
+    "psa_verify_extend_fwd",
 ]
 
 
@@ -98,6 +99,8 @@ def lib():
         "psa_prefill_bwd_tiles": ([I32, P, P], ctypes.c_int),
         "psa_verify_tree_fwd": ([P, P, P, P, P, I64, P, I64, P, P, P, P, I32, I32, I32, I32, I32,
                                  F, I32, P, P, SZ, P, P], ctypes.c_int),
+        "psa_verify_extend_fwd": ([P, P, P, P, P, I64, P, I32, I32, P, I64, P, P, P, P, P, I32,
+                                   I32, I32, I32, F, I32, P, P, SZ, P, P], ctypes.c_int),
         "psa_prefill_bwd_workspace_size": ([I32, I32], SZ),
         "psa_prefill_bwd": ([P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, F, P, I64, P, I64, P,
                              SZ, P, P], ctypes.c_int),
@@ -406,7 +409,8 @@ def prefill_bwd(q, k, v, o, lse, dout, schedules, scale: float, dq=None, dk=None
 
 def verify_tree(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr: torch.Tensor,
                 max_prefix_len: int, draft_mask: torch.Tensor, scale: float, Ld: int,
-                nsplit: int = 0, out=None, lse=None, workspace=None, status=None):
+                nsplit: int = 0, out=None, lse=None, workspace=None, status=None,
+                kv_indices=None):
     """Split-KV verify with a custom draft mask (device uint8 [B*Ld, Ld])."""
     _require_cuda(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr, draft_mask)
     BL, Hq, d = q_draft.shape
@@ -421,9 +425,40 @@ def verify_tree(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr: torch.Te
     feat = VerifyFeatures(1, 1, -1, 0, 0.0, -1, 0)
     rc = lib().psa_verify_tree_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft), _ptr(k_cache),
                                    _ptr(v_cache), k_cache.shape[0], _ptr(kv_indptr),
-                                   int(max_prefix_len), None, _ptr(draft_mask), _ptr(out),
+                                   int(max_prefix_len), _ptr(kv_indices), _ptr(draft_mask),
+                                   _ptr(out),
                                    _ptr(lse), B, Ld, Hq, Hkv, d, float(scale), ns,
                                    ctypes.byref(feat), _ptr(workspace), workspace.numel(),
                                    _ptr(status), _stream(q_draft.device))
     _check(rc, "psa_verify_tree_fwd")
+    return out, lse
+
+
+def verify_extend(q_draft, k_draft, v_draft, k_cache, v_cache, qo_indptr: torch.Tensor,
+                  max_draft_len: int, kv_indptr: torch.Tensor, max_prefix_len: int,
+                  scale: float, kv_indices=None, draft_mask=None, mask_indptr=None,
+                  nsplit: int = 0, out=None, lse=None, workspace=None, status=None):
+    """Verify in the extend form: ragged draft counts (qo_indptr, device int32
+    [B+1]), an optional page table (kv_indices: prefix position t is cache row
+    kv_indices[t]) and optional per-request tree masks (flat device uint8,
+    request b's Lb x Lb block at mask_indptr[b])."""
+    _require_cuda(q_draft, k_draft, v_draft, k_cache, v_cache, qo_indptr, kv_indptr)
+    NR, Hq, d = q_draft.shape
+    Hkv = k_draft.shape[1]
+    B = qo_indptr.numel() - 1
+    ns = nsplit or verify_auto_splits(B, max_prefix_len, Hkv, d)
+    out = torch.empty_like(q_draft) if out is None else out
+    lse = torch.empty((NR, Hq), dtype=torch.float32, device=q_draft.device) if lse is None else lse
+    if workspace is None:
+        workspace = torch.empty(max(verify_workspace_size(1, NR, Hq, d, ns), 256),
+                                dtype=torch.uint8, device=q_draft.device)
+    feat = VerifyFeatures(int(draft_mask is not None), 1, -1, 0, 0.0, -1, 1)
+    rc = lib().psa_verify_extend_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft),
+                                     _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
+                                     _ptr(qo_indptr), NR, int(max_draft_len), _ptr(kv_indptr),
+                                     int(max_prefix_len), _ptr(kv_indices), _ptr(draft_mask),
+                                     _ptr(mask_indptr), _ptr(out), _ptr(lse), B, Hq, Hkv, d,
+                                     float(scale), ns, ctypes.byref(feat), _ptr(workspace),
+                                     workspace.numel(), _ptr(status), _stream(q_draft.device))
+    _check(rc, "psa_verify_extend_fwd")
     return out, lse

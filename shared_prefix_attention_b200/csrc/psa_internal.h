@@ -40,6 +40,11 @@ struct VerifyArgs {
   int32_t* status;
   cudaStream_t stream;
   const uint8_t* dmask = nullptr;  // tree verify: [B*Ld, Ld] draft mask (device)
+  // Extend form (all null for uniform draft counts and a contiguous prefix):
+  const int32_t* kv_indices = nullptr;   // prefix position t -> cache row kv_indices[t]
+  const int32_t* qo_indptr = nullptr;    // [B+1] draft rows per request; Ld is their maximum
+  const int32_t* mask_indptr = nullptr;  // [B+1] start of request b's Lb x Lb mask in dmask
+  int32_t n_rows = 0;                    // draft rows in all (qo_indptr[B]); B*Ld when uniform
 };
 
 // KV heads per CTA, 16-row m-tiles per CTA and row blocks per KV head;

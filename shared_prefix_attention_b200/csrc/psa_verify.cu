@@ -37,8 +37,16 @@ constexpr int kTileKeys = 16;      // keys per pipeline stage
 __host__ __device__ constexpr int max_consumer_warps(int D) { return D > 128 ? 4 : 8; }
 
 struct Stage1Params {
-  const __nv_bfloat16* q;  // [B*Ld, Hq, D]
+  const __nv_bfloat16* q;  // [nrows, Hq, D]
   const int32_t* indptr;   // [B+1]
+  // Page table (nullable): prefix position t is cache row kv_indices[t];
+  // those rows are gathered with cp.async instead of TMA tiles.
+  const int32_t* kv_indices;
+  const __nv_bfloat16* kc;  // [ntok, Hkv, D], read directly only when paged
+  const __nv_bfloat16* vc;
+  int64_t ntok;
+  const int32_t* qo_indptr;  // nullable: request b's draft rows are b*Ld + [0, Ld)
+  int32_t nrows;             // draft rows in all
   float* part_o;
   float* part_lse;
   int32_t B, Ld, Hq, Hkv, G, R;
@@ -66,18 +74,70 @@ __device__ __forceinline__ Unit decode_unit(const Stage1Params& p, int u) {
   return x;
 }
 
+// First draft row and draft count of request b (Ld is the maximum count).
+// A count above Ld is reported and clamped; a decreasing qo_indptr or rows
+// outside [0, nrows) are reported and the request is treated as empty.
+__device__ __forceinline__ void request_rows(const int32_t* qo_indptr, int Ld, int nrows, int b,
+                                             int& q0, int& Lb, int32_t* status) {
+  if (!qo_indptr) {
+    q0 = b * Ld;
+    Lb = Ld;
+    return;
+  }
+  q0 = __ldg(qo_indptr + b);
+  Lb = __ldg(qo_indptr + b + 1) - q0;
+  if (Lb > Ld) {
+    report_status(status, PSA_ERR_INVALID_ARG);
+    Lb = Ld;
+  }
+  if (Lb < 0 || q0 < 0 || q0 > nrows - Lb) {
+    report_status(status, PSA_ERR_INVALID_ARG);
+    Lb = 0;
+  }
+}
+
+// A unit does work only if its row block holds a draft row of the request.
+__device__ __forceinline__ bool unit_live(const Stage1Params& p, const Unit& x, int Lb) {
+  return x.rb * p.MT * 16 < Lb * p.G;
+}
+
 __device__ __forceinline__ void split_range(const Stage1Params& p, int b, int s, int32_t& t0,
                                             int32_t& t1) {
   const int32_t a = __ldg(p.indptr + b), e = __ldg(p.indptr + b + 1);
-  const int32_t L = e - a;
+  int32_t L = e - a;
+  // a paged prefix must lie inside the page table, whose length is indptr[B]
+  if (L < 0 || a < 0 || (p.kv_indices && e > __ldg(p.indptr + p.B))) L = 0;
   int32_t c = (L + p.nsplit - 1) / p.nsplit;
   c = (c + kTileKeys - 1) / kTileKeys * kTileKeys;
   t0 = a + min(L, s * c);
   t1 = a + min(L, (s + 1) * c);
 }
 
-template <int D>
-__global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
+// Shared-memory layout of one stage (K then V, 16 keys each):
+//  - contiguous prefix: TMA tiles with 128-byte swizzling, [D/64][HB][key][64];
+//  - paged prefix: one bulk copy per key of its HB heads (HB*D*2 bytes), rows
+//    padded by 16 bytes so the 8 rows an ldmatrix reads fall in distinct banks.
+// Producer warps of the paged layout: bulk copies issued by the lanes of one
+// warp go out one after another, so the keys of a tile are spread over
+// several warps (each fills kTileKeys / kPagedProducers keys, K and V).
+constexpr int kPagedProducers = 4;
+
+template <bool PAGED>
+__host__ __device__ constexpr int producer_warps() { return PAGED ? kPagedProducers : 1; }
+
+template <int D, bool PAGED>
+__device__ __forceinline__ uint32_t kv_row_stride(int HB) {
+  return PAGED ? uint32_t(HB) * D * 2 + 16 : 0u;
+}
+
+template <int D, bool PAGED>
+__host__ __device__ constexpr uint32_t stage_kv_bytes(int HB) {
+  return PAGED ? uint32_t(kTileKeys) * (uint32_t(HB) * D * 2 + 16)
+               : uint32_t(D / 64) * HB * kTileKeys * 128;
+}
+
+template <int D, bool PAGED>
+__global__ void __launch_bounds__((max_consumer_warps(D) + producer_warps<PAGED>()) * 32, 1)
     verify_stage1_kernel(const __grid_constant__ CUtensorMap tmap_k,
                          const __grid_constant__ CUtensorMap tmap_v, Stage1Params p) {
   constexpr int KSTEPS = D / 16;  // MMA k-steps over the head dimension
@@ -89,8 +149,9 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
 
   const int NW = p.HB * p.MT;
   const uint32_t head_bytes = kTileKeys * 128;                // one head, one part
-  const uint32_t kv_bytes = uint32_t(NPART) * p.HB * head_bytes;  // K (or V) per stage
+  const uint32_t kv_bytes = stage_kv_bytes<D, PAGED>(p.HB);    // K (or V) per stage
   const uint32_t stage_bytes = 2 * kv_bytes;
+  const uint32_t row_stride = kv_row_stride<D, PAGED>(p.HB);   // paged layout only
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.nstage * stage_bytes);
   uint64_t* empty = full + p.nstage;
 
@@ -98,7 +159,8 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int i = 0; i < p.nstage; ++i) {
-      mbar_init(&full[i], 1);
+      // one arrival with the byte count per producer warp
+      mbar_init(&full[i], producer_warps<PAGED>());
       mbar_init(&empty[i], NW);
     }
     fence_barrier_init();
@@ -107,9 +169,97 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
 
   const int units = p.B * p.nsplit * p.nrb * p.nhb;
 
-  if (warp == NW) {
+  if (warp >= NW) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if constexpr (PAGED) {
+      // Paged prefix: producer warp pw fills keys [pw*TPW, (pw+1)*TPW) of
+      // each tile; its lane l < TPW copies key l's K row, lane TPW + l its V
+      // row (the key's HB heads, one bulk copy).  A key past the split end,
+      // or a cache row outside [0, ntok) (reported), is written as zeros.
+      constexpr int TPW = kTileKeys / kPagedProducers;
+      const int pw = warp - NW;
+      const bool active = lane < 2 * TPW;
+      const int tok = pw * TPW + lane % TPW;
+      const bool is_v = (lane / TPW) & 1;
+      const uint32_t row_bytes = uint32_t(p.HB) * D * 2;
+      const __nv_bfloat16* cache = is_v ? p.vc : p.kc;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int last_phase[8];
+      for (int i = 0; i < 8; ++i) last_phase[i] = -1;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const Unit x = decode_unit(p, u);
+        int q0, Lb;
+        request_rows(p.qo_indptr, p.Ld, p.nrows, x.b, q0, Lb, p.status);
+        if (!unit_live(p, x, Lb)) continue;
+        int32_t t0, t1;
+        split_range(p, x.b, x.s, t0, t1);
+        // The page-table entries are read kPrefetch tiles ahead, so a
+        // stage's copies never wait on the latency of its own lookups.
+        constexpr int kPrefetch = 8;
+        int32_t cur[kPrefetch], nxt[kPrefetch];
+        auto lookup = [&](int32_t tb, int32_t (&dst)[kPrefetch]) {
+#pragma unroll
+          for (int k = 0; k < kPrefetch; ++k) {
+            const int32_t pos = tb + k * kTileKeys + tok;
+            dst[k] = pos < t1 ? __ldg(p.kv_indices + pos) : -1;
+          }
+        };
+        lookup(t0, cur);
+        for (int32_t tb = t0; tb < t1 && ok; tb += kPrefetch * kTileKeys) {
+          if (tb + kPrefetch * kTileKeys < t1) lookup(tb + kPrefetch * kTileKeys, nxt);
+#pragma unroll
+          for (int k = 0; k < kPrefetch; ++k) {
+            if (tb + k * kTileKeys >= t1) break;
+            // every lane acquires the released stage before writing into it
+            const bool w = mbar_wait(&empty[stage], phase ^ 1, &abort_flag, p.status);
+            if (!__all_sync(0xffffffffu, w)) {
+              ok = false;
+              break;
+            }
+            last_phase[stage] = int(phase);
+            int32_t slot = cur[k];
+            if (slot >= p.ntok || (slot < 0 && tb + k * kTileKeys + tok < t1)) {
+              report_status(p.status, PSA_ERR_INVALID_ARG);
+              slot = -1;
+            }
+            uint8_t* dst =
+                smem + stage * stage_bytes + (is_v ? kv_bytes : 0u) + tok * row_stride;
+            if (active && slot < 0) {
+              const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+              for (uint32_t o = 0; o < row_bytes; o += 16)
+                *reinterpret_cast<uint4*>(dst + o) = z;
+              fence_proxy_async_smem();  // later bulk copies land after these stores
+            }
+            // one arrival per warp announces the bytes of all its copies,
+            // before any of them is issued
+            const uint32_t copies = __popc(__ballot_sync(0xffffffffu, active && slot >= 0));
+            if (lane == 0) mbar_arrive_expect_tx(&full[stage], copies * row_bytes);
+            __syncwarp();
+            if (active && slot >= 0)
+              bulk_load(dst, cache + (size_t(slot) * p.Hkv + x.hb * p.HB) * D, row_bytes,
+                        &full[stage]);
+            if (++stage == p.nstage) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kPrefetch; ++k) cur[k] = nxt[k];
+        }
+      }
+      if (!ok && lane == 0 && pw == 0) {
+        // Let copies already in flight land before the CTA exits.
+        for (int i = 0; i < p.nstage; ++i) {
+          if (last_phase[i] < 0) continue;
+          const uint64_t w0 = globaltimer();
+          while (!mbar_try_wait(&full[i], uint32_t(last_phase[i])) &&
+                 globaltimer() - w0 < kWaitTimeoutNs) {
+          }
+        }
+      }
+    } else if (lane == 0) {
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
       int stage = 0;
@@ -120,6 +270,9 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const Unit x = decode_unit(p, u);
         const int hb = x.hb;
+        int q0, Lb;
+        request_rows(p.qo_indptr, p.Ld, p.nrows, x.b, q0, Lb, nullptr);
+        if (!unit_live(p, x, Lb)) continue;
         int32_t t0, t1;
         split_range(p, x.b, x.s, t0, t1);
         for (int32_t t = t0; t < t1; t += kTileKeys) {
@@ -162,7 +315,7 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
   const int hh = warp / p.MT;  // KV head within the block
   const int mt = warp % p.MT;  // 16-row m-tile of that head's rows
   const int g = lane >> 2, c = lane & 3;
-  const int BL = p.B * p.Ld;
+  const int BL = p.nrows;
   int stage = 0;
   uint32_t phase = 0;
 
@@ -170,6 +323,9 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
     const Unit x = decode_unit(p, u);
     const int b = x.b, s = x.s;
     const int kvh = x.hb * p.HB + hh;
+    int q0, Lb;
+    request_rows(p.qo_indptr, p.Ld, p.nrows, b, q0, Lb, nullptr);
+    if (!unit_live(p, x, Lb)) continue;
     int32_t t0, t1;
     split_range(p, b, s, t0, t1);
 
@@ -179,10 +335,10 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int rr = (x.rb * p.MT + mt) * 16 + g + 8 * i;
-      rvalid[i] = rr < p.R;
+      rvalid[i] = rr < Lb * p.G;
       const int j = rvalid[i] ? rr / p.G : 0;
       rqh[i] = kvh * p.G + (rvalid[i] ? rr % p.G : 0);
-      rrow[i] = b * p.Ld + j;
+      rrow[i] = q0 + j;
     }
 
     // Q fragments for every k-step (A operand, row-major 16x16 per step)
@@ -212,8 +368,14 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
         ok = false;
         break;
       }
-      const uint32_t kbase = smem_u32(smem + stage * stage_bytes) + hh * head_bytes;
+      const uint32_t kbase =
+          smem_u32(smem + stage * stage_bytes) + hh * (PAGED ? uint32_t(D) * 2 : head_bytes);
       const uint32_t vbase = kbase + kv_bytes;
+      // byte address of 16-byte chunk `chunk` of key `key` in a K or V tile
+      auto at = [&](uint32_t base, uint32_t key, uint32_t chunk) {
+        return PAGED ? base + key * row_stride + chunk * 16
+                     : base + (chunk >> 3) * (p.HB * head_bytes) + sw128(key, chunk & 7);
+      };
 
       // S = Q K^T over 16 keys: two n-tiles of 8 keys
       float sc[2][4];
@@ -224,8 +386,7 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ks += 2) {
           const uint32_t chunk = ks * 2 + (lane >> 3);  // 16-byte chunk of the head dim
-          const uint32_t addr =
-              kbase + (chunk >> 3) * (p.HB * head_bytes) + sw128(key, chunk & 7);
+          const uint32_t addr = at(kbase, key, chunk);
           uint32_t b0, b1, b2, b3;
           ldmatrix_x4(addr, b0, b1, b2, b3);
           mma_bf16_16816(sc[nt], qa[ks], b0, b1);
@@ -281,8 +442,7 @@ __global__ void __launch_bounds__((max_consumer_warps(D) + 1) * 32, 1)
 #pragma unroll
         for (int dt = 0; dt < D / 8; dt += 2) {
           const uint32_t chunk = dt + (mi >> 1);
-          const uint32_t addr =
-              vbase + (chunk >> 3) * (p.HB * head_bytes) + sw128(key, chunk & 7);
+          const uint32_t addr = at(vbase, key, chunk);
           uint32_t b0, b1, b2, b3;
           ldmatrix_x4_trans(addr, b0, b1, b2, b3);
           mma_bf16_16816(acc[dt], pa, b0, b1);
@@ -329,9 +489,12 @@ struct Stage2Params {
   const float* part_lse;
   __nv_bfloat16* o;
   float* lse;
-  const uint8_t* dmask;  // nullable: causal draft block; else [B*Ld, Ld] tree mask
-  int32_t B, Ld, Hq, Hkv, G, nsplit;
+  const uint8_t* dmask;  // nullable: causal draft block; else a tree mask per request
+  const int32_t* qo_indptr;    // nullable: request b's draft rows are b*Ld + [0, Ld)
+  const int32_t* mask_indptr;  // nullable: request b's mask starts at b*Ld*Ld
+  int32_t B, Ld, Hq, Hkv, G, nsplit, nrows;
   float scale_log2;
+  int32_t* status;
 };
 
 template <int D>
@@ -339,10 +502,25 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
   constexpr int E = D / 32;  // head-dim elements per lane
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int BL = p.B * p.Ld;
+  const int BL = p.nrows;
   if (gw >= BL * p.Hq) return;
   const int row = gw / p.Hq, qh = gw % p.Hq;
-  const int b = row / p.Ld, j = row % p.Ld;
+  int b;
+  if (p.qo_indptr) {
+    // the last request whose first row is <= row (empty requests are passed over)
+    int lo = 0, hi = p.B;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(p.qo_indptr + mid) <= row) lo = mid; else hi = mid;
+    }
+    b = lo;
+  } else {
+    b = row / p.Ld;
+  }
+  int q0, Lb;
+  request_rows(p.qo_indptr, p.Ld, p.nrows, b, q0, Lb, lane == 0 ? p.status : nullptr);
+  const int j = row - q0;
+  if (j >= Lb) return;  // only after a reported inconsistent qo_indptr
   const int kvh = qh / p.G;
 
   float qv[E];
@@ -354,7 +532,7 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
 
   // draft keys 0..j (the causal draft-draft block), log2-domain logits
   auto draft_logit = [&](int i) {
-    const __nv_bfloat16* kp = p.kd + (size_t(b * p.Ld + i) * p.Hkv + kvh) * D + lane * E;
+    const __nv_bfloat16* kp = p.kd + (size_t(q0 + i) * p.Hkv + kvh) * D + lane * E;
     float sdot = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) sdot += qv[e] * __bfloat162float(kp[e]);
@@ -363,9 +541,12 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
     return sdot * p.scale_log2;
   };
   // the draft block: drafts 0..j, or the tree mask's row (the same for every head)
-  const uint8_t* mrow = p.dmask ? p.dmask + size_t(row) * p.Ld : nullptr;
+  const uint8_t* mrow = nullptr;
+  if (p.dmask)
+    mrow = p.dmask + (p.mask_indptr ? size_t(__ldg(p.mask_indptr + b)) : size_t(q0) * Lb) +
+           size_t(j) * Lb;
   auto sees = [&](int i) { return mrow ? __ldg(mrow + i) != 0 : i <= j; };
-  const int nd = mrow ? p.Ld : j + 1;
+  const int nd = mrow ? Lb : j + 1;
   float M = -INFINITY;
   for (int i = 0; i < nd; ++i)
     if (sees(i)) M = fmaxf(M, draft_logit(i));
@@ -403,7 +584,7 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
   for (int i = 0; i < nd; ++i) {
     if (!sees(i)) continue;
     const float w = fast_exp2(draft_logit(i) - M);
-    const __nv_bfloat16* vp = p.vd + (size_t(b * p.Ld + i) * p.Hkv + kvh) * D + lane * E;
+    const __nv_bfloat16* vp = p.vd + (size_t(q0 + i) * p.Hkv + kvh) * D + lane * E;
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] += w * __bfloat162float(vp[e]);
     wsum += w;
@@ -426,7 +607,9 @@ int launch_verify_d(const VerifyArgs& a, int HB, int MT, int NRB) {
   const int nhb = a.Hkv / HB;
 
   CUtensorMap tk, tv;
-  const uint64_t dims[3] = {uint64_t(D), uint64_t(a.n_cache_tokens), uint64_t(a.Hkv)};
+  // a tensor map needs a non-empty extent (an empty cache is never read)
+  const uint64_t rows = a.n_cache_tokens > 0 ? uint64_t(a.n_cache_tokens) : 1u;
+  const uint64_t dims[3] = {uint64_t(D), rows, uint64_t(a.Hkv)};
   const uint64_t strides[2] = {uint64_t(a.Hkv) * D * 2, uint64_t(D) * 2};
   const uint32_t box[3] = {64u, uint32_t(kTileKeys), uint32_t(HB)};
   int rc = encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.kc, dims, strides, box,
@@ -439,6 +622,12 @@ int launch_verify_d(const VerifyArgs& a, int HB, int MT, int NRB) {
   Stage1Params p1;
   p1.q = static_cast<const __nv_bfloat16*>(a.q);
   p1.indptr = a.indptr;
+  p1.kv_indices = a.kv_indices;
+  p1.kc = static_cast<const __nv_bfloat16*>(a.kc);
+  p1.vc = static_cast<const __nv_bfloat16*>(a.vc);
+  p1.ntok = a.n_cache_tokens;
+  p1.qo_indptr = a.qo_indptr;
+  p1.nrows = a.qo_indptr ? a.n_rows : a.B * a.Ld;
   p1.part_o = a.part_o;
   p1.part_lse = a.part_lse;
   p1.B = a.B;
@@ -455,14 +644,16 @@ int launch_verify_d(const VerifyArgs& a, int HB, int MT, int NRB) {
   p1.scale_log2 = a.scale * kLog2e;
   p1.status = a.status;
 
-  const size_t stage_bytes = size_t(2) * (D / 64) * HB * kTileKeys * 128;
+  const bool paged = a.kv_indices != nullptr;
+  const size_t stage_bytes =
+      size_t(2) * (paged ? stage_kv_bytes<D, true>(HB) : stage_kv_bytes<D, false>(HB));
   const size_t budget = 200 * 1024;
   int nstage = int(budget / stage_bytes);
   nstage = nstage > 8 ? 8 : nstage;
   if (nstage < 2) return PSA_ERR_UNSUPPORTED;
   p1.nstage = nstage;
   const size_t smem = 1024 + nstage * stage_bytes + 2 * nstage * sizeof(uint64_t);
-  auto k1 = verify_stage1_kernel<D>;
+  auto k1 = paged ? verify_stage1_kernel<D, true> : verify_stage1_kernel<D, false>;
   if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
     return PSA_ERR_CUDA;
@@ -470,7 +661,7 @@ int launch_verify_d(const VerifyArgs& a, int HB, int MT, int NRB) {
   int grid = sm_count(dev);
   if (grid <= 0) return PSA_ERR_CUDA;
   grid = units < grid ? units : grid;
-  const int threads = (HB * MT + 1) * 32;
+  const int threads = (HB * MT + (paged ? producer_warps<true>() : 1)) * 32;
   if (units > 0) {
     k1<<<grid, threads, smem, a.stream>>>(tk, tv, p1);
     if (cudaGetLastError() != cudaSuccess) return PSA_ERR_CUDA;
@@ -494,6 +685,10 @@ int launch_combine_d(const VerifyArgs& a) {
   p2.o = static_cast<__nv_bfloat16*>(a.o);
   p2.lse = a.lse;
   p2.dmask = a.dmask;
+  p2.qo_indptr = a.qo_indptr;
+  p2.mask_indptr = a.mask_indptr;
+  p2.nrows = a.qo_indptr ? a.n_rows : a.B * a.Ld;
+  p2.status = a.status;
   p2.B = a.B;
   p2.Ld = a.Ld;
   p2.Hq = a.Hq;
@@ -501,7 +696,7 @@ int launch_combine_d(const VerifyArgs& a) {
   p2.G = G;
   p2.nsplit = a.nsplit;
   p2.scale_log2 = a.scale * kLog2e;
-  const int warps = a.B * a.Ld * a.Hq;
+  const int warps = p2.nrows * a.Hq;
   const int blocks = (warps + 7) / 8;
   if (blocks > 0) {
     verify_stage2_kernel<D><<<blocks, 256, 0, a.stream>>>(p2);

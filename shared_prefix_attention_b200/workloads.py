@@ -267,6 +267,107 @@ class SharedVerifyWorkload:
 
 
 @dataclass
+class ExtendVerifyWorkload:
+    """Speculative verify in the extend form: per-request draft counts, each
+    request's prefix scattered over a token-granular KV pool through a page
+    table (distinct random pool rows), and optionally a random draft tree per
+    request (draft j's parent drawn uniformly from the prefix and drafts
+    0..j-1; a draft sees its ancestors and itself)."""
+    name: str
+    draft_lens: list[int]
+    prefix_lens: list[int]
+    Hq: int
+    Hkv: int
+    d: int
+    nsplit: int = 0
+    tree: bool = True
+    pool_slack: float = 1.25     # pool rows per prefix token
+    dtype: torch.dtype = torch.bfloat16
+    sigma: float = 0.5
+    seed: int = 8
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def B(self) -> int:
+        return len(self.draft_lens)
+
+    @property
+    def n_rows(self) -> int:
+        return sum(self.draft_lens)
+
+    @property
+    def max_draft_len(self) -> int:
+        return max(self.draft_lens + [1])
+
+    @property
+    def max_prefix_len(self) -> int:
+        return max(self.prefix_lens + [0])
+
+    @staticmethod
+    def _indptr(xs) -> list[int]:
+        out = [0]
+        for n in xs:
+            out.append(out[-1] + n)
+        return out
+
+    def qo_indptr(self) -> list[int]:
+        return self._indptr(self.draft_lens)
+
+    def kv_indptr(self) -> list[int]:
+        return self._indptr(self.prefix_lens)
+
+    def mask_indptr(self) -> list[int]:
+        return self._indptr([n * n for n in self.draft_lens])
+
+    def pool_rows(self) -> int:
+        return max(1, int(sum(self.prefix_lens) * self.pool_slack))
+
+    def prefix_kv_bytes(self) -> int:
+        elem = torch.tensor([], dtype=self.dtype).element_size()
+        return sum(self.prefix_lens) * self.Hkv * self.d * 2 * elem
+
+    def make(self, device="cpu", seed: int | None = None):
+        """q, k_draft, v_draft [n_rows, H, d]; k_pool, v_pool [pool rows,
+        Hkv, d]; kv_indices int32 [sum prefix]; draft mask uint8 (flat, the
+        requests' Lb x Lb blocks in order) or None."""
+        g = torch.Generator(device="cpu")
+        g.manual_seed(self.seed if seed is None else seed)
+
+        def draw(shape):
+            x = torch.randn(shape, generator=g, dtype=torch.float32)
+            return (x * self.sigma).to(self.dtype).to(device)
+
+        NR = self.n_rows
+        q = draw((NR, self.Hq, self.d))
+        kd = draw((NR, self.Hkv, self.d))
+        vd = draw((NR, self.Hkv, self.d))
+        npool = self.pool_rows()
+        kp = draw((npool, self.Hkv, self.d))
+        vp = draw((npool, self.Hkv, self.d))
+        idx = torch.randperm(npool, generator=g)[:sum(self.prefix_lens)].to(torch.int32)
+        mask = None
+        if self.tree:
+            blocks = []
+            for n in self.draft_lens:
+                m = torch.zeros((n, n), dtype=torch.uint8)
+                parent = []
+                for j in range(n):
+                    # -1 is the prefix (a root draft); else an earlier draft
+                    parent.append(int(torch.randint(-1, j, (1,), generator=g)) if j else -1)
+                    a = j
+                    while a >= 0:
+                        m[j, a] = 1
+                        a = parent[a]
+                blocks.append(m.reshape(-1))
+            mask = torch.cat(blocks) if blocks else torch.zeros(0, dtype=torch.uint8)
+            mask = mask.to(device)
+        return q, kd, vd, kp, vp, idx.to(device), mask
+
+
+@dataclass
 class SparseLatentWorkload:
     name: str
     T: int
@@ -339,3 +440,7 @@ VERIFY_SHARED = SharedVerifyWorkload("verify-shared B=32 L=16384 drafts=4 H=32/8
                                      B=32, L=16384, Ld=4, Hq=32, Hkv=8, d=128, seed=6)
 SPARSE = SparseLatentWorkload("sparse T=16384 H=64 dl=512 topk=2048 bf16", T=16384, H=64,
                               dl=512, topk=2048, seed=5)
+VERIFY_PAGED = ExtendVerifyWorkload(
+    "verify-extend B=32 L=16384 drafts 1..8 trees, token-granular page table H=32/8 d=128 bf16",
+    draft_lens=[1 + (5 * b) % 8 for b in range(32)], prefix_lens=[16384] * 32, Hq=32, Hkv=8,
+    d=128, nsplit=32, seed=8)

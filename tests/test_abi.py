@@ -63,7 +63,7 @@ def test_verify_gating_refuses_unsupported_features(field, value):
 
 
 def test_verify_host_validation():
-    assert _verify_call(kvi=16) == psa.PSA_ERR_UNSUPPORTED          # paged cache
+    assert _verify_call(kvi=16) == psa.PSA_ERR_WORKSPACE            # paged: passes the gate
     assert _verify_call(d=96) == psa.PSA_ERR_UNSUPPORTED             # head dim
     assert _verify_call(Hq=6, Hkv=4) == psa.PSA_ERR_INVALID_ARG      # Hq % Hkv
     assert _verify_call(scale=0.0) == psa.PSA_ERR_INVALID_ARG
@@ -130,6 +130,32 @@ def test_verify_tree_needs_a_mask():
                                        P(16), P(16), None, 1, 4, 8, 2, 128, 0.1, 1,
                                        ctypes.byref(f), None, 0, None, None)
     assert rc == psa.PSA_ERR_WORKSPACE
+
+
+def _extend_call(**kw):
+    args = dict(qo=16, nrows=6, maxld=4, B=2, mask=None, mi=None, feat=None, ws=None, wsb=0)
+    args.update(kw)
+    a = args
+    P = ctypes.c_void_p
+    opt = lambda v: P(v) if v else None  # noqa: E731
+    return psa.lib().psa_verify_extend_fwd(
+        P(16), P(16), P(16), P(16), P(16), 64, opt(a["qo"]), a["nrows"], a["maxld"], P(16), 64,
+        None, opt(a["mask"]), opt(a["mi"]), P(16), None, a["B"], 8, 2, 128, 0.1, 1,
+        ctypes.byref(a["feat"]) if a["feat"] is not None else None, opt(a["ws"]), a["wsb"],
+        None, None)
+
+
+def test_verify_extend_host_validation():
+    """The extend entry takes ragged draft counts and tree masks (can_handle's
+    two refusals) and checks what the host can see."""
+    ragged_tree = psa.VerifyFeatures(1, 1, -1, 0, 0.0, -1, 1)
+    assert _extend_call(feat=ragged_tree, mask=16, mi=16) == psa.PSA_ERR_WORKSPACE
+    assert _extend_call(qo=None) == psa.PSA_ERR_INVALID_ARG          # qo_indptr required
+    assert _extend_call(mask=16) == psa.PSA_ERR_INVALID_ARG          # mask without mask_indptr
+    assert _extend_call(feat=ragged_tree) == psa.PSA_ERR_UNSUPPORTED  # custom mask flag, no mask
+    assert _extend_call(nrows=9) == psa.PSA_ERR_INVALID_ARG          # more rows than B * max
+    assert _extend_call(maxld=17) == psa.PSA_ERR_UNSUPPORTED         # m-tile plan: 17 * 4 > 128
+    assert _extend_call(nrows=0) == psa.PSA_OK                       # no draft rows
 
 
 def test_verify_fp8_host_validation():
