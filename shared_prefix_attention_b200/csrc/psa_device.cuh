@@ -134,17 +134,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Plain (untiled) bulk copy of `bytes` contiguous global bytes into shared
-// memory, completing on `bar`'s transaction count.  Both addresses and the
-// size must be multiples of 16 bytes.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a tile
 // written by TMA with 128-byte swizzling (rows of 128 B, 1024-B aligned
 // base): the chunk index is XORed with the row index mod 8.

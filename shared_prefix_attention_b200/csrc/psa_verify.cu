@@ -31,6 +31,17 @@ int launch_combine_d(const VerifyArgs& a);
 
 namespace {
 
+// Plain (untiled) bulk copy of `bytes` contiguous global bytes into shared
+// memory, completing on `bar`'s transaction count.  Both addresses and the
+// size must be multiples of 16 bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 constexpr int kTileKeys = 16;      // keys per pipeline stage
 // Consumer warps per CTA: with the producer warp, 9 warps leave each warp
 // 168 registers; head_dim 256 needs more, so it runs 4 consumer warps.
