@@ -44,7 +44,9 @@ constexpr int BR = 64;             // rows of a half-block (the schedule's recta
 constexpr int BLK = 2 * BR;        // rows (or keys) per schedule block = TMEM lanes
 constexpr int BT = 64;             // columns per streamed tile
 constexpr int kThreads = 384;      // 12 warps
-constexpr int kStages = 3;         // streamed tiles in flight
+// streamed tiles in flight: the tiles the MMAs still read (two TMEM
+// buffers' worth) plus one being prefetched
+constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
 
 enum { kDq = 0, kDkdv = 1 };
@@ -125,6 +127,7 @@ struct BwdParams {
 
 template <int D, int MODE>
 struct TcCfg {
+  static constexpr int NST = kStages;
   static constexpr int NPART = D / 64;              // 128-byte swizzle atoms across d
   static constexpr uint32_t BLOCK = BLK * D * 2;    // one block operand
   static constexpr uint32_t TILE = BT * D * 2;      // one tile operand
@@ -137,14 +140,19 @@ struct TcCfg {
   static constexpr uint32_t STAGE_TX = 2 * TILE + (MODE == kDkdv ? 2 * STAT : 0u);
   static constexpr uint32_t OFF_BLK = 0;
   static constexpr uint32_t OFF_RING = 2 * BLOCK;
-  static constexpr uint32_t OFF_BAR = OFF_RING + kStages * STAGE;
-  static constexpr int NBAR = 2 + 2 * kStages + 2 + 2 + 2;
+  static constexpr uint32_t OFF_BAR = OFF_RING + NST * STAGE;
+  static constexpr int NBAR = 2 + 2 * NST + 3 + 3 + 2;
   // at least 116 KB, so that one CTA (holding all 512 TMEM columns) fits per SM
   static constexpr uint32_t SMEM_USED = 1024 + OFF_BAR + NBAR * 8 + 16;
   static constexpr uint32_t SMEM = SMEM_USED > 116u * 1024 ? SMEM_USED : 116u * 1024;
   // TMEM columns: buffer b holds S at 128 b and dP at 128 b + 64 (P and dS
   // overwrite their first 32 columns as packed bf16); the accumulators follow.
-  static constexpr uint32_t T_ACC = 256;  // dkdv: dV then dK; dq: dQ
+  // Two buffers: the MMA issuer runs one tile ahead of the P / dS warps.
+  // (dq has TMEM room for a third; with a deeper ring to match it measured
+  // the same, the tensor pipe being the limit there.)
+  static constexpr int NBUF = 2;
+  static constexpr uint32_t T_ACC = NBUF * 128;  // dkdv: dV then dK; dq: dQ
+  static_assert(T_ACC + (MODE == kDq ? D : 2 * D) <= kTmemCols, "TMEM budget");
 };
 
 struct Bars {
@@ -200,20 +208,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.blk_full = bar;
   B.blk_empty = bar + 1;
   B.ring_full = bar + 2;
-  B.ring_empty = B.ring_full + kStages;
-  B.s_full = B.ring_empty + kStages;
-  B.p_full = B.s_full + 2;
-  B.acc_full = B.p_full + 2;
+  B.ring_empty = B.ring_full + C::NST;
+  B.s_full = B.ring_empty + C::NST;
+  B.p_full = B.s_full + C::NBUF;
+  B.acc_full = B.p_full + C::NBUF;
   B.acc_free = B.acc_full + 1;
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(B.blk_full, 1);
     mbar_init(B.blk_empty, 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < C::NST; ++i) {
       mbar_init(B.ring_full + i, 1);
       mbar_init(B.ring_empty + i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NBUF; ++i) {
       mbar_init(B.s_full + i, 1);
       mbar_init(B.p_full + i, 4);  // the four warps of a compute warpgroup
     }
@@ -260,8 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int j = MODE == kDq ? t : t % it.w;
           const int yh = MODE == kDq ? head / p.G : head * p.G + t / it.w;
           const int c0 = __ldg(tiles + 8 * (it.z + j));
-          const int s = n % kStages;
-          if (!mbar_wait(B.ring_empty + s, ((n / kStages) & 1) ^ 1, &abort_flag, p.status)) {
+          const int s = n % C::NST;
+          if (!mbar_wait(B.ring_empty + s, ((n / C::NST) & 1) ^ 1, &abort_flag, p.status)) {
             ok = false;
             break;
           }
@@ -294,56 +302,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_acc = umma_idesc_bf16(BLK, D, false, true);
       const uint32_t sX = smem_u32(smem + C::OFF_BLK);
       const uint32_t sR = smem_u32(smem + C::OFF_RING);
+      static_assert(C::OFF_RING + C::NST * C::STAGE < (1u << 18), "descriptor address field");
       uint32_t n = 0, ub = 0;
       bool ok = true;
-      // S = X1 Y1^T and dP = X2 Y2^T of global tile m into TMEM buffer m & 1
+      // Descriptors are built once; a k-step or stage moves only the start
+      // address field (bits 0..13, in 16-byte units), so it is a plain add.
+      const uint64_t dX = umma_desc_sw128(sX, 16, 1024);
+      const uint64_t dR = umma_desc_sw128(sR, 16, 1024);          // K-major tile rows
+      const uint64_t dRmn = umma_desc_sw128(sR, BT * 128, 1024);  // MN-major tile rows
+      // S = X1 Y1^T and dP = X2 Y2^T of global tile m into TMEM buffer m % NBUF
       auto issue_s = [&](uint32_t m) -> bool {
-        const int s = m % kStages;
-        if (!mbar_wait(B.ring_full + s, (m / kStages) & 1, &abort_flag, p.status)) return false;
+        const int s = m % C::NST;
+        if (!mbar_wait(B.ring_full + s, (m / C::NST) & 1, &abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t tb = tmem + (m & 1) * 128;
-        const uint32_t y = sR + s * C::STAGE;
+        const uint32_t tb = tmem + (m % C::NBUF) * 128;
+        const uint64_t dY = dR + ((s * C::STAGE) >> 4);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t ox = (ks >> 2) * (BLK * 128) + (ks & 3) * 32;
-          const uint32_t oy = (ks >> 2) * (BT * 128) + (ks & 3) * 32;
-          umma_ss(tb, umma_desc_sw128(sX + ox, 16, 1024), umma_desc_sw128(y + oy, 16, 1024),
-                  idesc_s, ks > 0 ? 1u : 0u);
+          const uint32_t ox = ((ks >> 2) * (BLK * 128) + (ks & 3) * 32) >> 4;
+          const uint32_t oy = ((ks >> 2) * (BT * 128) + (ks & 3) * 32) >> 4;
+          umma_ss(tb, dX + ox, dY + oy, idesc_s, ks > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t ox = C::BLOCK + (ks >> 2) * (BLK * 128) + (ks & 3) * 32;
-          const uint32_t oy = C::TILE + (ks >> 2) * (BT * 128) + (ks & 3) * 32;
-          umma_ss(tb + 64, umma_desc_sw128(sX + ox, 16, 1024), umma_desc_sw128(y + oy, 16, 1024),
-                  idesc_s, ks > 0 ? 1u : 0u);
+          const uint32_t ox = (C::BLOCK + (ks >> 2) * (BLK * 128) + (ks & 3) * 32) >> 4;
+          const uint32_t oy = (C::TILE + (ks >> 2) * (BT * 128) + (ks & 3) * 32) >> 4;
+          umma_ss(tb + 64, dX + ox, dY + oy, idesc_s, ks > 0 ? 1u : 0u);
         }
-        umma_commit(B.s_full + (m & 1));
+        umma_commit(B.s_full + (m % C::NBUF));
         return true;
       };
       // the accumulating products of global tile m (the unit's tile t)
       auto issue_acc = [&](uint32_t m, int t) -> bool {
-        if (!mbar_wait(B.p_full + (m & 1), (m >> 1) & 1, &abort_flag, p.status)) return false;
+        if (!mbar_wait(B.p_full + (m % C::NBUF), (m / C::NBUF) & 1, &abort_flag, p.status))
+          return false;
         if (t == 0 && !mbar_wait(B.acc_free, (ub & 1) ^ 1, &abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t tb = tmem + (m & 1) * 128;
-        const uint32_t y = sR + (m % kStages) * C::STAGE;
+        const uint32_t tb = tmem + (m % C::NBUF) * 128;
+        const uint64_t dY = dRmn + (((m % C::NST) * C::STAGE) >> 4);
         // B operands: the tile's rows are the contraction, D the N dimension
 #pragma unroll
         for (int ks = 0; ks < BT / 16; ++ks) {
           const uint32_t acc = (t > 0 || ks > 0) ? 1u : 0u;
           if constexpr (MODE == kDq) {
             // dQ += dS K_t
-            umma_ts(tmem + C::T_ACC, tb + 64 + ks * 8,
-                    umma_desc_sw128(y + ks * 2048, BT * 128, 1024), idesc_acc, acc);
+            umma_ts(tmem + C::T_ACC, tb + 64 + ks * 8, dY + ks * (2048 >> 4), idesc_acc, acc);
           } else {
             // dV += P^T dO_t, dK += dS^T Q_t
-            umma_ts(tmem + C::T_ACC, tb + ks * 8,
-                    umma_desc_sw128(y + C::TILE + ks * 2048, BT * 128, 1024), idesc_acc, acc);
-            umma_ts(tmem + C::T_ACC + D, tb + 64 + ks * 8,
-                    umma_desc_sw128(y + ks * 2048, BT * 128, 1024), idesc_acc, acc);
+            umma_ts(tmem + C::T_ACC, tb + ks * 8, dY + ((C::TILE + ks * 2048) >> 4), idesc_acc,
+                    acc);
+            umma_ts(tmem + C::T_ACC + D, tb + 64 + ks * 8, dY + ks * (2048 >> 4), idesc_acc, acc);
           }
         }
-        umma_commit(B.ring_empty + (m % kStages));
+        umma_commit(B.ring_empty + (m % C::NST));
         return true;
       };
       for (int r = 0; ok; ++r) {
@@ -354,12 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nt = unit_tiles<MODE>(p, items, u, it, head);
         if (nt == 0) continue;
         if (!mbar_wait(B.blk_full, ub & 1, &abort_flag, p.status)) break;
-        ok = issue_s(n);
-        for (int t = 1; t < nt && ok; ++t) {
-          ok = issue_s(n + t);                 // the tensor pipe runs S(t) while
-          if (ok) ok = issue_acc(n + t - 1, t - 1);  // tile t-1's P and dS are made
+        // S runs NBUF - 1 tiles ahead of the accumulating products: the
+        // tensor pipe works on later tiles while tile t's P and dS are made
+        constexpr int L = C::NBUF - 1;
+        for (int t = 0; t < L && t < nt && ok; ++t) ok = issue_s(n + t);
+        for (int t = 0; t < nt && ok; ++t) {
+          if (t + L < nt) ok = issue_s(n + t + L);
+          if (ok) ok = issue_acc(n + t, t);
         }
-        if (ok) ok = issue_acc(n + nt - 1, nt - 1);
         if (!ok) break;
         umma_commit(B.blk_empty);
         umma_commit(B.acc_full);
@@ -427,44 +440,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float* lse_col = nullptr;
         const float* dlt_col = nullptr;
         if constexpr (MODE == kDkdv) {
-          const uint8_t* st = smem + C::OFF_RING + (m % kStages) * C::STAGE + 2 * C::TILE;
+          const uint8_t* st = smem + C::OFF_RING + (m % C::NST) * C::STAGE + 2 * C::TILE;
           lse_col = reinterpret_cast<const float*>(st) + (c0 & 3);
           dlt_col = reinterpret_cast<const float*>(st + C::STAT_SLOT) + (c0 & 3);
         }
         // the tile's stats came with its TMA copies: observe that phase
         // directly before reading them (dkdv), then wait for S and dP
-        if (MODE == kDkdv && !mbar_wait(B.ring_full + (m % kStages), (m / kStages) & 1,
+        if (MODE == kDkdv && !mbar_wait(B.ring_full + (m % C::NST), (m / C::NST) & 1,
                                         &abort_flag, p.status)) {
           ok = false;
           break;
         }
-        if (!mbar_wait(B.s_full + wg, (m >> 1) & 1, &abort_flag, p.status)) {
+        const int buf = m % C::NBUF;
+        if (!mbar_wait(B.s_full + buf, (m / C::NBUF) & 1, &abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t tS = tlane + wg * 128, tP = tS + 64;
+        const uint32_t tS = tlane + buf * 128, tP = tS + 64;
+        // every column visible (the common case): no per-element mask
+        const bool all_vis = vis == ~0ull;
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), zero2 = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t s[32], dp[32];
           tmem_ld32(tS + ch * 32, s);
           tmem_ld32(tP + ch * 32, dp);
           tmem_wait_ld();
+          const uint32_t vm = uint32_t(vis >> (32 * ch));
           uint32_t pk[16], dk[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            float pr[2], ds[2];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int col = ch * 32 + i + h2;
-              const float l = MODE == kDq ? lse_row : lse_col[col];
-              const float dl = MODE == kDq ? dlt_row : dlt_col[col];
-              const bool v = (vis >> col) & 1ull;
-              pr[h2] = v ? fast_exp2(__uint_as_float(s[i + h2]) * p.scale_log2 - l) : 0.f;
-              ds[h2] = pr[h2] * (__uint_as_float(dp[i + h2]) - dl);
+            const int col = ch * 32 + i;
+            float l0, l1, d0, d1;
+            if constexpr (MODE == kDq) {
+              l0 = l1 = lse_row;
+              d0 = d1 = dlt_row;
+            } else {
+              l0 = lse_col[col];
+              l1 = lse_col[col + 1];
+              d0 = dlt_col[col];
+              d1 = dlt_col[col + 1];
             }
-            pk[i / 2] = pack_bf16(pr[0], pr[1]);
-            dk[i / 2] = pack_bf16(ds[0], ds[1]);
+            // x = scale_log2 s - lse, P = 2^x, dS = P (dP - D), two columns at a time
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])),
+                                       sc2, f2_pack(-l0, -l1));
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            if (!all_vis) {
+              p0 = (vm >> i) & 1u ? p0 : 0.f;
+              p1 = (vm >> (i + 1)) & 1u ? p1 : 0.f;
+            }
+            const uint64_t g2 = f2_add(f2_pack(__uint_as_float(dp[i]), __uint_as_float(dp[i + 1])),
+                                       f2_pack(-d0, -d1));
+            float ds0, ds1;
+            f2_unpack(f2_fma(f2_pack(p0, p1), g2, zero2), ds0, ds1);
+            pk[i / 2] = pack_bf16(p0, p1);
+            dk[i / 2] = pack_bf16(ds0, ds1);
           }
           if constexpr (MODE == kDkdv) tmem_st16(tS + ch * 16, pk);
           tmem_st16(tP + ch * 16, dk);
@@ -472,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(B.p_full + wg);
+        if (lane == 0) mbar_arrive(B.p_full + buf);
       }
       if (!ok) break;
       // epilogue: this warpgroup's accumulator columns of the unit
