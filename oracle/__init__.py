@@ -72,13 +72,15 @@ def load(path: str | None = None):
     lib.oracle_verify_shared.argtypes = [P, P, P, P, P, ctypes.c_int64, I, I, I, I, I, D, P, I,
                                          P, P, I]
     lib.oracle_verify_fp8.argtypes = [P, P, P, P, P, D, D, P, I, I, I, I, I, D, P, I, P, P, I]
+    lib.oracle_verify_fp8_paged.argtypes = [P, P, P, P, P, D, D, P, P, I, I, I, I, I, D, P, I,
+                                            P, P, I]
     lib.oracle_decode_e4m3.argtypes = [P, P, ctypes.c_int64]
     lib.oracle_sparse_latent.argtypes = [P, P, P, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_visibility.argtypes = [P, P, P, I, I, I, I, P]
     for f in (lib.oracle_prefill, lib.oracle_prefill_bwd, lib.oracle_prefill_bwd_dq,
               lib.oracle_verify, lib.oracle_verify_tree, lib.oracle_verify_extend,
               lib.oracle_verify_shared,
-              lib.oracle_verify_fp8, lib.oracle_decode_e4m3, lib.oracle_sparse_latent,
+              lib.oracle_verify_fp8, lib.oracle_verify_fp8_paged, lib.oracle_decode_e4m3, lib.oracle_sparse_latent,
               lib.oracle_visibility):
         f.restype = I
     if path == _LIB_PATH:
@@ -310,9 +312,10 @@ def decode_e4m3(codes, lib=None):
 
 def verify_fp8(q_draft, k_draft, v_draft, k_cache8, v_cache8, k_scale: float, v_scale: float,
                kv_indptr, Ld: int, scale: float, rows=None, nthreads: int | None = None,
-               lib=None):
+               lib=None, kv_indices=None):
     """As verify, with e4m3 caches (uint8 or float8 tensors) standing for
-    k_scale * e4m3 and v_scale * e4m3."""
+    k_scale * e4m3 and v_scale * e4m3; with kv_indices, prefix position t of
+    the flat kv_indptr range is cache row kv_indices[t]."""
     lib = lib or load()
     qd, kd, vd = _f32(q_draft), _f32(k_draft), _f32(v_draft)
     kc, vc = _u8(k_cache8), _u8(v_cache8)
@@ -324,10 +327,17 @@ def verify_fp8(q_draft, k_draft, v_draft, k_cache8, v_cache8, k_scale: float, v_
     rows = np.arange(BL, dtype=np.int32) if rows is None else _i32(rows)
     o = np.zeros((len(rows), Hq, d), dtype=np.float64)
     lse = np.zeros((len(rows), Hq), dtype=np.float64)
-    rc = lib.oracle_verify_fp8(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kc), _ptr(vc), float(k_scale),
-                               float(v_scale), _ptr(indptr), B, Ld, Hq, Hkv, d, float(scale),
-                               _ptr(rows), len(rows), _ptr(o), _ptr(lse),
-                               nthreads or default_threads())
+    if kv_indices is None:
+        rc = lib.oracle_verify_fp8(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kc), _ptr(vc),
+                                   float(k_scale), float(v_scale), _ptr(indptr), B, Ld, Hq, Hkv,
+                                   d, float(scale), _ptr(rows), len(rows), _ptr(o), _ptr(lse),
+                                   nthreads or default_threads())
+    else:
+        idx = _i32(kv_indices)
+        rc = lib.oracle_verify_fp8_paged(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kc), _ptr(vc),
+                                         float(k_scale), float(v_scale), _ptr(indptr), _ptr(idx),
+                                         B, Ld, Hq, Hkv, d, float(scale), _ptr(rows), len(rows),
+                                         _ptr(o), _ptr(lse), nthreads or default_threads())
     assert rc == 0, "oracle_verify_fp8 rejected its arguments"
     return o, lse
 

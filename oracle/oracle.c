@@ -638,6 +638,7 @@ typedef struct {
     double scale, kscale, vscale;
     const int32_t *rows;
     double *o, *lse;
+    const int32_t *kv_indices; /* NULL, or prefix position t is cache row kv_indices[t] */
 } verify8_ctx;
 
 static void verify8_row(void *p, int r, double *z, const float **vr, double *o) {
@@ -651,7 +652,12 @@ static void verify8_row(void *p, int r, double *z, const float **vr, double *o) 
         const float *qrow = c->qd + ((size_t)row * c->Hq + h) * c->d;
         int n = 0;
         for (int64_t t = p0; t < p1; ++t) { /* the whole cached prefix, scaled keys */
-            const uint8_t *krow = c->kc + ((size_t)t * c->Hkv + kvh) * c->d;
+#if ORACLE_MUTANT == 7
+            int64_t slot = t;  /* planted: the page table is ignored */
+#else
+            int64_t slot = c->kv_indices ? c->kv_indices[t] : t;
+#endif
+            const uint8_t *krow = c->kc + ((size_t)slot * c->Hkv + kvh) * c->d;
             double sdot = 0.0;
             for (int e = 0; e < c->d; ++e) sdot += (double)qrow[e] * decode_e4m3(krow[e]);
             z[n++] = apply_scale(c->kscale * sdot, c->scale);
@@ -667,7 +673,8 @@ static void verify8_row(void *p, int r, double *z, const float **vr, double *o) 
         n = 0;
         for (int64_t t = p0; t < p1; ++t) {
             double w = exp(z[n++] - m) / l;
-            const uint8_t *vrow = c->vc + ((size_t)t * c->Hkv + kvh) * c->d;
+            int64_t slot = c->kv_indices ? c->kv_indices[t] : t;
+            const uint8_t *vrow = c->vc + ((size_t)slot * c->Hkv + kvh) * c->d;
             for (int e = 0; e < c->d; ++e) o[e] += w * c->vscale * decode_e4m3(vrow[e]);
         }
         for (int i = 0; i <= j; ++i) {
@@ -692,7 +699,26 @@ int oracle_verify_fp8(const float *qd, const float *kd, const float *vd,
     for (int b = 0; b < B; ++b)
         if (indptr[b + 1] - indptr[b] > maxlen) maxlen = indptr[b + 1] - indptr[b];
     verify8_ctx c = {qd, kd, vd, kc, vc, indptr, Ld, Hq, Hkv, d, scale, kscale, vscale,
-                     rows, o, lse};
+                     rows, o, lse, NULL};
+    run_rows(verify8_row, &c, nrows, (int)maxlen + Ld, d, nthreads);
+    return 0;
+}
+
+/* As oracle_verify_fp8 with the prefix read through a page table of one
+ * token per page ("Split-KV flash-decode attention for EAGLE target-verify",
+ * the verify entry's kv_indptr / kv_indices): prefix position t of the flat
+ * indptr range is cache row kv_indices[t]. */
+int oracle_verify_fp8_paged(const float *qd, const float *kd, const float *vd,
+                            const uint8_t *kc, const uint8_t *vc, double kscale, double vscale,
+                            const int64_t *indptr, const int32_t *kv_indices, int B, int Ld,
+                            int Hq, int Hkv, int d, double scale, const int32_t *rows,
+                            int nrows, double *o, double *lse, int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || B < 0 || Ld <= 0 || !kv_indices) return -1;
+    int64_t maxlen = 0;
+    for (int b = 0; b < B; ++b)
+        if (indptr[b + 1] - indptr[b] > maxlen) maxlen = indptr[b + 1] - indptr[b];
+    verify8_ctx c = {qd, kd, vd, kc, vc, indptr, Ld, Hq, Hkv, d, scale, kscale, vscale,
+                     rows, o, lse, kv_indices};
     run_rows(verify8_row, &c, nrows, (int)maxlen + Ld, d, nthreads);
     return 0;
 }

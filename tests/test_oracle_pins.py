@@ -462,6 +462,21 @@ def pin_verify_fp8_cache(lib):
             o2, lse2 = oracle.verify(q, kd, vd, kr.float(), vr.float(), indptr, Ld, scale,
                                      lib=lib)
             ok &= np.allclose(o, o2, atol=1e-12) and np.allclose(lse, lse2, atol=1e-12)
+    # through a page table: the cache rows scattered over a larger pool
+    # (numpy fancy indexing), the same result as the contiguous cache
+    ntok = kc.shape[0]
+    rng = np.random.default_rng(72)
+    table = rng.permutation(2 * ntok)[:ntok].astype(np.int32)
+    kc8 = (kc / 0.37).to(torch.float8_e4m3fn).view(torch.uint8)
+    vc8 = (vc / 1.9).to(torch.float8_e4m3fn).view(torch.uint8)
+    kpool = torch.zeros((2 * ntok,) + tuple(kc8.shape[1:]), dtype=torch.uint8)
+    vpool = torch.zeros_like(kpool)
+    kpool[torch.from_numpy(table.astype(np.int64))] = kc8
+    vpool[torch.from_numpy(table.astype(np.int64))] = vc8
+    o1, l1 = oracle.verify_fp8(q, kd, vd, kc8, vc8, 0.37, 1.9, indptr, Ld, scale, lib=lib)
+    o2, l2 = oracle.verify_fp8(q, kd, vd, kpool, vpool, 0.37, 1.9, indptr, Ld, scale, lib=lib,
+                               kv_indices=table)
+    ok &= np.array_equal(o1, o2) and np.array_equal(l1, l2)
     return bool(ok)
 
 
