@@ -369,10 +369,11 @@ int psa_verify_fwd_noalloc(const void *q_draft, const void *k_draft, const void 
  *                    k_scale * e4m3, a cached value for v_scale * e4m3
  *   k_scale, v_scale host values, finite and > 0
  * Draft keys and values stay bf16 and are not scaled.  Every other argument,
- * layout and status is that of psa_verify_fwd, except that head_dim must be
- * 128 (PSA_ERR_UNSUPPORTED otherwise).  The prefix read is half the bytes of
- * the bf16 cache.  Q is widened to f16 for the tensor cores: |q| must stay
- * below 65504.
+ * layout and status is that of psa_verify_fwd (kv_indices included: NULL for
+ * a contiguous prefix, else the token-granular page table), except that
+ * head_dim must be 128 (PSA_ERR_UNSUPPORTED otherwise).  The prefix read is
+ * half the bytes of the bf16 cache.  Q is widened to f16 for the tensor
+ * cores: |q| must stay below 65504.
  */
 int psa_verify_fp8_fwd(const void *q_draft, const void *k_draft, const void *v_draft,
                        const void *k_cache, const void *v_cache, int64_t n_cache_tokens,

@@ -345,9 +345,11 @@ def verify_shared(q_draft, k_draft, v_draft, k_prefix, v_prefix, scale: float, L
 
 def verify_fp8(q_draft, k_draft, v_draft, k_cache8, v_cache8, k_scale: float, v_scale: float,
                kv_indptr: torch.Tensor, max_prefix_len: int, scale: float, Ld: int,
-               nsplit: int = 0, out=None, lse=None, workspace=None, status=None):
+               nsplit: int = 0, out=None, lse=None, workspace=None, status=None,
+               kv_indices=None):
     """Split-KV verify over an e4m3 prefix cache (uint8 or float8_e4m3fn
-    tensors [Ntok, Hkv, d]) standing for k_scale * e4m3 and v_scale * e4m3."""
+    tensors [Ntok, Hkv, d]) standing for k_scale * e4m3 and v_scale * e4m3;
+    kv_indices: optional token-granular page table (device int32)."""
     _require_cuda(q_draft, k_draft, v_draft, k_cache8, v_cache8, kv_indptr)
     BL, Hq, d = q_draft.shape
     Hkv = k_draft.shape[1]
@@ -360,7 +362,8 @@ def verify_fp8(q_draft, k_draft, v_draft, k_cache8, v_cache8, k_scale: float, v_
                                 dtype=torch.uint8, device=q_draft.device)
     rc = lib().psa_verify_fp8_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft), _ptr(k_cache8),
                                   _ptr(v_cache8), k_cache8.shape[0], _ptr(kv_indptr),
-                                  int(max_prefix_len), None, float(k_scale), float(v_scale),
+                                  int(max_prefix_len), _ptr(kv_indices), float(k_scale),
+                                  float(v_scale),
                                   _ptr(out), _ptr(lse), B, Ld, Hq, Hkv, d, float(scale), ns, None,
                                   _ptr(workspace), workspace.numel(), _ptr(status),
                                   _stream(q_draft.device))

@@ -270,7 +270,6 @@ extern "C" int psa_verify_fp8_fwd(const void* q_draft, const void* k_draft, cons
         features->xai_temperature_len > 0 || features->ragged_extend)
       return PSA_ERR_UNSUPPORTED;
   }
-  if (kv_indices) return PSA_ERR_UNSUPPORTED;
   if (B < 0 || Ld <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n_cache_tokens < 0 ||
       max_prefix_len < 0 || n_cache_tokens > INT32_MAX || !(scale > 0.f) ||
       !(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
@@ -290,7 +289,6 @@ extern "C" int psa_verify_fp8_fwd(const void* q_draft, const void* k_draft, cons
   const size_t need = psa_verify_workspace_size(B, Ld, Hq, head_dim, nsplit);
   if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return PSA_ERR_WORKSPACE;
-  if (n_cache_tokens == 0) n_cache_tokens = 1;  // a tensor map needs a non-empty extent
 
   VerifyArgs a;
   a.q = q_draft;
@@ -315,6 +313,7 @@ extern "C" int psa_verify_fp8_fwd(const void* q_draft, const void* k_draft, cons
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + o_bytes);
   a.status = dev_status;
   a.stream = static_cast<cudaStream_t>(stream);
+  a.kv_indices = kv_indices;
   return launch_verify_fp8(a, k_scale, v_scale);
 }
 

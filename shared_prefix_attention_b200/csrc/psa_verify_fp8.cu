@@ -40,6 +40,12 @@ constexpr uint32_t kPrivBytes = 2 * kKeys * 128;  // f16 V tile, two d-parts
 struct P8Params {
   const __nv_bfloat16* q;  // [B*Ld, Hq, D]
   const int32_t* indptr;   // [B+1]
+  // Page table (paged instantiation only): prefix position t is cache row
+  // kv_indices[t], gathered with one bulk copy per key.
+  const int32_t* kv_indices;
+  const uint8_t* kc8;      // [ntok, Hkv, 128] e4m3
+  const uint8_t* vc8;
+  int64_t ntok;
   float* part_o;
   float* part_lse;
   int32_t B, Ld, Hq, Hkv, G, R;
@@ -67,7 +73,9 @@ __device__ __forceinline__ Unit8 decode_unit8(const P8Params& p, int u) {
 __device__ __forceinline__ void split_range8(const P8Params& p, int b, int s, int32_t& t0,
                                              int32_t& t1) {
   const int32_t a = __ldg(p.indptr + b), e = __ldg(p.indptr + b + 1);
-  const int32_t L = e - a;
+  int32_t L = e - a;
+  // a paged prefix must lie inside the page table, whose length is indptr[B]
+  if (L < 0 || a < 0 || (p.kv_indices && e > __ldg(p.indptr + p.B))) L = 0;
   int32_t c = (L + p.nsplit - 1) / p.nsplit;
   c = (c + kKeys - 1) / kKeys * kKeys;
   t0 = a + min(L, s * c);
@@ -103,15 +111,29 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// One lane widens 64 e4m3 values (half a key row) of a swizzled e4m3 tile into
-// the f16 tile: key row `key`, d half `half` (d = 64 half .. 64 half + 63 is
-// the f16 tile's d-part `half`).
+// Paged prefix: producer warps of the gathered layout (each fills
+// kKeys / kPagedProducers8 keys, K and V, one bulk copy per key and tensor)
+// and the byte address of 16-byte chunk `chunk` of key `key` in a K or V
+// tile: 128-byte swizzled TMA tile [head][key][128], or rows of HB heads
+// padded by 16 bytes (row stride rs) so an 8-key access hits 8 bank groups.
+constexpr int kPagedProducers8 = 4;
+
+template <bool PAGED>
+__device__ __forceinline__ uint32_t tile_at(uint32_t base, uint32_t key, uint32_t chunk,
+                                            uint32_t rs) {
+  return PAGED ? base + key * rs + chunk * 16 : base + sw128(key, chunk);
+}
+
+// One lane widens 64 e4m3 values (half a key row) of an e4m3 tile into the
+// f16 tile: key row `key`, d half `half` (d = 64 half .. 64 half + 63 is the
+// f16 tile's d-part `half`).
+template <bool PAGED>
 __device__ __forceinline__ void widen_row(uint32_t src_tile, uint32_t dst_tile, int key,
-                                          int half) {
+                                          int half, uint32_t rs) {
   uint32_t w[16];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t addr = src_tile + sw128(key, half * 4 + i);
+    const uint32_t addr = tile_at<PAGED>(src_tile, key, half * 4 + i, rs);
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(w[4 * i]), "=r"(w[4 * i + 1]), "=r"(w[4 * i + 2]), "=r"(w[4 * i + 3])
                  : "r"(addr));
@@ -129,7 +151,18 @@ __device__ __forceinline__ void widen_row(uint32_t src_tile, uint32_t dst_tile, 
   }
 }
 
-__global__ void __launch_bounds__((kMaxWarps + 1) * 32, 1)
+// Plain (untiled) bulk copy of `bytes` contiguous global bytes into shared
+// memory, completing on `bar`'s transaction count (16-byte multiples).
+__device__ __forceinline__ void bulk_load8(void* dst, const void* src, uint32_t bytes,
+                                           uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <bool PAGED>
+__global__ void __launch_bounds__((kMaxWarps + (PAGED ? kPagedProducers8 : 1)) * 32, 1)
     verify_stage1_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k,
                              const __grid_constant__ CUtensorMap tmap_v, P8Params p) {
   constexpr int KSTEPS = D8 / 16;
@@ -139,7 +172,9 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32, 1)
   __shared__ int abort_flag;
 
   const int NW = p.HB * p.MT;
-  const uint32_t kv_bytes = uint32_t(p.HB) * kHeadTile8;  // K (or V) per stage
+  // K (or V) bytes per stage, and the paged layout's row stride
+  const uint32_t rs = PAGED ? uint32_t(p.HB) * D8 + 16 : 0u;
+  const uint32_t kv_bytes = PAGED ? kKeys * rs : uint32_t(p.HB) * kHeadTile8;
   const uint32_t stage_bytes = 2 * kv_bytes;
   uint8_t* priv = smem + p.nstage * stage_bytes;           // kPrivBytes per consumer warp
   uint64_t* full = reinterpret_cast<uint64_t*>(priv + NW * kPrivBytes);
@@ -149,7 +184,8 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int i = 0; i < p.nstage; ++i) {
-      mbar_init(&full[i], 1);
+      // one arrival with the byte count per producer warp
+      mbar_init(&full[i], PAGED ? kPagedProducers8 : 1);
       mbar_init(&empty[i], NW);
     }
     fence_barrier_init();
@@ -158,9 +194,91 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32, 1)
 
   const int units = p.B * p.nsplit * p.nrb * p.nhb;
 
-  if (warp == NW) {
+  if (warp >= NW) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if constexpr (PAGED) {
+      // producer warp pw fills keys [pw*TPW, (pw+1)*TPW) of each tile: lane
+      // l < TPW copies key l's K row, lane TPW + l its V row (HB heads); a key
+      // past the split end, or a cache row outside [0, ntok) (reported), is
+      // written as zeros.  Table entries are read eight tiles ahead.
+      constexpr int TPW = kKeys / kPagedProducers8;
+      const int pw = warp - NW;
+      const bool active = lane < 2 * TPW;
+      const int tok = pw * TPW + lane % TPW;
+      const bool is_v = (lane / TPW) & 1;
+      const uint32_t row_bytes = uint32_t(p.HB) * D8;
+      const uint8_t* cache = is_v ? p.vc8 : p.kc8;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int last_phase[16];
+      for (int i = 0; i < 16; ++i) last_phase[i] = -1;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const Unit8 x = decode_unit8(p, u);
+        int32_t t0, t1;
+        split_range8(p, x.b, x.s, t0, t1);
+        constexpr int kPrefetch = 8;
+        int32_t cur[kPrefetch], nxt[kPrefetch];
+        auto lookup = [&](int32_t tb, int32_t (&dst)[kPrefetch]) {
+#pragma unroll
+          for (int k = 0; k < kPrefetch; ++k) {
+            const int32_t pos = tb + k * kKeys + tok;
+            dst[k] = pos < t1 ? __ldg(p.kv_indices + pos) : -1;
+          }
+        };
+        lookup(t0, cur);
+        for (int32_t tb = t0; tb < t1 && ok; tb += kPrefetch * kKeys) {
+          if (tb + kPrefetch * kKeys < t1) lookup(tb + kPrefetch * kKeys, nxt);
+#pragma unroll
+          for (int k = 0; k < kPrefetch; ++k) {
+            if (tb + k * kKeys >= t1) break;
+            // every lane acquires the released stage before writing into it
+            const bool w = mbar_wait(&empty[stage], phase ^ 1, &abort_flag, p.status);
+            if (!__all_sync(0xffffffffu, w)) {
+              ok = false;
+              break;
+            }
+            last_phase[stage] = int(phase);
+            int32_t slot = cur[k];
+            if (slot >= p.ntok || (slot < 0 && tb + k * kKeys + tok < t1)) {
+              report_status(p.status, PSA_ERR_INVALID_ARG);
+              slot = -1;
+            }
+            uint8_t* dst = smem + stage * stage_bytes + (is_v ? kv_bytes : 0u) + tok * rs;
+            if (active && slot < 0) {
+              const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+              for (uint32_t o = 0; o < row_bytes; o += 16)
+                *reinterpret_cast<uint4*>(dst + o) = z;
+              fence_proxy_async_smem();  // later bulk copies land after these stores
+            }
+            // one arrival per warp announces the bytes of all its copies,
+            // before any of them is issued
+            const uint32_t copies = __popc(__ballot_sync(0xffffffffu, active && slot >= 0));
+            if (lane == 0) mbar_arrive_expect_tx(&full[stage], copies * row_bytes);
+            __syncwarp();
+            if (active && slot >= 0)
+              bulk_load8(dst, cache + (size_t(slot) * p.Hkv + x.hb * p.HB) * D8, row_bytes,
+                         &full[stage]);
+            if (++stage == p.nstage) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kPrefetch; ++k) cur[k] = nxt[k];
+        }
+      }
+      if (!ok && lane == 0 && pw == 0) {
+        // Let copies already in flight land before the CTA exits.
+        for (int i = 0; i < p.nstage; ++i) {
+          if (last_phase[i] < 0) continue;
+          const uint64_t w0 = globaltimer();
+          while (!mbar_try_wait(&full[i], uint32_t(last_phase[i])) &&
+                 globaltimer() - w0 < kWaitTimeoutNs) {
+          }
+        }
+      }
+    } else if (lane == 0) {
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_v);
       int stage = 0;
@@ -257,10 +375,11 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32, 1)
         ok = false;
         break;
       }
-      const uint32_t k8 = smem_u32(smem + stage * stage_bytes) + hh * kHeadTile8;
+      const uint32_t k8 =
+          smem_u32(smem + stage * stage_bytes) + hh * (PAGED ? uint32_t(D8) : kHeadTile8);
       // widen this head's V tile into the warp's private f16 tile (the PV
       // operand needs it transposed, which ldmatrix.trans does on 16-bit data)
-      widen_row(k8 + kv_bytes, vpriv, lane >> 1, lane & 1);
+      widen_row<PAGED>(k8 + kv_bytes, vpriv, lane >> 1, lane & 1, rs);
 
       // S = Q K^T over 16 keys: two n-tiles of 8 keys; the B fragments come
       // straight from the e4m3 tile: key g, d = 16 ks + 2c (+1) and + 8 (+9)
@@ -271,7 +390,7 @@ __global__ void __launch_bounds__((kMaxWarps + 1) * 32, 1)
         const uint32_t key = nt * 8 + g;
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
-          const uint32_t addr = k8 + sw128(key, ks) + 2 * c;
+          const uint32_t addr = tile_at<PAGED>(k8, key, ks, rs) + 2 * c;
           uint32_t x0, x1;
           asm volatile("ld.shared.u16 %0, [%1];" : "=r"(x0) : "r"(addr));
           asm volatile("ld.shared.u16 %0, [%1];" : "=r"(x1) : "r"(addr + 8));
@@ -380,7 +499,9 @@ int launch_verify_fp8(const VerifyArgs& a, float k_scale, float v_scale) {
   const int G = a.Hq / a.Hkv;
 
   CUtensorMap tk, tv;
-  const uint64_t dims[3] = {uint64_t(D8), uint64_t(a.n_cache_tokens), uint64_t(a.Hkv)};
+  // a tensor map needs a non-empty extent (an empty cache is never read)
+  const uint64_t rows = a.n_cache_tokens > 0 ? uint64_t(a.n_cache_tokens) : 1u;
+  const uint64_t dims[3] = {uint64_t(D8), rows, uint64_t(a.Hkv)};
   const uint64_t strides[2] = {uint64_t(a.Hkv) * D8, uint64_t(D8)};
   const uint32_t box[3] = {uint32_t(D8), uint32_t(kKeys), uint32_t(HB)};
   int rc = encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.kc, dims, strides, box,
@@ -393,6 +514,10 @@ int launch_verify_fp8(const VerifyArgs& a, float k_scale, float v_scale) {
   P8Params p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.indptr = a.indptr;
+  p.kv_indices = a.kv_indices;
+  p.kc8 = static_cast<const uint8_t*>(a.kc);
+  p.vc8 = static_cast<const uint8_t*>(a.vc);
+  p.ntok = a.n_cache_tokens;
   p.part_o = a.part_o;
   p.part_lse = a.part_lse;
   p.B = a.B;
@@ -411,7 +536,9 @@ int launch_verify_fp8(const VerifyArgs& a, float k_scale, float v_scale) {
   p.status = a.status;
 
   const int NW = HB * MT;
-  const size_t stage_bytes = size_t(2) * HB * kHeadTile8;
+  const bool paged = a.kv_indices != nullptr;
+  const size_t stage_bytes =
+      size_t(2) * (paged ? size_t(kKeys) * (size_t(HB) * D8 + 16) : size_t(HB) * kHeadTile8);
   const size_t priv_bytes = size_t(NW) * kPrivBytes;
   const size_t budget = 200 * 1024;
   int nstage = int((budget - priv_bytes) / stage_bytes);
@@ -419,7 +546,7 @@ int launch_verify_fp8(const VerifyArgs& a, float k_scale, float v_scale) {
   if (nstage < 2) return PSA_ERR_UNSUPPORTED;
   p.nstage = nstage;
   const size_t smem = 1024 + nstage * stage_bytes + priv_bytes + 2 * nstage * sizeof(uint64_t);
-  auto k1 = verify_stage1_fp8_kernel;
+  auto k1 = paged ? verify_stage1_fp8_kernel<true> : verify_stage1_fp8_kernel<false>;
   if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
     return PSA_ERR_CUDA;
@@ -428,7 +555,7 @@ int launch_verify_fp8(const VerifyArgs& a, float k_scale, float v_scale) {
   if (grid <= 0) return PSA_ERR_CUDA;
   grid = units < grid ? units : grid;
   if (units > 0) {
-    k1<<<grid, (NW + 1) * 32, smem, a.stream>>>(tk, tv, p);
+    k1<<<grid, (NW + (paged ? kPagedProducers8 : 1)) * 32, smem, a.stream>>>(tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return PSA_ERR_CUDA;
   }
   return launch_verify_combine(a);

@@ -166,7 +166,7 @@ def test_verify_fp8_host_validation():
                                             P(kvi) if kvi else None, ks, vs, P(16), None, B, 4,
                                             8, 2, d, 0.1, 1, None, None, 0, None, None)
     assert call(d=64) == psa.PSA_ERR_UNSUPPORTED       # e4m3 path is head_dim 128 only
-    assert call(kvi=16) == psa.PSA_ERR_UNSUPPORTED     # paged cache
+    assert call(kvi=16) == psa.PSA_ERR_WORKSPACE       # paged cache: passes the gate
     assert call(ks=0.0) == psa.PSA_ERR_INVALID_ARG
     assert call(vs=float("inf")) == psa.PSA_ERR_INVALID_ARG
     assert call() == psa.PSA_ERR_WORKSPACE

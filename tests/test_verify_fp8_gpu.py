@@ -85,3 +85,37 @@ def test_verify_fp8_matches_bf16_path_on_decoded_cache():
     torch.cuda.synchronize()
     assert (o8.float() - o2.float()).abs().max().item() <= 1e-2
     assert (l8 - l2).abs().max().item() <= 1e-3
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,Ld,nsplit", [
+    ([300, 37, 1000], 32, 8, 4, 4),      # ragged prefixes, tail tiles, GQA 4:1
+    ([0, 700, 16], 16, 2, 8, 3),         # an empty prefix; 8 drafts
+    ([2048, 129], 32, 1, 4, 32),         # MQA: several row blocks
+])
+def test_verify_fp8_paged(lens, Hq, Hkv, Ld, nsplit):
+    """The e4m3 prefix read through a token-granular page table ([SKV] the
+    verify entry's kv_indices with its fp8 scales): against the oracle on
+    the same pool and table, and byte-identical to the contiguous cache."""
+    wl = _wl(B=len(lens), lens=lens, Hq=Hq, Hkv=Hkv, Ld=Ld, nsplit=nsplit, seed=75)
+    q, kd, vd, kc8, vc8 = (t.cuda() for t in wl.make_fp8("cpu"))
+    ntok = kc8.shape[0]
+    gen = torch.Generator().manual_seed(11)
+    table = torch.randperm(2 * ntok + 3, generator=gen)[:ntok].to(torch.int32)
+    kp = torch.zeros((2 * ntok + 3,) + tuple(kc8.shape[1:]), dtype=torch.uint8)
+    vp = torch.zeros_like(kp)
+    kp[table.long()] = kc8.cpu()
+    vp[table.long()] = vc8.cpu()
+    indptr = torch.tensor(wl.kv_indptr(), dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = psa.verify_fp8(q, kd, vd, kp.cuda(), vp.cuda(), wl.k_scale, wl.v_scale, indptr,
+                            max(lens), wl.scale, wl.Ld, nsplit=nsplit, status=status,
+                            kv_indices=table.cuda())
+    o2, l2 = psa.verify_fp8(q, kd, vd, kc8, vc8, wl.k_scale, wl.v_scale, indptr, max(lens),
+                            wl.scale, wl.Ld, nsplit=nsplit)
+    torch.cuda.synchronize()
+    assert psa.read_status(status) == 0
+    assert torch.equal(o, o2) and torch.equal(lse, l2)
+    ro, rl = oracle.verify_fp8(q.cpu(), kd.cpu(), vd.cpu(), kp, vp, wl.k_scale, wl.v_scale,
+                               np.array(wl.kv_indptr(), dtype=np.int64), wl.Ld, wl.scale,
+                               kv_indices=table)
+    assert_parity(o, lse, ro, rl, f"paged lens={lens}")
