@@ -467,6 +467,9 @@ class ExtendVerifyRunner(Runner):
 
 VERIFY_SMALL = W.VerifyWorkload("verify B=8 L=16384 drafts=4 H=32/8 d=128 splits=32 bf16", B=8,
                                 L=16384, Ld=4, Hq=32, Hkv=8, d=128, nsplit=32, seed=4)
+VERIFY_FP8_SMALL = W.VerifyWorkload(
+    "verify-fp8 B=8 L=16384 drafts=4 H=32/8 d=128 splits=32 e4m3 cache", B=8, L=16384, Ld=4,
+    Hq=32, Hkv=8, d=128, nsplit=32, seed=7)
 VERIFY_PAGED_SMALL = W.ExtendVerifyWorkload(
     "verify-extend B=8 L=16384 drafts 1..8 trees, token-granular page table H=32/8 d=128 bf16",
     draft_lens=[1 + (5 * b) % 8 for b in range(8)], prefix_lens=[16384] * 8, Hq=32, Hkv=8, d=128,
@@ -484,6 +487,7 @@ def make_runner(name: str, dev):
             "verify": lambda: VerifyRunner(W.VERIFY, dev),
             "verify-shared": lambda: SharedVerifyRunner(W.VERIFY_SHARED, dev),
             "verify-fp8": lambda: VerifyFp8Runner(W.VERIFY_FP8, dev),
+            "verify-fp8-8": lambda: VerifyFp8Runner(VERIFY_FP8_SMALL, dev),
             "verify-extend": lambda: ExtendVerifyRunner(W.VERIFY_PAGED, dev),
             "verify-extend8": lambda: ExtendVerifyRunner(VERIFY_PAGED_SMALL, dev),
             "grpo-backward": lambda: BackwardRunner(W.GRPO, dev),
@@ -564,7 +568,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="grpo",
                     choices=["grpo", "tiny", "large", "verify", "verify8", "verify-shared",
-                             "verify-fp8", "verify-extend", "verify-extend8", "grpo-backward",
+                             "verify-fp8", "verify-fp8-8", "verify-extend", "verify-extend8",
+                             "grpo-backward",
                              "sparse",
                              "sparse4k"])
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
