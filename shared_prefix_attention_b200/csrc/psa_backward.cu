@@ -8,8 +8,9 @@
 //   dV += P^T dO,  dS = P (dO V^T - D),  dQ += scale dS K,  dK += scale dS^T Q.
 //
 // Three launches, no atomics:
-//   prep     D and the log2-domain LSE per (row, head), stored head-major so a
-//            tile of 64 rows is one contiguous 256-byte run.
+//   prep     -D and -LSE (log2 domain) per (row, head), stored head-major so a
+//            tile of 64 rows is one contiguous 256-byte run; stored negated so
+//            two adjacent columns feed a paired fp32 add as one 8-byte load.
 //   dq pass  row-major over the forward's kind of schedule (blocks of 128
 //            rows, KV tiles of 64 keys): a CTA owns one (row block, query
 //            head) and streams the K and V tiles its rows see.
@@ -33,6 +34,8 @@
 // PSA_ERR_TIMEOUT instead of hanging; TMEM is freed on every exit path.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "psa_device.cuh"
 #include "psa_internal.h"
@@ -105,8 +108,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (lane == 0) {
-    delta_t[size_t(h) * Tp + t] = s;
-    lse2_t[size_t(h) * Tp + t] = lse[size_t(t) * Hq + h] * kLog2e;
+    delta_t[size_t(h) * Tp + t] = -s;
+    lse2_t[size_t(h) * Tp + t] = -lse[size_t(t) * Hq + h] * kLog2e;
   }
 }
 
@@ -115,8 +118,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 struct BwdParams {
   const int32_t* sched;
   int64_t sched_len;
-  const float* lse2_t;        // [Hq, Tp]
-  const float* delta_t;       // [Hq, Tp]
+  const float* lse2_t;        // [Hq, Tp], -LSE * log2(e)
+  const float* delta_t;       // [Hq, Tp], -D
   __nv_bfloat16* dq;          // [T, Hq, D]
   __nv_bfloat16* dk;          // [T, Hkv, D]
   __nv_bfloat16* dv;
@@ -419,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         continue;
       }
-      float lse_row = 0.f, dlt_row = 0.f;
+      float lse_row = 0.f, dlt_row = 0.f;  // negated, as stored
       if (MODE == kDq && rvalid) {
         lse_row = __ldg(p.lse2_t + size_t(head) * p.Tp + grow);
         dlt_row = __ldg(p.delta_t + size_t(head) * p.Tp + grow);
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             vis = rect_mask(rects, __ldg(e + 2 + 2 * half), __ldg(e + 3 + 2 * half), grow, c0);
         }
-        const float* lse_col = nullptr;
+        const float* lse_col = nullptr;  // negated, as stored
         const float* dlt_col = nullptr;
         if constexpr (MODE == kDkdv) {
           const uint8_t* st = smem + C::OFF_RING + (m % C::NST) * C::STAGE + 2 * C::TILE;
@@ -461,47 +464,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         // every column visible (the common case): no per-element mask
         const bool all_vis = vis == ~0ull;
         const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), zero2 = f2_pack(0.f, 0.f);
+        const uint64_t nl_row2 = f2_pack(lse_row, lse_row), nd_row2 = f2_pack(dlt_row, dlt_row);
+        // x = scale_log2 s - lse, P = 2^x, dS = P (dP - D), two columns at a time;
+        // PAIRS: the dkdv stats of columns (c, c + 1) are one aligned 8-byte load
+        auto tile = [&](auto pairs_tag) {
+          constexpr bool PAIRS = decltype(pairs_tag)::value;
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t s[32], dp[32];
-          tmem_ld32(tS + ch * 32, s);
-          tmem_ld32(tP + ch * 32, dp);
-          tmem_wait_ld();
-          const uint32_t vm = uint32_t(vis >> (32 * ch));
-          uint32_t pk[16], dk[16];
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t s[32], dp[32];
+            tmem_ld32(tS + ch * 32, s);
+            tmem_ld32(tP + ch * 32, dp);
+            tmem_wait_ld();
+            const uint32_t vm = uint32_t(vis >> (32 * ch));
+            uint32_t pk[16], dk[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const int col = ch * 32 + i;
-            float l0, l1, d0, d1;
-            if constexpr (MODE == kDq) {
-              l0 = l1 = lse_row;
-              d0 = d1 = dlt_row;
-            } else {
-              l0 = lse_col[col];
-              l1 = lse_col[col + 1];
-              d0 = dlt_col[col];
-              d1 = dlt_col[col + 1];
+            for (int i = 0; i < 32; i += 2) {
+              const int col = ch * 32 + i;
+              uint64_t nl2, nd2;
+              if constexpr (MODE == kDq) {
+                nl2 = nl_row2;
+                nd2 = nd_row2;
+              } else if constexpr (PAIRS) {
+                nl2 = *reinterpret_cast<const uint64_t*>(lse_col + col);
+                nd2 = *reinterpret_cast<const uint64_t*>(dlt_col + col);
+              } else {
+                nl2 = f2_pack(lse_col[col], lse_col[col + 1]);
+                nd2 = f2_pack(dlt_col[col], dlt_col[col + 1]);
+              }
+              const uint64_t x2 =
+                  f2_fma(f2_pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])), sc2, nl2);
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+              if (!all_vis) {
+                p0 = (vm >> i) & 1u ? p0 : 0.f;
+                p1 = (vm >> (i + 1)) & 1u ? p1 : 0.f;
+              }
+              const uint64_t g2 =
+                  f2_add(f2_pack(__uint_as_float(dp[i]), __uint_as_float(dp[i + 1])), nd2);
+              float ds0, ds1;
+              f2_unpack(f2_fma(f2_pack(p0, p1), g2, zero2), ds0, ds1);
+              pk[i / 2] = pack_bf16(p0, p1);
+              dk[i / 2] = pack_bf16(ds0, ds1);
             }
-            // x = scale_log2 s - lse, P = 2^x, dS = P (dP - D), two columns at a time
-            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[i]), __uint_as_float(s[i + 1])),
-                                       sc2, f2_pack(-l0, -l1));
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            if (!all_vis) {
-              p0 = (vm >> i) & 1u ? p0 : 0.f;
-              p1 = (vm >> (i + 1)) & 1u ? p1 : 0.f;
-            }
-            const uint64_t g2 = f2_add(f2_pack(__uint_as_float(dp[i]), __uint_as_float(dp[i + 1])),
-                                       f2_pack(-d0, -d1));
-            float ds0, ds1;
-            f2_unpack(f2_fma(f2_pack(p0, p1), g2, zero2), ds0, ds1);
-            pk[i / 2] = pack_bf16(p0, p1);
-            dk[i / 2] = pack_bf16(ds0, ds1);
+            if constexpr (MODE == kDkdv) tmem_st16(tS + ch * 16, pk);
+            tmem_st16(tP + ch * 16, dk);
           }
-          if constexpr (MODE == kDkdv) tmem_st16(tS + ch * 16, pk);
-          tmem_st16(tP + ch * 16, dk);
-        }
+        };
+        // the stats slot is 512-byte aligned and starts at column -(c0 & 3)
+        if (MODE == kDq || ((c0 & 3) & 1) == 0)
+          tile(std::true_type{});
+        else
+          tile(std::false_type{});
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

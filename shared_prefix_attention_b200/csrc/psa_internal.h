@@ -115,8 +115,8 @@ struct BackwardArgs {
   int64_t sched_q_len;
   const int32_t* sched_kv;  // psa_build_schedule(transposed spec, ...), same tile sizes
   int64_t sched_kv_len;
-  float* lse2_t;            // workspace [Hq, Tp], Tp = T rounded up to a multiple of 4
-  float* delta_t;           // workspace [Hq, Tp]
+  float* lse2_t;            // workspace [Hq, Tp], -LSE * log2(e); Tp = T rounded up to 4
+  float* delta_t;           // workspace [Hq, Tp], -rowsum(dO * O)
   int32_t* status;
   cudaStream_t stream;
 };
