@@ -227,9 +227,10 @@ int32_t psa_verify_auto_splits(int32_t B, int64_t max_prefix_len, int32_t Hkv,
                                int32_t head_dim);
 
 /* Workspace bytes for the split partials: nsplit * B*Ld*Hq * (d + 1) fp32,
- * plus alignment padding.  Size it for the largest batch you will run and
- * reuse it ([SKV] review: key scratch by the maximum batch, not by the
- * current one). */
+ * plus alignment padding (B*Ld is the number of draft rows: pass B = 1 and
+ * Ld = n_rows for psa_verify_extend_fwd).  Size it for the largest batch you
+ * will run and reuse it ([SKV] review: key scratch by the maximum batch, not
+ * by the current one). */
 size_t psa_verify_workspace_size(int32_t B, int32_t Ld, int32_t Hq, int32_t head_dim,
                                  int32_t nsplit);
 
