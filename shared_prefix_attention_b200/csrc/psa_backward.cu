@@ -28,9 +28,9 @@
 //   dq:   dQ += dS Y1                  tcgen05 TS MMAs (A from TMEM), the
 //   dkdv: dV += P^T Y2, dK += dS^T Y1  accumulators stay in TMEM per unit.
 // Warps: 0 TMA producer (128-byte swizzle, no multicast), 1 MMA issuer and
-// TMEM owner, 4-7 and 8-11 two compute warpgroups taking alternate tiles
-// (while one works on tile t the tensor pipe runs tile t+1's S and dP), and
-// both run the unit's epilogue.  Every wait is bounded and reports
+// TMEM owner, 4-7 and 8-11 two compute warpgroups that split every tile's
+// columns (while they work on tile t the tensor pipe runs tile t+1's S and
+// dP), and both run the unit's epilogue.  Every wait is bounded and reports
 // PSA_ERR_TIMEOUT instead of hanging; TMEM is freed on every exit path.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -158,6 +158,12 @@ struct TcCfg {
   static_assert(T_ACC + (MODE == kDq ? D : 2 * D) <= kTmemCols, "TMEM budget");
 };
 
+// Column (within a 64-column S or dP region of TMEM) of the packed bf16 P or
+// dS that k-step ks (16 tile columns) of the accumulating products reads:
+// the warpgroup that made tile columns 32 w .. 32 w + 31 packs them over the
+// first 16 of the fp32 columns it read, at 32 w.
+__host__ __device__ constexpr uint32_t a_col(int ks) { return (ks >> 1) * 32 + (ks & 1) * 8; }
+
 struct Bars {
   uint64_t *blk_full, *blk_empty, *ring_full, *ring_empty, *s_full, *p_full, *acc_full,
       *acc_free;
@@ -226,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < C::NBUF; ++i) {
       mbar_init(B.s_full + i, 1);
-      mbar_init(B.p_full + i, 4);  // the four warps of a compute warpgroup
+      mbar_init(B.p_full + i, 8);  // both compute warpgroups (half a tile each)
     }
     mbar_init(B.acc_full, 1);
     mbar_init(B.acc_free, 8);      // both compute warpgroups
@@ -349,12 +355,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t acc = (t > 0 || ks > 0) ? 1u : 0u;
           if constexpr (MODE == kDq) {
             // dQ += dS K_t
-            umma_ts(tmem + C::T_ACC, tb + 64 + ks * 8, dY + ks * (2048 >> 4), idesc_acc, acc);
+            umma_ts(tmem + C::T_ACC, tb + 64 + a_col(ks), dY + ks * (2048 >> 4), idesc_acc, acc);
           } else {
             // dV += P^T dO_t, dK += dS^T Q_t
-            umma_ts(tmem + C::T_ACC, tb + ks * 8, dY + ((C::TILE + ks * 2048) >> 4), idesc_acc,
+            umma_ts(tmem + C::T_ACC, tb + a_col(ks), dY + ((C::TILE + ks * 2048) >> 4), idesc_acc,
                     acc);
-            umma_ts(tmem + C::T_ACC + D, tb + 64 + ks * 8, dY + ks * (2048 >> 4), idesc_acc, acc);
+            umma_ts(tmem + C::T_ACC + D, tb + 64 + a_col(ks), dY + ks * (2048 >> 4), idesc_acc,
+                    acc);
           }
         }
         umma_commit(B.ring_empty + (m % C::NST));
@@ -429,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int t = 0; t < nt; ++t) {
         const uint32_t m = n + t;
-        if (int(m & 1) != wg) continue;
+
         const int j = MODE == kDq ? t : t % it.w;
         const int32_t* e = tiles + 8 * (it.z + j);
         const int c0 = __ldg(e), clen = __ldg(e + 1), flags = __ldg(e + 6);
@@ -468,9 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // x = scale_log2 s - lse, P = 2^x, dS = P (dP - D), two columns at a time;
         // PAIRS: the dkdv stats of columns (c, c + 1) are one aligned 8-byte load
         auto tile = [&](auto pairs_tag) {
-          constexpr bool PAIRS = decltype(pairs_tag)::value;
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
+          [[maybe_unused]] constexpr bool PAIRS = decltype(pairs_tag)::value;
+          {
+            const int ch = wg;  // this warpgroup's half of the tile: columns 32 ch ..
             uint32_t s[32], dp[32];
             tmem_ld32(tS + ch * 32, s);
             tmem_ld32(tP + ch * 32, dp);
@@ -479,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[16], dk[16];
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-              const int col = ch * 32 + i;
+              [[maybe_unused]] const int col = ch * 32 + i;
               uint64_t nl2, nd2;
               if constexpr (MODE == kDq) {
                 nl2 = nl_row2;
@@ -507,8 +514,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[i / 2] = pack_bf16(p0, p1);
               dk[i / 2] = pack_bf16(ds0, ds1);
             }
-            if constexpr (MODE == kDkdv) tmem_st16(tS + ch * 16, pk);
-            tmem_st16(tP + ch * 16, dk);
+            // packed over columns this thread has read itself (32 ch ..)
+            if constexpr (MODE == kDkdv) tmem_st16(tS + ch * 32, pk);
+            tmem_st16(tP + ch * 32, dk);
           }
         };
         // the stats slot is 512-byte aligned and starts at column -(c0 & 3)
