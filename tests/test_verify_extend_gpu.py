@@ -112,3 +112,30 @@ def test_paged_row_outside_the_cache_is_reported():
     torch.cuda.synchronize()
     assert psa.read_status(status) == psa.PSA_ERR_INVALID_ARG
     assert bool(torch.isfinite(o.float()).all())
+
+
+def test_verify_extend_row_that_sees_nothing():
+    """The degenerate case: a request with an empty prefix whose mask row is
+    empty sees no key at all, so O = 0 and LSE = -inf (both sides); every
+    other row matches the oracle."""
+    wl = W.ExtendVerifyWorkload("t", draft_lens=[3, 4], prefix_lens=[0, 200], Hq=8, Hkv=2,
+                                d=128, nsplit=3, tree=True, seed=97)
+    q, kd, vd, kp, vp, idx, mask = wl.make("cpu")
+    mask = mask.clone()
+    mask[1 * 3:2 * 3] = 0            # request 0, draft 1: sees nothing
+    g = [t.cuda() for t in (q, kd, vd, kp, vp, idx)]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = psa.verify_extend(g[0], g[1], g[2], g[3], g[4], _dev(wl.qo_indptr()),
+                               wl.max_draft_len, _dev(wl.kv_indptr()), wl.max_prefix_len,
+                               wl.scale, kv_indices=g[5], draft_mask=mask.cuda(),
+                               mask_indptr=_dev(wl.mask_indptr()), nsplit=wl.nsplit,
+                               status=status)
+    torch.cuda.synchronize()
+    assert psa.read_status(status) == 0
+    ro, rl = oracle.verify_extend(q, kd, vd, kp, vp, wl.qo_indptr(), wl.kv_indptr(), wl.scale,
+                                  kv_indices=idx, draft_mask=mask,
+                                  mask_indptr=wl.mask_indptr())
+    assert np.all(np.isneginf(rl[1])) and not np.any(ro[1])
+    assert bool(torch.all(o[1] == 0)) and bool(torch.all(torch.isneginf(lse[1])))
+    keep = [r for r in range(wl.n_rows) if r != 1]
+    assert_parity(o[keep], lse[keep], ro[keep], rl[keep], "rows that see keys")
