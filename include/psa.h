@@ -221,6 +221,14 @@ typedef struct psa_verify_features {
     int32_t ragged_extend;       /* per-request draft counts differ: must be 0 */
 } psa_verify_features;
 
+/* Per-tensor scales of an e4m3 KV cache ([SKV] the verify entry's k_scale /
+ * v_scale): a cached key stands for k_scale * e4m3, a cached value for
+ * v_scale * e4m3.  Both finite and > 0. */
+typedef struct psa_kv_scales {
+    float k_scale;
+    float v_scale;
+} psa_kv_scales;
+
 /* Split count chosen when nsplit == 0: enough (request, split) units to
  * fill the GPU, each covering a whole number of key tiles. */
 int32_t psa_verify_auto_splits(int32_t B, int64_t max_prefix_len, int32_t Hkv,
@@ -306,6 +314,9 @@ int psa_verify_tree_fwd(const void *q_draft, const void *k_draft, const void *v_
  *                    count) starting at dev_draft_mask[mask_indptr[b]]: draft
  *                    j sees draft i iff its (j, i) byte is non-zero
  *   dev_mask_indptr  device int32 [B+1] (required with a mask)
+ *   e4m3_scales      NULL: k_cache / v_cache are bf16; else they hold e4m3
+ *                    bytes standing for k_scale * e4m3 and v_scale * e4m3
+ *                    (as psa_verify_fp8_fwd; head_dim must be 128)
  *   o, lse           device [n_rows, Hq, d] bf16 / [n_rows, Hq] fp32
  * features->ragged_extend and ->has_custom_mask may be set here.  The
  * workspace holds the partials of n_rows rows:
@@ -318,8 +329,9 @@ int psa_verify_extend_fwd(const void *q_draft, const void *k_draft, const void *
                           const int32_t *dev_qo_indptr, int32_t n_rows, int32_t max_draft_len,
                           const int32_t *dev_kv_indptr, int64_t max_prefix_len,
                           const int32_t *dev_kv_indices, const uint8_t *dev_draft_mask,
-                          const int32_t *dev_mask_indptr, void *o, float *lse, int32_t B,
-                          int32_t Hq, int32_t Hkv, int32_t head_dim, float scale,
+                          const int32_t *dev_mask_indptr, const psa_kv_scales *e4m3_scales,
+                          void *o, float *lse, int32_t B, int32_t Hq, int32_t Hkv,
+                          int32_t head_dim, float scale,
                           int32_t nsplit, const psa_verify_features *features,
                           void *workspace, size_t ws_bytes, int32_t *dev_status, void *stream);
 

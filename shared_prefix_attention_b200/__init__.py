@@ -6,7 +6,8 @@ seeded workload generators.  The library is loaded on first use and a
 missing build raises -- there is no CPU fallback.
 """
 from ._binding import (  # noqa: F401
-    EXPORTS, LIB_PATH, PsaError, Rect, Segment, VerifyFeatures, build_schedule, build_spec,
+    EXPORTS, LIB_PATH, PsaError, Rect, Segment, VerifyFeatures, KvScales, build_schedule,
+    build_spec,
     lib, plan_prefill, prefill, prefill_tiles, read_status, sparse_latent, spec_flat,
     status_string, verify, verify_auto_splits, verify_noalloc, verify_workspace_size,
     wait_selftest, verify_shared, verify_shared_auto_splits, verify_fp8, transpose_spec,

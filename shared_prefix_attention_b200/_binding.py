@@ -60,6 +60,11 @@ class VerifyFeatures(ctypes.Structure):
                 ("ragged_extend", ctypes.c_int32)]
 
 
+class KvScales(ctypes.Structure):
+    """psa_kv_scales: per-tensor scales of an e4m3 KV cache."""
+    _fields_ = [("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
+
+
 _lib = None
 
 
@@ -99,8 +104,8 @@ def lib():
         "psa_prefill_bwd_tiles": ([I32, P, P], ctypes.c_int),
         "psa_verify_tree_fwd": ([P, P, P, P, P, I64, P, I64, P, P, P, P, I32, I32, I32, I32, I32,
                                  F, I32, P, P, SZ, P, P], ctypes.c_int),
-        "psa_verify_extend_fwd": ([P, P, P, P, P, I64, P, I32, I32, P, I64, P, P, P, P, P, I32,
-                                   I32, I32, I32, F, I32, P, P, SZ, P, P], ctypes.c_int),
+        "psa_verify_extend_fwd": ([P, P, P, P, P, I64, P, I32, I32, P, I64, P, P, P, P, P, P,
+                                   I32, I32, I32, I32, F, I32, P, P, SZ, P, P], ctypes.c_int),
         "psa_prefill_bwd_workspace_size": ([I32, I32], SZ),
         "psa_prefill_bwd": ([P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, F, P, I64, P, I64, P,
                              SZ, P, P], ctypes.c_int),
@@ -440,11 +445,13 @@ def verify_tree(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr: torch.Te
 def verify_extend(q_draft, k_draft, v_draft, k_cache, v_cache, qo_indptr: torch.Tensor,
                   max_draft_len: int, kv_indptr: torch.Tensor, max_prefix_len: int,
                   scale: float, kv_indices=None, draft_mask=None, mask_indptr=None,
-                  nsplit: int = 0, out=None, lse=None, workspace=None, status=None):
+                  nsplit: int = 0, out=None, lse=None, workspace=None, status=None,
+                  k_scale: float | None = None, v_scale: float | None = None):
     """Verify in the extend form: ragged draft counts (qo_indptr, device int32
     [B+1]), an optional page table (kv_indices: prefix position t is cache row
     kv_indices[t]) and optional per-request tree masks (flat device uint8,
-    request b's Lb x Lb block at mask_indptr[b])."""
+    request b's Lb x Lb block at mask_indptr[b]).  With k_scale / v_scale the
+    caches hold e4m3 bytes standing for k_scale * e4m3 and v_scale * e4m3."""
     _require_cuda(q_draft, k_draft, v_draft, k_cache, v_cache, qo_indptr, kv_indptr)
     NR, Hq, d = q_draft.shape
     Hkv = k_draft.shape[1]
@@ -456,11 +463,14 @@ def verify_extend(q_draft, k_draft, v_draft, k_cache, v_cache, qo_indptr: torch.
         workspace = torch.empty(max(verify_workspace_size(1, NR, Hq, d, ns), 256),
                                 dtype=torch.uint8, device=q_draft.device)
     feat = VerifyFeatures(int(draft_mask is not None), 1, -1, 0, 0.0, -1, 1)
+    sc = None
+    if k_scale is not None or v_scale is not None:
+        sc = ctypes.byref(KvScales(float(k_scale), float(v_scale)))
     rc = lib().psa_verify_extend_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft),
                                      _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
                                      _ptr(qo_indptr), NR, int(max_draft_len), _ptr(kv_indptr),
                                      int(max_prefix_len), _ptr(kv_indices), _ptr(draft_mask),
-                                     _ptr(mask_indptr), _ptr(out), _ptr(lse), B, Hq, Hkv, d,
+                                     _ptr(mask_indptr), sc, _ptr(out), _ptr(lse), B, Hq, Hkv, d,
                                      float(scale), ns, ctypes.byref(feat), _ptr(workspace),
                                      workspace.numel(), _ptr(status), _stream(q_draft.device))
     _check(rc, "psa_verify_extend_fwd")

@@ -143,7 +143,8 @@ static int verify_common(const void* q_draft, const void* k_draft, const void* v
                               void* workspace, size_t ws_bytes, int32_t* dev_status,
                               void* stream, const uint8_t* dmask,
                               const int32_t* qo_indptr = nullptr, int32_t n_rows = 0,
-                              const int32_t* mask_indptr = nullptr) {
+                              const int32_t* mask_indptr = nullptr,
+                              const psa_kv_scales* e4m3 = nullptr) {
   // The split-KV path's gating ("can_handle"): everything else is refused;
   // a custom draft mask only through the entries that pass dmask, ragged
   // draft counts only through the extend entry, which passes qo_indptr.
@@ -161,7 +162,11 @@ static int verify_common(const void* q_draft, const void* k_draft, const void* v
   const int64_t rows_all = qo_indptr ? int64_t(n_rows) : int64_t(B) * Ld;
   if (qo_indptr && (n_rows < 0 || int64_t(n_rows) > int64_t(B) * Ld)) return PSA_ERR_INVALID_ARG;
   if (rows_all * Hq > INT32_MAX) return PSA_ERR_INVALID_ARG;
-  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PSA_ERR_UNSUPPORTED;
+  if (e4m3 && (!(e4m3->k_scale > 0.f) || !(e4m3->v_scale > 0.f) ||
+               !std::isfinite(e4m3->k_scale) || !std::isfinite(e4m3->v_scale)))
+    return PSA_ERR_INVALID_ARG;
+  if (e4m3 ? head_dim != 128 : (head_dim != 64 && head_dim != 128 && head_dim != 256))
+    return PSA_ERR_UNSUPPORTED;
   if (B == 0 || rows_all == 0) return PSA_OK;
   if (!q_draft || !k_draft || !v_draft || !k_cache || !v_cache || !dev_kv_indptr || !o)
     return PSA_ERR_INVALID_ARG;
@@ -205,7 +210,7 @@ static int verify_common(const void* q_draft, const void* k_draft, const void* v
   a.qo_indptr = qo_indptr;
   a.mask_indptr = mask_indptr;
   a.n_rows = int32_t(rows_all);
-  return launch_verify(a);
+  return e4m3 ? launch_verify_fp8(a, e4m3->k_scale, e4m3->v_scale) : launch_verify(a);
 }
 
 extern "C" int psa_verify_fwd(const void* q_draft, const void* k_draft, const void* v_draft,
@@ -243,7 +248,8 @@ extern "C" int psa_verify_extend_fwd(
     const void* v_cache, int64_t n_cache_tokens, const int32_t* dev_qo_indptr, int32_t n_rows,
     int32_t max_draft_len, const int32_t* dev_kv_indptr, int64_t max_prefix_len,
     const int32_t* dev_kv_indices, const uint8_t* dev_draft_mask,
-    const int32_t* dev_mask_indptr, void* o, float* lse, int32_t B, int32_t Hq, int32_t Hkv,
+    const int32_t* dev_mask_indptr, const psa_kv_scales* e4m3_scales, void* o, float* lse,
+    int32_t B, int32_t Hq, int32_t Hkv,
     int32_t head_dim, float scale, int32_t nsplit, const psa_verify_features* features,
     void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
   if (B > 0 && !dev_qo_indptr) return PSA_ERR_INVALID_ARG;
@@ -252,7 +258,7 @@ extern "C" int psa_verify_extend_fwd(
                        dev_kv_indptr, max_prefix_len, dev_kv_indices, o, lse, B, max_draft_len,
                        Hq, Hkv, head_dim, scale, nsplit, features, workspace, ws_bytes,
                        dev_status, stream, dev_draft_mask, B > 0 ? dev_qo_indptr : nullptr,
-                       n_rows, dev_mask_indptr);
+                       n_rows, dev_mask_indptr, e4m3_scales);
 }
 
 extern "C" int psa_verify_fp8_fwd(const void* q_draft, const void* k_draft, const void* v_draft,
@@ -264,57 +270,11 @@ extern "C" int psa_verify_fp8_fwd(const void* q_draft, const void* k_draft, cons
                                   float scale, int32_t nsplit,
                                   const psa_verify_features* features, void* workspace,
                                   size_t ws_bytes, int32_t* dev_status, void* stream) {
-  if (features) {
-    if (features->has_custom_mask || !features->is_causal || features->sliding_window > 0 ||
-        features->has_sinks || features->logit_cap != 0.f ||
-        features->xai_temperature_len > 0 || features->ragged_extend)
-      return PSA_ERR_UNSUPPORTED;
-  }
-  if (B < 0 || Ld <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n_cache_tokens < 0 ||
-      max_prefix_len < 0 || n_cache_tokens > INT32_MAX || !(scale > 0.f) ||
-      !(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
-    return PSA_ERR_INVALID_ARG;
-  if (head_dim != 128) return PSA_ERR_UNSUPPORTED;
-  if (B == 0) return PSA_OK;
-  if (!q_draft || !k_draft || !v_draft || !k_cache || !v_cache || !dev_kv_indptr || !o)
-    return PSA_ERR_INVALID_ARG;
-  if (!aligned16(q_draft) || !aligned16(k_draft) || !aligned16(v_draft) ||
-      !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
-    return PSA_ERR_INVALID_ARG;
-  int32_t HB = 0, MT = 0, NRB = 0;
-  if (!verify_plan(Ld, Hq, Hkv, head_dim, &HB, &MT, &NRB)) return PSA_ERR_UNSUPPORTED;
-  if (nsplit == 0) nsplit = psa_verify_auto_splits(B, max_prefix_len, Hkv, head_dim);
-  if (nsplit < 1 || nsplit > 256) return PSA_ERR_INVALID_ARG;
-  const size_t need = psa_verify_workspace_size(B, Ld, Hq, head_dim, nsplit);
-  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-    return PSA_ERR_WORKSPACE;
-
-  VerifyArgs a;
-  a.q = q_draft;
-  a.kd = k_draft;
-  a.vd = v_draft;
-  a.kc = k_cache;
-  a.vc = v_cache;
-  a.indptr = dev_kv_indptr;
-  a.n_cache_tokens = n_cache_tokens;
-  a.o = o;
-  a.lse = lse;
-  a.B = B;
-  a.Ld = Ld;
-  a.Hq = Hq;
-  a.Hkv = Hkv;
-  a.D = head_dim;
-  a.scale = scale;
-  a.nsplit = nsplit;
-  const size_t rows = size_t(nsplit) * B * Ld * Hq;
-  const size_t o_bytes = (rows * head_dim * sizeof(float) + 255) / 256 * 256;
-  a.part_o = static_cast<float*>(workspace);
-  a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + o_bytes);
-  a.status = dev_status;
-  a.stream = static_cast<cudaStream_t>(stream);
-  a.kv_indices = kv_indices;
-  return launch_verify_fp8(a, k_scale, v_scale);
+  const psa_kv_scales sc{k_scale, v_scale};
+  return verify_common(q_draft, k_draft, v_draft, k_cache, v_cache, n_cache_tokens,
+                       dev_kv_indptr, max_prefix_len, kv_indices, o, lse, B, Ld, Hq, Hkv,
+                       head_dim, scale, nsplit, features, workspace, ws_bytes, dev_status, stream,
+                       nullptr, nullptr, 0, nullptr, &sc);
 }
 
 // ------------------------------------------------------- shared-prefix verify

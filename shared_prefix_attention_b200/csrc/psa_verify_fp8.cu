@@ -48,6 +48,10 @@ struct P8Params {
   int64_t ntok;
   float* part_o;
   float* part_lse;
+  // Extend form (nullable): request b's draft rows are [qo_indptr[b],
+  // qo_indptr[b+1]); Ld is then the largest draft count, nrows the total.
+  const int32_t* qo_indptr;
+  int32_t nrows;
   int32_t B, Ld, Hq, Hkv, G, R;
   int32_t MT, nrb, HB, nhb, nsplit, nstage;
   float logit_scale_log2;  // scale * k_scale * log2(e)
@@ -68,6 +72,32 @@ __device__ __forceinline__ Unit8 decode_unit8(const P8Params& p, int u) {
   x.s = u % p.nsplit;
   x.b = u / p.nsplit;
   return x;
+}
+
+// First draft row and draft count of request b (a count above Ld is
+// reported and clamped; rows outside [0, nrows) empty the request).
+__device__ __forceinline__ void request_rows8(const P8Params& p, int b, int& q0, int& Lb,
+                                              int32_t* status) {
+  if (!p.qo_indptr) {
+    q0 = b * p.Ld;
+    Lb = p.Ld;
+    return;
+  }
+  q0 = __ldg(p.qo_indptr + b);
+  Lb = __ldg(p.qo_indptr + b + 1) - q0;
+  if (Lb > p.Ld) {
+    report_status(status, PSA_ERR_INVALID_ARG);
+    Lb = p.Ld;
+  }
+  if (Lb < 0 || q0 < 0 || q0 > p.nrows - Lb) {
+    report_status(status, PSA_ERR_INVALID_ARG);
+    Lb = 0;
+  }
+}
+
+// A unit does work only if its row block holds a draft row of the request.
+__device__ __forceinline__ bool unit_live8(const P8Params& p, const Unit8& x, int Lb) {
+  return x.rb * p.MT * 16 < Lb * p.G;
 }
 
 __device__ __forceinline__ void split_range8(const P8Params& p, int b, int s, int32_t& t0,
@@ -215,6 +245,9 @@ __global__ void __launch_bounds__((kMaxWarps + (PAGED ? kPagedProducers8 : 1)) *
       for (int i = 0; i < 16; ++i) last_phase[i] = -1;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const Unit8 x = decode_unit8(p, u);
+        int q0, Lb;
+        request_rows8(p, x.b, q0, Lb, nullptr);
+        if (!unit_live8(p, x, Lb)) continue;
         int32_t t0, t1;
         split_range8(p, x.b, x.s, t0, t1);
         constexpr int kPrefetch = 8;
@@ -288,6 +321,9 @@ __global__ void __launch_bounds__((kMaxWarps + (PAGED ? kPagedProducers8 : 1)) *
       for (int i = 0; i < 16; ++i) last_phase[i] = -1;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const Unit8 x = decode_unit8(p, u);
+        int q0, Lb;
+        request_rows8(p, x.b, q0, Lb, nullptr);
+        if (!unit_live8(p, x, Lb)) continue;
         int32_t t0, t1;
         split_range8(p, x.b, x.s, t0, t1);
         for (int32_t t = t0; t < t1; t += kKeys) {
@@ -324,7 +360,7 @@ __global__ void __launch_bounds__((kMaxWarps + (PAGED ? kPagedProducers8 : 1)) *
   const int hh = warp / p.MT;  // KV head within the group
   const int mt = warp % p.MT;  // 16-row m-tile of that head's rows
   const int g = lane >> 2, c = lane & 3;
-  const int BL = p.B * p.Ld;
+  const int BL = p.nrows;
   const uint32_t vpriv = smem_u32(priv + warp * kPrivBytes);
   int stage = 0;
   uint32_t phase = 0;
@@ -333,6 +369,9 @@ __global__ void __launch_bounds__((kMaxWarps + (PAGED ? kPagedProducers8 : 1)) *
     const Unit8 x = decode_unit8(p, u);
     const int b = x.b, s = x.s;
     const int kvh = x.hb * p.HB + hh;
+    int q0, Lb;
+    request_rows8(p, b, q0, Lb, nullptr);
+    if (!unit_live8(p, x, Lb)) continue;
     int32_t t0, t1;
     split_range8(p, b, s, t0, t1);
 
@@ -341,10 +380,10 @@ __global__ void __launch_bounds__((kMaxWarps + (PAGED ? kPagedProducers8 : 1)) *
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int rr = (x.rb * p.MT + mt) * 16 + g + 8 * i;
-      rvalid[i] = rr < p.R;
+      rvalid[i] = rr < Lb * p.G;
       const int j = rvalid[i] ? rr / p.G : 0;
       rqh[i] = kvh * p.G + (rvalid[i] ? rr % p.G : 0);
-      rrow[i] = b * p.Ld + j;
+      rrow[i] = q0 + j;
     }
 
     // Q fragments (A operand) widened to f16
@@ -515,6 +554,8 @@ int launch_verify_fp8(const VerifyArgs& a, float k_scale, float v_scale) {
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.indptr = a.indptr;
   p.kv_indices = a.kv_indices;
+  p.qo_indptr = a.qo_indptr;
+  p.nrows = a.qo_indptr ? a.n_rows : a.B * a.Ld;
   p.kc8 = static_cast<const uint8_t*>(a.kc);
   p.vc8 = static_cast<const uint8_t*>(a.vc);
   p.ntok = a.n_cache_tokens;

@@ -133,14 +133,16 @@ def test_verify_tree_needs_a_mask():
 
 
 def _extend_call(**kw):
-    args = dict(qo=16, nrows=6, maxld=4, B=2, mask=None, mi=None, feat=None, ws=None, wsb=0)
+    args = dict(qo=16, nrows=6, maxld=4, B=2, mask=None, mi=None, feat=None, ws=None, wsb=0,
+                sc=None, d=128)
     args.update(kw)
     a = args
     P = ctypes.c_void_p
     opt = lambda v: P(v) if v else None  # noqa: E731
+    sc = ctypes.byref(a["sc"]) if a["sc"] is not None else None
     return psa.lib().psa_verify_extend_fwd(
         P(16), P(16), P(16), P(16), P(16), 64, opt(a["qo"]), a["nrows"], a["maxld"], P(16), 64,
-        None, opt(a["mask"]), opt(a["mi"]), P(16), None, a["B"], 8, 2, 128, 0.1, 1,
+        None, opt(a["mask"]), opt(a["mi"]), sc, P(16), None, a["B"], 8, 2, a["d"], 0.1, 1,
         ctypes.byref(a["feat"]) if a["feat"] is not None else None, opt(a["ws"]), a["wsb"],
         None, None)
 
@@ -156,6 +158,11 @@ def test_verify_extend_host_validation():
     assert _extend_call(nrows=9) == psa.PSA_ERR_INVALID_ARG          # more rows than B * max
     assert _extend_call(maxld=17) == psa.PSA_ERR_UNSUPPORTED         # m-tile plan: 17 * 4 > 128
     assert _extend_call(nrows=0) == psa.PSA_OK                       # no draft rows
+    # an e4m3 cache: head_dim 128 only, finite positive scales
+    assert _extend_call(sc=psa.KvScales(0.5, 0.25)) == psa.PSA_ERR_WORKSPACE
+    assert _extend_call(sc=psa.KvScales(0.5, 0.25), d=64) == psa.PSA_ERR_UNSUPPORTED
+    assert _extend_call(sc=psa.KvScales(0.0, 0.25)) == psa.PSA_ERR_INVALID_ARG
+    assert _extend_call(sc=psa.KvScales(0.5, float("inf"))) == psa.PSA_ERR_INVALID_ARG
 
 
 def test_verify_fp8_host_validation():

@@ -139,3 +139,36 @@ def test_verify_extend_row_that_sees_nothing():
     assert bool(torch.all(o[1] == 0)) and bool(torch.all(torch.isneginf(lse[1])))
     keep = [r for r in range(wl.n_rows) if r != 1]
     assert_parity(o[keep], lse[keep], ro[keep], rl[keep], "rows that see keys")
+
+
+@pytest.mark.parametrize("drafts,prefixes,Hq,Hkv,nsplit,tree", [
+    ([3, 0, 5, 1], [300, 77, 0, 1000], 32, 8, 4, True),   # ragged, paged, trees, an empty one
+    ([8, 8, 2], [2048, 15, 513], 16, 2, 16, False),      # ragged drafts, causal blocks
+])
+def test_verify_extend_e4m3(drafts, prefixes, Hq, Hkv, nsplit, tree):
+    """The extend form over an e4m3 cache ([SKV]: the verify entry takes
+    k_scale / v_scale with the page table and the masks).  Reference: the
+    oracle's extend form on the decoded, scaled cache (the fp8 verify equals
+    the float verify on that cache, a pinned identity)."""
+    wl = W.ExtendVerifyWorkload("t", draft_lens=drafts, prefix_lens=prefixes, Hq=Hq, Hkv=Hkv,
+                                d=128, nsplit=nsplit, tree=tree, seed=sum(drafts) + 31)
+    q, kd, vd, kp, vp, idx, mask = wl.make("cpu")
+    ks, vs = 1.0 / 96, 1.0 / 80
+    kp8 = (kp.float() / ks).to(torch.float8_e4m3fn).view(torch.uint8)
+    vp8 = (vp.float() / vs).to(torch.float8_e4m3fn).view(torch.uint8)
+    g = [t.cuda() for t in (q, kd, vd, kp8, vp8, idx)]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = psa.verify_extend(g[0], g[1], g[2], g[3], g[4], _dev(wl.qo_indptr()),
+                               wl.max_draft_len, _dev(wl.kv_indptr()), wl.max_prefix_len,
+                               wl.scale, kv_indices=g[5],
+                               draft_mask=None if mask is None else mask.cuda(),
+                               mask_indptr=None if mask is None else _dev(wl.mask_indptr()),
+                               nsplit=nsplit, status=status, k_scale=ks, v_scale=vs)
+    torch.cuda.synchronize()
+    assert psa.read_status(status) == 0
+    kdec = torch.from_numpy(oracle.decode_e4m3(kp8) * ks)
+    vdec = torch.from_numpy(oracle.decode_e4m3(vp8) * vs)
+    ro, rl = oracle.verify_extend(q, kd, vd, kdec, vdec, wl.qo_indptr(), wl.kv_indptr(),
+                                  wl.scale, kv_indices=idx, draft_mask=mask,
+                                  mask_indptr=None if mask is None else wl.mask_indptr())
+    assert_parity(o, lse, ro, rl, f"e4m3 drafts={drafts} prefixes={prefixes}")
