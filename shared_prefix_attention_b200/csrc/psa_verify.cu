@@ -15,7 +15,14 @@
 // normalised partial O and its log2-domain LSE in the workspace.
 //
 // Stage 2 has one warp per (draft row, query head): it scores the draft
-// keys 0..j, then merges them with every split by LSE weights.
+// keys 0..j (or the row of a tree mask), then merges them with every split
+// by LSE weights.
+//
+// The extend form of the same call: a paged prefix (a page table of one
+// token per page; the PAGED instantiation gathers each key's row of HB heads
+// with one bulk copy, issued by four producer warps, into a padded row
+// layout), ragged draft counts (rows mapped through qo_indptr; units with no
+// live row skipped) and per-request tree masks (stage 2).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

@@ -21,6 +21,10 @@
 // Q is widened from bf16 to f16 for the f16 MMAs (exact for |q| < 65504 and
 // above the f16 subnormal range) and P is rounded to f16 (finer than bf16).
 // Stage 2 is the bf16 verify's combine kernel, unchanged.
+// The same kernel serves the verify entry's other forms: a paged prefix (the
+// PAGED instantiation gathers each key's e4m3 row with a bulk copy into a
+// padded row layout) and ragged draft counts (units whose rows are all past
+// their request's count are skipped); tree masks live in the combine.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
