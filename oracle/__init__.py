@@ -72,6 +72,8 @@ def load(path: str | None = None):
     lib.oracle_verify_shared.argtypes = [P, P, P, P, P, ctypes.c_int64, I, I, I, I, I, D, P, I,
                                          P, P, I]
     lib.oracle_verify_fp8.argtypes = [P, P, P, P, P, D, D, P, I, I, I, I, I, D, P, I, P, P, I]
+    lib.oracle_verify_shared_tree.argtypes = [P, P, P, P, P, ctypes.c_int64, P, I, I, I, I, I, D,
+                                              P, I, P, P, I]
     lib.oracle_verify_fp8_paged.argtypes = [P, P, P, P, P, D, D, P, P, I, I, I, I, I, D, P, I,
                                             P, P, I]
     lib.oracle_decode_e4m3.argtypes = [P, P, ctypes.c_int64]
@@ -79,7 +81,7 @@ def load(path: str | None = None):
     lib.oracle_visibility.argtypes = [P, P, P, I, I, I, I, P]
     for f in (lib.oracle_prefill, lib.oracle_prefill_bwd, lib.oracle_prefill_bwd_dq,
               lib.oracle_verify, lib.oracle_verify_tree, lib.oracle_verify_extend,
-              lib.oracle_verify_shared,
+              lib.oracle_verify_shared, lib.oracle_verify_shared_tree,
               lib.oracle_verify_fp8, lib.oracle_verify_fp8_paged, lib.oracle_decode_e4m3, lib.oracle_sparse_latent,
               lib.oracle_visibility):
         f.restype = I
@@ -272,7 +274,7 @@ def verify_extend(q_draft, k_draft, v_draft, k_cache, v_cache, qo_indptr, kv_ind
 
 
 def verify_shared(q_draft, k_draft, v_draft, k_prefix, v_prefix, Ld: int, scale: float,
-                  rows=None, nthreads: int | None = None, lib=None):
+                  rows=None, nthreads: int | None = None, lib=None, draft_mask=None):
     """O [nrows, Hq, d] and LSE [nrows, Hq] for draft rows b*Ld + j when every
     request sees the same prefix k_prefix/v_prefix [L, Hkv, d]."""
     lib = lib or load()
@@ -284,9 +286,18 @@ def verify_shared(q_draft, k_draft, v_draft, k_prefix, v_prefix, Ld: int, scale:
     rows = np.arange(BL, dtype=np.int32) if rows is None else _i32(rows)
     o = np.zeros((len(rows), Hq, d), dtype=np.float64)
     lse = np.zeros((len(rows), Hq), dtype=np.float64)
-    rc = lib.oracle_verify_shared(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kp), _ptr(vp),
-                                  int(kp.shape[0]), B, Ld, Hq, Hkv, d, float(scale), _ptr(rows),
-                                  len(rows), _ptr(o), _ptr(lse), nthreads or default_threads())
+    if draft_mask is None:
+        rc = lib.oracle_verify_shared(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kp), _ptr(vp),
+                                      int(kp.shape[0]), B, Ld, Hq, Hkv, d, float(scale),
+                                      _ptr(rows), len(rows), _ptr(o), _ptr(lse),
+                                      nthreads or default_threads())
+    else:
+        dm = _u8(draft_mask)
+        assert dm.shape == (BL, Ld)
+        rc = lib.oracle_verify_shared_tree(_ptr(qd), _ptr(kd), _ptr(vd), _ptr(kp), _ptr(vp),
+                                           int(kp.shape[0]), _ptr(dm), B, Ld, Hq, Hkv, d,
+                                           float(scale), _ptr(rows), len(rows), _ptr(o),
+                                           _ptr(lse), nthreads or default_threads())
     assert rc == 0, "oracle_verify_shared rejected its arguments"
     return o, lse
 

@@ -603,6 +603,24 @@ int oracle_verify_shared(const float *qd, const float *kd, const float *vd,
     return 0;
 }
 
+/*
+ * Tree verify against one shared prefix: oracle_verify_shared with the draft
+ * block given by dmask [B*Ld, Ld] as in oracle_verify_tree (the prefix stays
+ * fully visible).  By definition this equals oracle_verify_tree on a cache
+ * holding B copies of the prefix.
+ */
+int oracle_verify_shared_tree(const float *qd, const float *kd, const float *vd,
+                              const float *kp, const float *vp, int64_t L,
+                              const uint8_t *dmask, int B, int Ld, int Hq, int Hkv, int d,
+                              double scale, const int32_t *rows, int nrows, double *o,
+                              double *lse, int nthreads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || d <= 0 || B < 0 || Ld <= 0 || L < 0 || !dmask) return -1;
+    verify_ctx c = {qd, kd, vd, kp, vp, NULL, L, Ld, Hq, Hkv, d, scale, rows, o, lse, dmask,
+                    NULL, NULL, NULL};
+    run_rows(verify_row, &c, nrows, (int)L + Ld, d, nthreads);
+    return 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* verify with an fp8 (e4m3) prefix cache and per-tensor scales         */
 /* ------------------------------------------------------------------ */

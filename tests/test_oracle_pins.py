@@ -420,6 +420,21 @@ def pin_verify_shared_prefix(lib):
     indptr = np.arange(B + 1, dtype=np.int64) * L
     o2, lse2 = oracle.verify(q, kd, vd, kc, vc, indptr, Ld, scale, lib=lib)
     ok &= np.array_equal(o, o2) and np.array_equal(lse, lse2)
+    # with a draft tree per request ([SKV] can_handle: topk > 1): SDPA with the
+    # tree over the drafts, and the per-request tree verify on the B copies
+    rng = np.random.default_rng(56)
+    trees = [_random_tree(Ld, rng) for _ in range(B)]
+    dm = np.concatenate(trees).astype(np.uint8)
+    o3, l3 = oracle.verify_shared(q, kd, vd, kp, vp, Ld, scale, lib=lib, draft_mask=dm)
+    for b in range(B):
+        ks = torch.cat([kp, kd[b * Ld:(b + 1) * Ld]])
+        vs = torch.cat([vp, vd[b * Ld:(b + 1) * Ld]])
+        mask = torch.ones((Ld, L + Ld), dtype=torch.bool)
+        mask[:, L:] = torch.from_numpy(trees[b].astype(bool))
+        ref = _sdpa(q[b * Ld:(b + 1) * Ld], _expand_kv(ks, Hq), _expand_kv(vs, Hq), mask, scale)
+        ok &= np.allclose(o3[b * Ld:(b + 1) * Ld], ref, atol=1e-12)
+    o4, l4 = oracle.verify_tree(q, kd, vd, kc, vc, indptr, dm, Ld, scale, lib=lib)
+    ok &= np.array_equal(o3, o4) and np.array_equal(l3, l4)
     return bool(ok)
 
 
