@@ -438,6 +438,23 @@ int psa_verify_shared_fwd(const void *q_draft, const void *k_draft, const void *
                           int32_t head_dim, float scale, int32_t nsplit, void *workspace,
                           size_t ws_bytes, int32_t *dev_status, void *stream);
 
+/*
+ * psa_verify_shared_fwd with the draft block given by a custom mask (tree
+ * verify against one shared prefix: [SKV] key code, can_handle -- EAGLE
+ * trees with topk > 1 bring a custom mask; [PS] design summary -- the prefix
+ * stored once).  dev_draft_mask: device uint8 [B*Ld, Ld], draft j of request
+ * b sees draft i of b iff dev_draft_mask[(b*Ld + j)*Ld + i] != 0 (required
+ * when B > 0: PSA_ERR_INVALID_ARG otherwise); every draft sees the whole
+ * prefix.  A row that sees no key gets O = 0 and LSE = -inf.  Everything
+ * else as psa_verify_shared_fwd.
+ */
+int psa_verify_shared_tree_fwd(const void *q_draft, const void *k_draft, const void *v_draft,
+                               const void *k_prefix, const void *v_prefix, int64_t prefix_len,
+                               const uint8_t *dev_draft_mask, void *o, float *lse, int32_t B,
+                               int32_t Ld, int32_t Hq, int32_t Hkv, int32_t head_dim,
+                               float scale, int32_t nsplit, void *workspace, size_t ws_bytes,
+                               int32_t *dev_status, void *stream);
+
 /* ------------------------------------------------------------------------
  * Shared-latent sparse attention                     [MLA] environment,
  * analysis (head-blocked tiles; the latent is shared by every head)

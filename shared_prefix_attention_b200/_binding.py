@@ -32,6 +32,7 @@ EXPORTS = [
     "psa_prefill_fwd", "psa_verify_auto_splits", "psa_verify_workspace_size",
     "psa_verify_fwd", "psa_verify_fwd_noalloc", "psa_sparse_latent_fwd", "psa_read_status",
     "psa_wait_selftest", "psa_verify_shared_auto_splits", "psa_verify_shared_fwd",
+    "psa_verify_shared_tree_fwd",
     "psa_verify_fp8_fwd", "psa_transpose_spec", "psa_prefill_bwd_tiles",
     "psa_prefill_bwd_workspace_size", "psa_prefill_bwd", "psa_verify_tree_fwd",
     "psa_verify_extend_fwd",
@@ -111,6 +112,8 @@ def lib():
                              SZ, P, P], ctypes.c_int),
         "psa_verify_fp8_fwd": ([P, P, P, P, P, I64, P, I64, P, F, F, P, P, I32, I32, I32, I32,
                                 I32, F, I32, P, P, SZ, P, P], ctypes.c_int),
+        "psa_verify_shared_tree_fwd": ([P, P, P, P, P, I64, P, P, P, I32, I32, I32, I32, I32, F,
+                                        I32, P, ctypes.c_size_t, P, P], ctypes.c_int),
         "psa_verify_shared_fwd": ([P, P, P, P, P, I64, P, P, I32, I32, I32, I32, I32, F, I32, P,
                                    ctypes.c_size_t, P, P], ctypes.c_int),
     }
@@ -325,9 +328,11 @@ def verify_shared_auto_splits(B: int, Ld: int, Hq: int, Hkv: int, prefix_len: in
 
 
 def verify_shared(q_draft, k_draft, v_draft, k_prefix, v_prefix, scale: float, Ld: int,
-                  nsplit: int = 0, out=None, lse=None, workspace=None, status=None):
+                  nsplit: int = 0, out=None, lse=None, workspace=None, status=None,
+                  draft_mask=None):
     """Verify against one prefix shared by every request: O [B*Ld, Hq, d]
-    bf16 and LSE [B*Ld, Hq] fp32; k_prefix/v_prefix [L, Hkv, d]."""
+    bf16 and LSE [B*Ld, Hq] fp32; k_prefix/v_prefix [L, Hkv, d].  With
+    draft_mask (device uint8 [B*Ld, Ld]) the draft block is that tree mask."""
     _require_cuda(q_draft, k_draft, v_draft, k_prefix, v_prefix)
     BL, Hq, d = q_draft.shape
     Hkv = k_draft.shape[1]
@@ -339,12 +344,20 @@ def verify_shared(q_draft, k_draft, v_draft, k_prefix, v_prefix, scale: float, L
     if workspace is None:
         workspace = torch.empty(max(verify_workspace_size(B, Ld, Hq, d, ns), 256),
                                 dtype=torch.uint8, device=q_draft.device)
-    rc = lib().psa_verify_shared_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft),
-                                     _ptr(k_prefix) if L else None,
-                                     _ptr(v_prefix) if L else None, L, _ptr(out), _ptr(lse), B,
-                                     Ld, Hq, Hkv, d, float(scale), ns, _ptr(workspace),
-                                     workspace.numel(), _ptr(status), _stream(q_draft.device))
-    _check(rc, "psa_verify_shared_fwd")
+    kp, vp = (_ptr(k_prefix) if L else None), (_ptr(v_prefix) if L else None)
+    if draft_mask is None:
+        rc = lib().psa_verify_shared_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft), kp, vp, L,
+                                         _ptr(out), _ptr(lse), B, Ld, Hq, Hkv, d, float(scale), ns,
+                                         _ptr(workspace), workspace.numel(), _ptr(status),
+                                         _stream(q_draft.device))
+        _check(rc, "psa_verify_shared_fwd")
+    else:
+        rc = lib().psa_verify_shared_tree_fwd(_ptr(q_draft), _ptr(k_draft), _ptr(v_draft), kp, vp,
+                                              L, _ptr(draft_mask), _ptr(out), _ptr(lse), B, Ld,
+                                              Hq, Hkv, d, float(scale), ns, _ptr(workspace),
+                                              workspace.numel(), _ptr(status),
+                                              _stream(q_draft.device))
+        _check(rc, "psa_verify_shared_tree_fwd")
     return out, lse
 
 

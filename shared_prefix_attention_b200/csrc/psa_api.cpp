@@ -295,13 +295,12 @@ extern "C" int32_t psa_verify_shared_auto_splits(int32_t B, int32_t Ld, int32_t 
   return int32_t(n);
 }
 
-extern "C" int psa_verify_shared_fwd(const void* q_draft, const void* k_draft,
-                                     const void* v_draft, const void* k_prefix,
-                                     const void* v_prefix, int64_t prefix_len, void* o,
-                                     float* lse, int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv,
-                                     int32_t head_dim, float scale, int32_t nsplit,
-                                     void* workspace, size_t ws_bytes, int32_t* dev_status,
-                                     void* stream) {
+static int verify_shared_common(const void* q_draft, const void* k_draft, const void* v_draft,
+                                const void* k_prefix, const void* v_prefix, int64_t prefix_len,
+                                void* o, float* lse, int32_t B, int32_t Ld, int32_t Hq,
+                                int32_t Hkv, int32_t head_dim, float scale, int32_t nsplit,
+                                void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                void* stream, const uint8_t* dmask) {
   if (B < 0 || Ld <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || prefix_len < 0 ||
       prefix_len > (int64_t(1) << 30) || !(scale > 0.f))
     return PSA_ERR_INVALID_ARG;
@@ -347,7 +346,34 @@ extern "C" int psa_verify_shared_fwd(const void* q_draft, const void* k_draft,
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + o_bytes);
   a.status = dev_status;
   a.stream = static_cast<cudaStream_t>(stream);
+  a.dmask = dmask;
   return launch_verify_shared(a);
+}
+
+extern "C" int psa_verify_shared_fwd(const void* q_draft, const void* k_draft,
+                                     const void* v_draft, const void* k_prefix,
+                                     const void* v_prefix, int64_t prefix_len, void* o,
+                                     float* lse, int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv,
+                                     int32_t head_dim, float scale, int32_t nsplit,
+                                     void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                     void* stream) {
+  return verify_shared_common(q_draft, k_draft, v_draft, k_prefix, v_prefix, prefix_len, o, lse,
+                              B, Ld, Hq, Hkv, head_dim, scale, nsplit, workspace, ws_bytes,
+                              dev_status, stream, nullptr);
+}
+
+extern "C" int psa_verify_shared_tree_fwd(const void* q_draft, const void* k_draft,
+                                          const void* v_draft, const void* k_prefix,
+                                          const void* v_prefix, int64_t prefix_len,
+                                          const uint8_t* dev_draft_mask, void* o, float* lse,
+                                          int32_t B, int32_t Ld, int32_t Hq, int32_t Hkv,
+                                          int32_t head_dim, float scale, int32_t nsplit,
+                                          void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                          void* stream) {
+  if (B > 0 && !dev_draft_mask) return PSA_ERR_INVALID_ARG;
+  return verify_shared_common(q_draft, k_draft, v_draft, k_prefix, v_prefix, prefix_len, o, lse,
+                              B, Ld, Hq, Hkv, head_dim, scale, nsplit, workspace, ws_bytes,
+                              dev_status, stream, dev_draft_mask);
 }
 
 // ------------------------------------------------------------------ backward

@@ -75,6 +75,7 @@ struct VerifySharedArgs {
   float* part_lse;        // [nsplit][B*Ld][Hq], log2 domain
   int32_t* status;
   cudaStream_t stream;
+  const uint8_t* dmask = nullptr;  // tree verify: [B*Ld, Ld] draft mask (device)
 };
 int launch_verify_shared(const VerifySharedArgs& a);
 

@@ -518,6 +518,7 @@ int launch_verify_shared(const VerifySharedArgs& a) {
   c.part_lse = a.part_lse;
   c.status = a.status;
   c.stream = a.stream;
+  c.dmask = a.dmask;
   return launch_verify_combine(c);
 }
 

@@ -82,3 +82,39 @@ def test_verify_shared_equals_per_request_verify():
     torch.cuda.synchronize()
     assert (o1.float() - o2.float()).abs().max().item() <= 1e-2
     assert (l1 - l2).abs().max().item() <= 1e-3
+
+
+def test_verify_shared_tree():
+    """Tree verify against the shared prefix ([SKV] can_handle: EAGLE trees
+    with topk > 1 bring a custom draft mask) against the oracle, with a draft
+    row that sees no other draft; the lower-triangular mask reproduces the
+    causal shared verify exactly."""
+    wl = W.SharedVerifyWorkload("t", B=5, L=777, Ld=6, Hq=32, Hkv=8, d=128, seed=61)
+    q, kd, vd, kp, vp = (t.cuda() for t in wl.make("cpu"))
+    rng = np.random.default_rng(62)
+    blocks = []
+    for _ in range(wl.B):
+        parent = [-1] + [int(rng.integers(-1, j)) for j in range(1, wl.Ld)]
+        m = np.zeros((wl.Ld, wl.Ld), dtype=np.uint8)
+        for j in range(wl.Ld):
+            a = j
+            while a >= 0:
+                m[j, a] = 1
+                a = parent[a]
+        blocks.append(m)
+    dm = np.concatenate(blocks)
+    dm[3] = 0                        # request 0, draft 3: only the prefix
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = psa.verify_shared(q, kd, vd, kp, vp, wl.scale, wl.Ld, nsplit=4, status=status,
+                               draft_mask=torch.from_numpy(dm).cuda())
+    torch.cuda.synchronize()
+    assert psa.read_status(status) == 0
+    ro, rl = oracle.verify_shared(q.cpu(), kd.cpu(), vd.cpu(), kp.cpu(), vp.cpu(), wl.Ld,
+                                  wl.scale, draft_mask=dm)
+    assert_parity(o, lse, ro, rl, "shared tree")
+    causal = torch.from_numpy(np.tile(np.tril(np.ones((wl.Ld, wl.Ld), np.uint8)), (wl.B, 1)))
+    o1, l1 = psa.verify_shared(q, kd, vd, kp, vp, wl.scale, wl.Ld, nsplit=4,
+                               draft_mask=causal.cuda())
+    o2, l2 = psa.verify_shared(q, kd, vd, kp, vp, wl.scale, wl.Ld, nsplit=4)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
