@@ -212,7 +212,20 @@ def test_prefill_and_sparse_host_validation():
 
 
 def test_python_binding_refuses_cpu_tensors():
+    """No CPU fallback: every compute entry of the binding refuses host
+    tensors before any library call."""
     import torch
     x = torch.zeros(4, 2, 64, dtype=torch.bfloat16)
+    i32 = torch.zeros(3, dtype=torch.int32)
     with pytest.raises(ValueError):
         psa.sparse_latent(x, x[:, 0], torch.zeros(4, 1, dtype=torch.int32), 0.1)
+    with pytest.raises(ValueError):
+        psa.verify(x, x, x, x, x, i32, 8, 0.1, 2)
+    with pytest.raises(ValueError):
+        psa.verify_tree(x, x, x, x, x, i32, 8, torch.ones(4, 2, dtype=torch.uint8), 0.1, 2)
+    with pytest.raises(ValueError):
+        psa.verify_extend(x, x, x, x, x, i32, 2, i32, 8, 0.1)
+    with pytest.raises(ValueError):
+        psa.verify_shared(x, x, x, x, x, 0.1, 2)
+    with pytest.raises(ValueError):
+        psa.verify_fp8(x, x, x, x, x, 1.0, 1.0, i32, 8, 0.1, 2)
