@@ -3,19 +3,23 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl psa|reference] [--no-extras]
 
-One JSON line on rank 0.  The headline workload is the GRPO rollout group
-(P=2048, N=8, S=512, 16/16 heads, d=128, bf16): metric = visible-block
-attention TFLOP/s (exact visible-pair FLOPs, 4*d*Hq*pairs) over the flat
-packed layout.  With extras on (default) the line also carries the
-speculative-verify prefix-KV GB/s, the large two-group prefill and the
-shared-latent sparse prefill, each device-timed the same way.
+One JSON line on rank 0.  The headline workload is the largest single-GPU
+prefill: two packed rollout groups of P=8192, N=16, S=1024 (32 query heads
+on 8 KV heads, d=128, bf16); metric = visible-block attention TFLOP/s
+(exact visible-pair FLOPs, 4*d*Hq*pairs) over the flat packed layout.  With
+extras on (default) the line also carries the GRPO group, the
+speculative-verify prefix-KV GB/s (bf16, e4m3, paged extend form), the
+shared-prefix verify, the GRPO backward and the shared-latent sparse
+prefill, each timed with the headline's steps and warm-up, each with its own
+end-to-end number and CPU-oracle baseline.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA
 events on the launching stream, with an L2 flush (a 256 MiB write) between
 steps outside the events; barrier + synchronize around the whole region;
 max over ranks.  N > 1 runs independent replicas (weak scaling): the path
 has no exchange step.  ``--impl reference`` times the fp64 CPU oracle on the
-host cores on a bounded sample of the same workload.
+host cores on a bounded sample of the same workload, on inputs built on the
+host (the GPU and the CUDA library are not touched).
 """
 from __future__ import annotations
 
@@ -148,16 +152,37 @@ def host_cores() -> int:
 # --------------------------------------------------------------------------- workloads
 
 class Runner:
-    """One workload: inputs resident on the device, one step = one call of
-    the public C-ABI entry point, algorithmic work per step."""
+    """One workload on the GPU: inputs resident on the device, one step = one
+    call of the public C-ABI entry point, algorithmic work per step.
+    ``inputs`` are the tensors an end-to-end step copies in from pinned host
+    memory, ``outputs`` the ones it reads back."""
     name = ""
     unit = ""
     kernels_per_step = 1
     bound = "tensor"
     kernel_file = ""
+    inputs: list = []
+    outputs: list = []
 
     def work(self) -> float: ...
     def step(self): ...
+
+    # end to end: host (pinned) inputs in, outputs back to the host
+    def e2e_setup(self):
+        self.h_in = [t.cpu().pin_memory() for t in self.inputs]
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outputs]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+
+    def e2e_step(self):
+        for d, h in zip(self.inputs, self.h_in):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        for h, d in zip(self.h_out, self.outputs):
+            h.copy_(d, non_blocking=True)
+
+    def e2e_release(self):
+        self.h_in, self.h_out = [], []
 
 
 class PrefillRunner(Runner):
@@ -177,6 +202,7 @@ class PrefillRunner(Runner):
                                                  wl.Hq, wl.Hkv, wl.d)
         self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
         self.kernels_per_step = 1 if wl.dtype == torch.bfloat16 else 4
+        self.inputs, self.outputs = [self.q, self.k, self.v], [self.o, self.lse]
 
     def work(self):
         return self.wl.flops()
@@ -184,57 +210,6 @@ class PrefillRunner(Runner):
     def step(self):
         self.psa.prefill(self.q, self.k, self.v, self.sched, self.wl.scale, out=self.o,
                          lse=self.lse, workspace=self.ws)
-
-    # end to end: host (pinned) inputs in, O and LSE back to the host
-    def e2e_setup(self):
-        self.hq, self.hk, self.hv = (t.cpu().pin_memory() for t in (self.q, self.k, self.v))
-        self.ho = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
-        self.hl = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
-        self.h2d = sum(t.numel() * t.element_size() for t in (self.hq, self.hk, self.hv))
-        self.d2h = self.ho.numel() * self.ho.element_size() + self.hl.numel() * 4
-
-    def e2e_step(self):
-        self.q.copy_(self.hq, non_blocking=True)
-        self.k.copy_(self.hk, non_blocking=True)
-        self.v.copy_(self.hv, non_blocking=True)
-        self.step()
-        self.ho.copy_(self.o, non_blocking=True)
-        self.hl.copy_(self.lse, non_blocking=True)
-
-    def oracle_sample(self, budget_s: float):
-        """(work done, seconds) of the oracle on a bounded row sample."""
-        import oracle
-        wl = self.wl
-        q, k, v = (t.cpu() for t in (self.q, self.k, self.v))
-        vis_per_row = None
-        rows = []
-        # rows spread over every segment, the last rows of each group first
-        # (the longest ones), grown until the budget is used
-        g = torch.Generator().manual_seed(0)
-        perm = torch.randperm(wl.T, generator=g).tolist()
-        t0 = time.perf_counter()
-        done_flops = 0.0
-        segs = wl.segments()
-        start, lens, parent = oracle.segment_arrays(segs)
-        seg_of = {}
-        for s_i, (a, n) in enumerate(zip(start, lens)):
-            for t in range(a, a + n):
-                seg_of[t] = s_i
-        chunk = 8
-        i = 0
-        while time.perf_counter() - t0 < budget_s and i < len(perm):
-            rows = perm[i:i + chunk]
-            i += chunk
-            oracle.prefill(q, k, v, segs, wl.scale, rows=rows)
-            for r in rows:
-                s_i = seg_of[r]
-                cnt = r - int(start[s_i]) + 1
-                p = int(parent[s_i])
-                while p >= 0:
-                    cnt += int(lens[p])
-                    p = int(parent[p])
-                done_flops += 4.0 * wl.d * wl.Hq * cnt
-        return done_flops, time.perf_counter() - t0, f"{i} random query rows x {wl.Hq} heads"
 
 
 class VerifyRunner(Runner):
@@ -253,6 +228,8 @@ class VerifyRunner(Runner):
         self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=dev)
         n = psa.verify_workspace_size(wl.B, wl.Ld, wl.Hq, wl.d, wl.nsplit)
         self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.inputs = [self.q, self.kd, self.vd, self.kc, self.vc]
+        self.outputs = [self.o, self.lse]
 
     def work(self):
         return float(self.wl.prefix_kv_bytes())
@@ -261,40 +238,6 @@ class VerifyRunner(Runner):
         wl = self.wl
         self.psa.verify(self.q, self.kd, self.vd, self.kc, self.vc, self.indptr, wl.L, wl.scale,
                         wl.Ld, nsplit=wl.nsplit, out=self.o, lse=self.lse, workspace=self.ws)
-
-    def e2e_setup(self):
-        ts = (self.q, self.kd, self.vd, self.kc, self.vc)
-        self.hin = [t.cpu().pin_memory() for t in ts]
-        self.ho = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
-        self.hl = torch.empty(self.lse.shape, dtype=torch.float32).pin_memory()
-        self.h2d = sum(t.numel() * t.element_size() for t in self.hin)
-        self.d2h = self.ho.numel() * self.ho.element_size() + self.hl.numel() * 4
-
-    def e2e_step(self):
-        for d, h in zip((self.q, self.kd, self.vd, self.kc, self.vc), self.hin):
-            d.copy_(h, non_blocking=True)
-        self.step()
-        self.ho.copy_(self.o, non_blocking=True)
-        self.hl.copy_(self.lse, non_blocking=True)
-
-    def oracle_sample(self, budget_s: float):
-        import numpy as np
-        import oracle
-        wl = self.wl
-        t0 = time.perf_counter()
-        done, n = 0.0, 0
-        per_row_bytes = wl.L * wl.Hkv * wl.d * 2 * 2 / wl.Ld  # prefix bytes per draft row
-        b = 0
-        while time.perf_counter() - t0 < budget_s and b < wl.B:
-            p0, p1 = b * wl.L, (b + 1) * wl.L
-            sl = slice(b * wl.Ld, (b + 1) * wl.Ld)
-            oracle.verify(self.q[sl].cpu(), self.kd[sl].cpu(), self.vd[sl].cpu(),
-                          self.kc[p0:p1].cpu(), self.vc[p0:p1].cpu(),
-                          np.array([0, wl.L], dtype=np.int64), wl.Ld, wl.scale)
-            done += per_row_bytes * wl.Ld
-            n += 1
-            b += 1
-        return done, time.perf_counter() - t0, f"{n} whole requests ({n * wl.Ld} draft rows)"
 
 
 class SparseRunner(Runner):
@@ -309,6 +252,7 @@ class SparseRunner(Runner):
         self.q, self.lat, self.idx = wl.make(dev)
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty((wl.T, wl.H), dtype=torch.float32, device=dev)
+        self.inputs, self.outputs = [self.q, self.lat, self.idx], [self.o, self.lse]
 
     def work(self):
         return self.wl.flops()
@@ -329,7 +273,7 @@ class BackwardRunner(Runner):
     def __init__(self, wl: W.PrefillWorkload, dev):
         import shared_prefix_attention_b200 as psa
         self.psa, self.wl, self.dev = psa, wl, dev
-        self.name = wl.name.replace("grpo", "grpo-backward", 1)
+        self.name = backward_name(wl)
         self.q, self.k, self.v = wl.make(dev)
         g = torch.Generator(device=dev)
         g.manual_seed(wl.seed + 100)
@@ -340,10 +284,11 @@ class BackwardRunner(Runner):
         self.dq, self.dk, self.dv = (torch.empty_like(t) for t in (self.q, self.k, self.v))
         n = int(psa.lib().psa_prefill_bwd_workspace_size(wl.T, wl.Hq))
         self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.inputs = [self.q, self.k, self.v, self.o, self.lse, self.dout]
+        self.outputs = [self.dq, self.dk, self.dv]
 
     def work(self):
-        # five products of the visible pairs (S, dP, dV, dQ, dK), 2 d FLOP each
-        return self.wl.flops() * 10.0 / 4.0
+        return backward_flops(self.wl)
 
     def step(self):
         self.psa.prefill_bwd(self.q, self.k, self.v, self.o, self.lse, self.dout, self.scheds,
@@ -369,6 +314,8 @@ class VerifyFp8Runner(Runner):
         self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=dev)
         n = psa.verify_workspace_size(wl.B, wl.Ld, wl.Hq, wl.d, wl.nsplit)
         self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.inputs = [self.q, self.kd, self.vd, self.kc8, self.vc8]
+        self.outputs = [self.o, self.lse]
 
     def work(self):
         return float(self.wl.prefix_fp8_bytes())
@@ -398,6 +345,8 @@ class SharedVerifyRunner(Runner):
         self.ns = wl.nsplit or psa.verify_shared_auto_splits(wl.B, wl.Ld, wl.Hq, wl.Hkv, wl.L)
         n = psa.verify_workspace_size(wl.B, wl.Ld, wl.Hq, wl.d, self.ns)
         self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.inputs = [self.q, self.kd, self.vd, self.kp, self.vp]
+        self.outputs = [self.o, self.lse]
 
     def work(self):
         return self.wl.flops()
@@ -410,7 +359,7 @@ class SharedVerifyRunner(Runner):
 
 class ExtendVerifyRunner(Runner):
     """Verify in the extend form: ragged drafts in trees, each prefix read
-    through a token-granular page table (gathered with 16-byte copies)."""
+    through a token-granular page table (gathered with bulk copies)."""
     unit = "GB/s"
     bound = "hbm"
     kernels_per_step = 2
@@ -430,6 +379,9 @@ class ExtendVerifyRunner(Runner):
         self.lse = torch.empty(self.q.shape[:2], dtype=torch.float32, device=dev)
         n = psa.verify_workspace_size(1, wl.n_rows, wl.Hq, wl.d, wl.nsplit)
         self.ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.inputs = [self.q, self.kd, self.vd, self.kp, self.vp, self.idx] + (
+            [] if self.mask is None else [self.mask])
+        self.outputs = [self.o, self.lse]
 
     def work(self):
         return float(self.wl.prefix_kv_bytes())
@@ -442,27 +394,14 @@ class ExtendVerifyRunner(Runner):
                                mask_indptr=None if self.mask is None else self.mi,
                                nsplit=wl.nsplit, out=self.o, lse=self.lse, workspace=self.ws)
 
-    def oracle_sample(self, budget_s: float):
-        import numpy as np
-        import oracle
-        wl = self.wl
-        qo, kvp = wl.qo_indptr(), wl.kv_indptr()
-        host = [t.cpu() for t in (self.q, self.kd, self.vd, self.kp, self.vp, self.idx)]
-        mask = None if self.mask is None else self.mask.cpu()
-        t0 = time.perf_counter()
-        done, n, b = 0.0, 0, 0
-        per_tok = wl.Hkv * wl.d * 2 * 2  # prefix K and V bytes per token
-        while time.perf_counter() - t0 < budget_s and b < wl.B:
-            rows = np.arange(qo[b], qo[b + 1], dtype=np.int32)
-            if len(rows):
-                oracle.verify_extend(*host[:5], qo, kvp, wl.scale, kv_indices=host[5],
-                                     draft_mask=mask,
-                                     mask_indptr=None if mask is None else wl.mask_indptr(),
-                                     rows=rows)
-            done += per_tok * wl.prefix_lens[b]
-            n += 1
-            b += 1
-        return done, time.perf_counter() - t0, f"{n} whole requests"
+
+def backward_name(wl: W.PrefillWorkload) -> str:
+    return wl.name.replace("grpo", "grpo-backward", 1)
+
+
+def backward_flops(wl: W.PrefillWorkload) -> float:
+    """Five products of the visible pairs (S, dP, dV, dQ, dK), 2 d FLOP each."""
+    return wl.flops() * 10.0 / 4.0
 
 
 VERIFY_SMALL = W.VerifyWorkload("verify B=8 L=16384 drafts=4 H=32/8 d=128 splits=32 bf16", B=8,
@@ -476,22 +415,344 @@ VERIFY_PAGED_SMALL = W.ExtendVerifyWorkload(
     nsplit=32, seed=8)
 SPARSE_SMALL = W.SparseLatentWorkload("sparse T=4096 H=64 dl=512 topk=2048 bf16", T=4096, H=64,
                                       dl=512, topk=2048, seed=5)
+VERIFY_SHARED_SMALL = W.SharedVerifyWorkload(
+    "verify-shared B=8 L=16384 drafts=4 H=32/8 d=128 bf16", B=8, L=16384, Ld=4, Hq=32, Hkv=8,
+    d=128, seed=6)
+
+# name -> (runner class, workload)
+WORKLOADS = {
+    "tiny": (PrefillRunner, W.TINY),
+    "grpo": (PrefillRunner, W.GRPO),
+    "large": (PrefillRunner, W.LARGE),
+    "verify": (VerifyRunner, W.VERIFY),
+    "verify8": (VerifyRunner, VERIFY_SMALL),
+    "verify-shared": (SharedVerifyRunner, W.VERIFY_SHARED),
+    "verify-shared8": (SharedVerifyRunner, VERIFY_SHARED_SMALL),
+    "verify-fp8": (VerifyFp8Runner, W.VERIFY_FP8),
+    "verify-fp8-8": (VerifyFp8Runner, VERIFY_FP8_SMALL),
+    "verify-extend": (ExtendVerifyRunner, W.VERIFY_PAGED),
+    "verify-extend8": (ExtendVerifyRunner, VERIFY_PAGED_SMALL),
+    "grpo-backward": (BackwardRunner, W.GRPO),
+    "sparse": (SparseRunner, W.SPARSE),
+    "sparse4k": (SparseRunner, SPARSE_SMALL),
+}
+
+# the headline is the largest single-GPU prefill workload; every other
+# workload of the metric rides along as an extra, timed the same way
+HEADLINE = "large"
+EXTRAS = ("grpo", "verify", "verify-fp8", "verify-extend", "verify-shared", "grpo-backward",
+          "sparse")
 
 
 def make_runner(name: str, dev):
-    return {"grpo": lambda: PrefillRunner(W.GRPO, dev),
-            "verify8": lambda: VerifyRunner(VERIFY_SMALL, dev),
-            "sparse4k": lambda: SparseRunner(SPARSE_SMALL, dev),
-            "tiny": lambda: PrefillRunner(W.TINY, dev),
-            "large": lambda: PrefillRunner(W.LARGE, dev),
-            "verify": lambda: VerifyRunner(W.VERIFY, dev),
-            "verify-shared": lambda: SharedVerifyRunner(W.VERIFY_SHARED, dev),
-            "verify-fp8": lambda: VerifyFp8Runner(W.VERIFY_FP8, dev),
-            "verify-fp8-8": lambda: VerifyFp8Runner(VERIFY_FP8_SMALL, dev),
-            "verify-extend": lambda: ExtendVerifyRunner(W.VERIFY_PAGED, dev),
-            "verify-extend8": lambda: ExtendVerifyRunner(VERIFY_PAGED_SMALL, dev),
-            "grpo-backward": lambda: BackwardRunner(W.GRPO, dev),
-            "sparse": lambda: SparseRunner(W.SPARSE, dev)}[name]()
+    cls, wl = WORKLOADS[name]
+    return cls(wl, dev)
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+class OracleSampler:
+    """The fp64 oracle, as it stands, on a bounded sample of one workload.
+
+    Inputs are built on the host from the workload's recipe (same shapes and
+    distributions as the GPU's; nothing here touches the GPU or the CUDA
+    library).  ``run(budget)`` returns (work done in the metric's unit
+    numerator, seconds, description); ``full_work()`` is the whole
+    workload's work, so the full-config CPU time is extrapolated as
+    full_work / (work / seconds)."""
+    unit = ""
+    threads = 0      # host threads the oracle calls use (0: every core)
+
+    def run(self, budget_s: float): ...
+    def full_work(self) -> float: ...
+
+
+def _visible_keys_per_row(segments) -> "np.ndarray":
+    """Keys each flat row sees: its own segment up to itself plus every
+    ancestor segment in full (the flat layout's visibility)."""
+    import numpy as np
+    lens = [n for n, _ in segments]
+    start = np.cumsum([0] + lens[:-1])
+    anc = []
+    for i, (_, p) in enumerate(segments):
+        a = 0
+        while p >= 0:
+            a += lens[p]
+            p = segments[p][1]
+        anc.append(a)
+    out = np.zeros(sum(lens), dtype=np.int64)
+    for s, (n, _) in enumerate(segments):
+        out[start[s]:start[s] + n] = anc[s] + np.arange(1, n + 1)
+    return out
+
+
+class PrefillSampler(OracleSampler):
+    unit = "TFLOP/s"
+
+    def __init__(self, wl: W.PrefillWorkload):
+        import numpy as np
+        self.wl = wl
+        q, k, v = wl.make("cpu")
+        self.q, self.k, self.v = (np.ascontiguousarray(t.float().numpy()) for t in (q, k, v))
+        self.vis = _visible_keys_per_row(wl.segments())
+        self.perm = torch.randperm(wl.T, generator=torch.Generator().manual_seed(0)).numpy()
+        self.pos = 0
+
+    def full_work(self):
+        return self.wl.flops()
+
+    def run(self, budget_s):
+        import numpy as np
+        import oracle
+        wl = self.wl
+        chunk = 4 * oracle.default_threads()
+        t0 = time.perf_counter()
+        done, n = 0.0, 0
+        while time.perf_counter() - t0 < budget_s:
+            rows = self.perm[np.arange(self.pos, self.pos + chunk) % wl.T].astype(np.int32)
+            self.pos += chunk
+            oracle.prefill(self.q, self.k, self.v, wl.segments(), wl.scale, rows=rows)
+            done += 4.0 * wl.d * wl.Hq * float(self.vis[rows].sum())
+            n += chunk
+        return done, time.perf_counter() - t0, f"{n} random query rows x {wl.Hq} heads"
+
+
+class BackwardSampler(OracleSampler):
+    """Whole heads of the backward: a KV head with its query heads over all
+    T rows (the oracle's full backward on that head slice)."""
+    unit = "TFLOP/s"
+
+    def __init__(self, wl: W.PrefillWorkload):
+        self.wl = wl
+        q, k, v = wl.make("cpu")
+        g = torch.Generator().manual_seed(wl.seed + 100)
+        do = (torch.randn(q.shape, generator=g) * wl.sigma).to(q.dtype)
+        self.t = (q, k, v, do)
+        self.h = 0
+
+    def full_work(self):
+        return backward_flops(self.wl)
+
+    def run(self, budget_s):
+        import oracle
+        wl = self.wl
+        G = wl.Hq // wl.Hkv
+        q, k, v, do = self.t
+        t0 = time.perf_counter()
+        done, n = 0.0, 0
+        while n == 0 or time.perf_counter() - t0 < budget_s:
+            h = self.h % wl.Hkv
+            self.h += 1
+            qs, dos = (x[:, h * G:(h + 1) * G].contiguous() for x in (q, do))
+            ks, vs = (x[:, h:h + 1].contiguous() for x in (k, v))
+            oracle.prefill_bwd(qs, ks, vs, dos, wl.segments(), wl.scale)
+            done += backward_flops(wl) / wl.Hkv
+            n += 1
+        return done, time.perf_counter() - t0, (
+            f"{n} whole KV head(s) ({G} query head(s) each) over all {wl.T} rows")
+
+
+class VerifySampler(OracleSampler):
+    """Whole requests: each sampled request's drafts against its own prefix,
+    its inputs drawn on the host from the workload's recipe.  Enough
+    requests go to one oracle call to give every host thread a draft row."""
+    unit = "GB/s"
+
+    def __init__(self, wl: W.VerifyWorkload, fp8: bool = False):
+        import oracle
+        self.wl, self.fp8 = wl, fp8
+        self.b = 0
+        self.per_call = max(1, oracle.default_threads() // wl.Ld)
+        self.threads = min(oracle.default_threads(), self.per_call * wl.Ld)
+
+    def _bytes(self, ntok):
+        wl = self.wl
+        return ntok * wl.Hkv * wl.d * 2 * (1 if self.fp8 else 2)
+
+    def full_work(self):
+        return float(self.wl.prefix_fp8_bytes() if self.fp8 else self.wl.prefix_kv_bytes())
+
+    def run(self, budget_s):
+        import numpy as np
+        import oracle
+        wl = self.wl
+        t_wall = 0.0
+        done, n = 0.0, 0
+        while n == 0 or t_wall < budget_s:
+            bs = [(self.b + i) % wl.B for i in range(self.per_call)]
+            self.b += self.per_call
+            lens = [wl.lens()[b] for b in bs]
+            part = W.VerifyWorkload("part", B=len(bs), L=0, Ld=wl.Ld, Hq=wl.Hq, Hkv=wl.Hkv,
+                                    d=wl.d, nsplit=1, prefix_lens=lens,
+                                    seed=wl.seed * 1000 + bs[0])
+            ind = np.array(part.kv_indptr(), dtype=np.int64)
+            if self.fp8:
+                q, kd, vd, kc, vc = part.make_fp8("cpu")
+                t0 = time.perf_counter()
+                oracle.verify_fp8(q, kd, vd, kc, vc, wl.k_scale, wl.v_scale, ind, wl.Ld,
+                                  wl.scale)
+            else:
+                q, kd, vd, kc, vc = part.make("cpu")
+                t0 = time.perf_counter()
+                oracle.verify(q, kd, vd, kc, vc, ind, wl.Ld, wl.scale)
+            t_wall += time.perf_counter() - t0
+            done += self._bytes(sum(lens))
+            n += len(bs)
+        return done, t_wall, f"{n} whole requests ({n * wl.Ld} draft rows)"
+
+
+class ExtendSampler(OracleSampler):
+    """Whole requests of the extend form, batched per oracle call until every
+    host thread has a draft row."""
+    unit = "GB/s"
+
+    def __init__(self, wl: W.ExtendVerifyWorkload):
+        import oracle
+        self.wl = wl
+        self.b = 0
+        self.threads = oracle.default_threads()
+
+    def full_work(self):
+        return float(self.wl.prefix_kv_bytes())
+
+    def run(self, budget_s):
+        import oracle
+        wl = self.wl
+        t_wall = 0.0
+        done, n = 0.0, 0
+        while n == 0 or t_wall < budget_s:
+            bs = []
+            while sum(wl.draft_lens[b] for b in bs) < self.threads and len(bs) < wl.B:
+                bs.append(self.b % wl.B)
+                self.b += 1
+            part = W.ExtendVerifyWorkload(
+                "part", draft_lens=[wl.draft_lens[b] for b in bs],
+                prefix_lens=[wl.prefix_lens[b] for b in bs], Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d,
+                nsplit=1, tree=wl.tree, pool_slack=wl.pool_slack, seed=wl.seed * 1000 + bs[0])
+            q, kd, vd, kp, vp, idx, mask = part.make("cpu")
+            t0 = time.perf_counter()
+            oracle.verify_extend(q, kd, vd, kp, vp, part.qo_indptr(), part.kv_indptr(), wl.scale,
+                                 kv_indices=idx, draft_mask=mask,
+                                 mask_indptr=None if mask is None else part.mask_indptr())
+            t_wall += time.perf_counter() - t0
+            done += float(part.prefix_kv_bytes())
+            n += len(bs)
+        return done, t_wall, f"{n} whole requests"
+
+
+class SharedVerifySampler(OracleSampler):
+    """Whole requests against the whole shared prefix, enough per oracle call
+    to give every host thread a draft row."""
+    unit = "TFLOP/s"
+
+    def __init__(self, wl: W.SharedVerifyWorkload):
+        import oracle
+        self.wl = wl
+        self.b = 0
+        self.per_call = max(1, oracle.default_threads() // wl.Ld)
+        self.threads = min(oracle.default_threads(), self.per_call * wl.Ld)
+
+    def full_work(self):
+        return self.wl.flops()
+
+    def run(self, budget_s):
+        import oracle
+        wl = self.wl
+        t_wall = 0.0
+        done, n = 0.0, 0
+        while n == 0 or t_wall < budget_s:
+            part = W.SharedVerifyWorkload("part", B=self.per_call, L=wl.L, Ld=wl.Ld, Hq=wl.Hq,
+                                          Hkv=wl.Hkv, d=wl.d, seed=wl.seed * 1000 + self.b)
+            self.b += self.per_call
+            q, kd, vd, kp, vp = part.make("cpu")
+            t0 = time.perf_counter()
+            oracle.verify_shared(q, kd, vd, kp, vp, wl.Ld, wl.scale)
+            t_wall += time.perf_counter() - t0
+            done += part.flops()
+            n += self.per_call
+        return done, t_wall, f"{n} whole requests ({n * wl.Ld} draft rows)"
+
+
+class SparseSampler(OracleSampler):
+    """Random query rows: the full latent, and for each sampled row its own
+    Q and index list drawn on the host from the workload's recipe."""
+    unit = "TFLOP/s"
+
+    def __init__(self, wl: W.SparseLatentWorkload):
+        self.wl = wl
+        self.g = torch.Generator().manual_seed(wl.seed)
+        self.lat = (torch.randn((wl.T, wl.dl), generator=self.g) * wl.sigma).to(wl.dtype)
+
+    def full_work(self):
+        return self.wl.flops()
+
+    def _rows(self, rows):
+        wl = self.wl
+        idx = torch.full((len(rows), wl.topk), -1, dtype=torch.int32)
+        for i, t in enumerate(rows):
+            if t < wl.topk:
+                idx[i, :t + 1] = torch.arange(t + 1, dtype=torch.int32)
+            else:
+                idx[i] = torch.sort(torch.randperm(t + 1, generator=self.g)[:wl.topk]).values
+        q = (torch.randn((len(rows), wl.H, wl.dl), generator=self.g) * wl.sigma).to(wl.dtype)
+        return q, idx
+
+    def run(self, budget_s):
+        import oracle
+        wl = self.wl
+        chunk = 2 * oracle.default_threads()
+        t_wall = 0.0
+        done, n = 0.0, 0
+        while n == 0 or t_wall < budget_s:
+            rows = torch.randint(0, wl.T, (chunk,), generator=self.g).tolist()
+            q, idx = self._rows(rows)
+            t0 = time.perf_counter()
+            oracle.sparse_latent(q, self.lat, idx, wl.scale)
+            t_wall += time.perf_counter() - t0
+            done += 4.0 * wl.dl * wl.H * sum(min(t + 1, wl.topk) for t in rows)
+            n += chunk
+        return done, t_wall, f"{n} random query rows x {wl.H} heads"
+
+
+def default_oracle_threads() -> int:
+    import oracle
+    return oracle.default_threads()
+
+
+def make_sampler(name: str) -> OracleSampler:
+    cls, wl = WORKLOADS[name]
+    if cls is PrefillRunner:
+        return PrefillSampler(wl)
+    if cls is BackwardRunner:
+        return BackwardSampler(wl)
+    if cls is VerifyRunner:
+        return VerifySampler(wl)
+    if cls is VerifyFp8Runner:
+        return VerifySampler(wl, fp8=True)
+    if cls is ExtendVerifyRunner:
+        return ExtendSampler(wl)
+    if cls is SharedVerifyRunner:
+        return SharedVerifySampler(wl)
+    return SparseSampler(wl)
+
+
+def workload_label(name: str) -> str:
+    cls, wl = WORKLOADS[name]
+    return backward_name(wl) if cls is BackwardRunner else wl.name
+
+
+def cpu_baseline(name: str, budget_s: float) -> dict:
+    """The oracle's rate on a bounded sample of ``name``, with the whole
+    workload's CPU time extrapolated from it (labelled as such)."""
+    sampler = make_sampler(name)
+    done, secs, sample = sampler.run(budget_s)
+    scale = 1e12 if sampler.unit == "TFLOP/s" else 1e9
+    rate = done / secs
+    return {"value": rate / scale, "unit": sampler.unit,
+            "cores": sampler.threads or min(host_cores(), default_oracle_threads()),
+            "kind": "oracle", "sample": f"{sample}, {secs:.1f} s",
+            "full_config_s": round(sampler.full_work() / rate, 1),
+            "full_config_s_is": "extrapolated (sampled rate x whole-workload work)"}
 
 
 # --------------------------------------------------------------------------- timing
@@ -561,22 +822,35 @@ def measure(runner, steps, warmup, flush, dist_on, world, peaks):
 
 # --------------------------------------------------------------------------- main
 
+def e2e_measure(runner, steps, warmup, flush, dist_on, world):
+    """The same call with the inputs copied in from pinned host memory and
+    the outputs read back inside the timed region."""
+    runner.e2e_setup()
+    per = time_steps(runner.e2e_step, steps, warmup, flush, dist_on)
+    ems = max_over_ranks(sum(per) / len(per), dist_on)
+    out = {"value": round(job_throughput(world, runner.work(), ems, runner.unit), 3),
+           "unit": runner.unit, "ms_per_step": round(ems, 4),
+           "h2d_bytes_per_step": runner.h2d, "d2h_bytes_per_step": runner.d2h}
+    runner.e2e_release()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="grpo",
-                    choices=["grpo", "tiny", "large", "verify", "verify8", "verify-shared",
-                             "verify-fp8", "verify-fp8-8", "verify-extend", "verify-extend8",
-                             "grpo-backward",
-                             "sparse",
-                             "sparse4k"])
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="psa", choices=["psa", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0,
-                    help="seconds of oracle work for the CPU baseline")
+                    help="seconds of oracle work for the headline's CPU baseline")
+    ap.add_argument("--extra-cpu-budget", type=float, default=4.0,
+                    help="seconds of oracle work for each extra's CPU baseline")
+    ap.add_argument("--ref-step-s", type=float, default=0.0,
+                    help="--impl reference: seconds of oracle work per step (0: spread "
+                         "about a minute over warm-up and timed steps)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -596,6 +870,7 @@ def main():
     dev = torch.device("cuda", local)
     peaks = load_peaks()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    do_cpu = rank == 0 and world == 1
 
     runner = make_runner(args.workload, dev)
     with ClockSampler(local) as clk:
@@ -612,36 +887,37 @@ def main():
            "roofline": roof, "clocks": clocks,
            "gpu_launches": runner.kernels_per_step * args.steps}
 
-    if not args.no_e2e and hasattr(runner, "e2e_setup"):
-        runner.e2e_setup()
-        per = time_steps(runner.e2e_step, max(3, min(args.steps, 10)), 2, flush, dist_on)
-        ems = max_over_ranks(sum(per) / len(per), dist_on)
-        out["e2e"] = {"value": round(job_throughput(world, runner.work(), ems, runner.unit), 3),
-                      "unit": runner.unit, "ms_per_step": round(ems, 4),
-                      "h2d_bytes_per_step": runner.h2d, "d2h_bytes_per_step": runner.d2h}
+    if not args.no_e2e:
+        out["e2e"] = e2e_measure(runner, args.steps, args.warmup, flush, dist_on, world)
+    del runner
+    torch.cuda.empty_cache()
 
-    if not args.no_extras and args.workload == "grpo":
+    if not args.no_extras and args.workload == HEADLINE:
         extras = {}
-        for name in ("verify", "verify-fp8", "verify-extend", "verify-shared", "large",
-                     "grpo-backward", "sparse"):
+        for name in EXTRAS:
             try:
                 r = make_runner(name, dev)
-                v, m, rf = measure(r, max(3, min(args.steps, 10)), 3, flush, dist_on, world,
-                                   peaks)
-                extras[name] = {"workload": r.name, "value": round(v, 3), "unit": r.unit,
-                                "ms_per_step": round(m, 4), "roofline": rf}
+                with ClockSampler(local) as eclk:
+                    v, m, rf = measure(r, args.steps, args.warmup, flush, dist_on, world, peaks)
+                ex = {"workload": r.name, "value": round(v, 3), "unit": r.unit,
+                      "ms_per_step": round(m, 4), "steps": args.steps, "warmup": args.warmup,
+                      "roofline": rf, "clocks": eclk.summary(),
+                      "gpu_launches": r.kernels_per_step * args.steps}
+                if not args.no_e2e:
+                    ex["e2e"] = e2e_measure(r, args.steps, args.warmup, flush, dist_on, world)
                 del r
             except Exception as e:  # a kernel that is not built yet
-                extras[name] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+                ex = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
             torch.cuda.empty_cache()
+            extras[name] = ex
+        if do_cpu and args.extra_cpu_budget > 0:
+            for name, ex in extras.items():
+                if "unavailable" not in ex:
+                    ex["cpu_baseline"] = cpu_baseline(name, args.extra_cpu_budget)
         out["extras"] = extras
 
-    if rank == 0 and world == 1 and args.cpu_budget > 0:
-        done, secs, sample = runner.oracle_sample(args.cpu_budget)
-        scale = 1e12 if runner.unit == "TFLOP/s" else 1e9
-        out["cpu_baseline"] = {"value": done / secs / scale, "unit": runner.unit,
-                               "cores": host_cores(), "kind": "oracle",
-                               "sample": f"{sample}, {secs:.1f} s"}
+    if do_cpu and args.cpu_budget > 0:
+        out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_budget)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist_on:
@@ -651,31 +927,35 @@ def main():
 
 def run_reference(args, world, rank):
     """The oracle, as it stands, on the host cores: each step is a bounded
-    sample of the same workload (rank 0 only)."""
+    sample of the same workload (rank 0 only).  Inputs are built on the host;
+    neither the GPU nor the CUDA library is touched."""
     if rank != 0:
         return
-    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
-    runner = make_runner(args.workload, dev)
-    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    sampler = make_sampler(args.workload)
+    per_step = args.ref_step_s or max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        runner.oracle_sample(per_step / 4)
+        sampler.run(per_step / 4)
     done_t, secs_t, sample = 0.0, 0.0, ""
     for _ in range(args.steps):
-        d, s, sample = runner.oracle_sample(per_step)
+        d, s, sample = sampler.run(per_step)
         done_t += d
         secs_t += s
-    scale = 1e12 if runner.unit == "TFLOP/s" else 1e9
+    scale = 1e12 if sampler.unit == "TFLOP/s" else 1e9
     value = done_t / secs_t / scale
-    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": runner.unit,
+    cores = sampler.threads or min(host_cores(), default_oracle_threads())
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": sampler.unit,
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": 1e3 * secs_t / args.steps, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic (seeded N(0,1)*sigma; no dataset)",
-           "config": {"workload": runner.name, "l2": "n/a (CPU)",
+           "config": {"workload": workload_label(args.workload), "l2": "n/a (CPU)",
                       "parallelism": "host cores"},
-           "cpu_baseline": {"value": value, "unit": runner.unit, "cores": host_cores(),
-                            "kind": "oracle", "sample": f"per step: {sample}"},
-           "e2e": {"value": value, "unit": runner.unit, "h2d_bytes_per_step": 0,
+           "cpu_baseline": {"value": value, "unit": sampler.unit, "cores": cores,
+                            "kind": "oracle", "sample": f"per step: {sample}",
+                            "full_config_s": round(sampler.full_work() / (done_t / secs_t), 1),
+                            "full_config_s_is": "extrapolated (sampled rate x whole-workload "
+                                                "work)"},
+           "e2e": {"value": value, "unit": sampler.unit, "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 

@@ -357,9 +357,12 @@ int psa_verify_extend_fwd(const void *q_draft, const void *k_draft, const void *
  *     psa_verify_workspace_size(B, Ld, Hq, head_dim, nsplit) exceeds it
  *     (nsplit == 0 is resolved with psa_verify_auto_splits first).
  *   - Allocates and frees nothing, directly or through any library.
- *   - The first call on each device looks up the array's device address with
- *     that device current (cudaGetSymbolAddress) and caches it; make that
- *     first call before any stream capture on the device.
+ *   - Every call looks up the array's device address in the context that is
+ *     current for the call (cudaGetSymbolAddress; no allocation), so a caller
+ *     that switches contexts on a device, or rebuilds its context after a
+ *     device reset, still gets the array of the context it calls from.  The
+ *     first call in a context also loads the library's module there; make it
+ *     before any stream capture in that context.
  *   - Every call on a device shares the one array, which keeps whatever the
  *     last call left there.  Nothing in it needs to start at zero (stage 1
  *     writes every partial that stage 2 reads).  Calls whose GPU work

@@ -77,7 +77,7 @@ def load(path: str | None = None):
     lib.oracle_verify_fp8_paged.argtypes = [P, P, P, P, P, D, D, P, P, I, I, I, I, I, D, P, I,
                                             P, P, I]
     lib.oracle_decode_e4m3.argtypes = [P, P, ctypes.c_int64]
-    lib.oracle_sparse_latent.argtypes = [P, P, P, I, I, I, I, D, P, I, P, P, I]
+    lib.oracle_sparse_latent.argtypes = [P, P, P, I, I, I, I, I, D, P, I, P, P, I]
     lib.oracle_visibility.argtypes = [P, P, P, I, I, I, I, P]
     for f in (lib.oracle_prefill, lib.oracle_prefill_bwd, lib.oracle_prefill_bwd_dq,
               lib.oracle_verify, lib.oracle_verify_tree, lib.oracle_verify_extend,
@@ -356,16 +356,23 @@ def verify_fp8(q_draft, k_draft, v_draft, k_cache8, v_cache8, k_scale: float, v_
 def sparse_latent(q, latent, idx, scale: float, rows=None, nthreads: int | None = None,
                   lib=None):
     """O [nrows, H, dl] and LSE [nrows, H]; q [T, H, dl], latent [Tk, dl],
-    idx [T, topk] int32 with -1 padding."""
+    idx [T, topk] int32 with -1 padding.  An index outside [-1, Tk) names no
+    latent row: ValueError, before anything is read through it."""
     lib = lib or load()
     q, lat, idx = _f32(q), _f32(latent), _i32(idx)
     T, H, dl = q.shape
+    Tk = lat.shape[0]
+    if lat.shape[1] != dl or idx.shape[0] != T:
+        raise ValueError("sparse_latent: latent [Tk, dl] and idx [T, topk] must match q")
     topk = idx.shape[1]
     rows = np.arange(T, dtype=np.int32) if rows is None else _i32(rows)
     o = np.zeros((len(rows), H, dl), dtype=np.float64)
     lse = np.zeros((len(rows), H), dtype=np.float64)
-    rc = lib.oracle_sparse_latent(_ptr(q), _ptr(lat), _ptr(idx), T, H, dl, topk,
+    rc = lib.oracle_sparse_latent(_ptr(q), _ptr(lat), _ptr(idx), T, Tk, H, dl, topk,
                                   float(scale), _ptr(rows), len(rows), _ptr(o), _ptr(lse),
                                   nthreads or default_threads())
+    if rc == -2:
+        raise ValueError("sparse_latent: an index entry is outside [-1, Tk) or a row "
+                         "outside [0, T)")
     assert rc == 0, "oracle_sparse_latent rejected its arguments"
     return o, lse

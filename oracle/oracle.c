@@ -775,13 +775,20 @@ static void sparse_row(void *p, int r, double *z, const float **vr, double *o) {
     }
 }
 
-/* q [T, H, dl]; latent [Tk, dl]; idx [T, topk] (-1 = pad). */
+/* q [T, H, dl]; latent [Tk, dl]; idx [T, topk] (-1 = pad).  An entry
+ * outside [-1, Tk) names no latent row: the call is refused (returns -2)
+ * before anything is read through it, as is a requested row outside [0, T). */
 int oracle_sparse_latent(const float *q, const float *lat, const int32_t *idx,
-                         int T, int H, int dl, int topk, double scale,
+                         int T, int Tk, int H, int dl, int topk, double scale,
                          const int32_t *rows, int nrows, double *o, double *lse,
                          int nthreads) {
-    (void)T;
-    if (H <= 0 || dl <= 0 || topk < 0) return -1;
+    if (T < 0 || Tk < 0 || H <= 0 || dl <= 0 || topk < 0 || nrows < 0) return -1;
+    for (int r = 0; r < nrows; ++r) {
+        if (rows[r] < 0 || rows[r] >= T) return -2;
+        const int32_t *list = idx + (size_t)rows[r] * topk;
+        for (int i = 0; i < topk; ++i)
+            if (list[i] < -1 || list[i] >= Tk) return -2;
+    }
     sparse_ctx c = {q, lat, idx, H, dl, topk, scale, rows, o, lse};
     run_rows(sparse_row, &c, nrows, topk, dl, nthreads);
     return 0;

@@ -283,6 +283,9 @@ def verify_noalloc(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr: torch
     _require_cuda(q_draft, k_draft, v_draft, k_cache, v_cache, kv_indptr)
     BL, Hq, d = q_draft.shape
     Hkv = k_cache.shape[1]
+    if Ld <= 0 or BL % Ld != 0:
+        raise ValueError(f"verify_noalloc: {BL} draft rows are not a whole number of "
+                         f"requests of {Ld} drafts")
     B = BL // Ld
     out = torch.empty_like(q_draft) if out is None else out
     lse = torch.empty((BL, Hq), dtype=torch.float32, device=q_draft.device) if lse is None else lse

@@ -26,7 +26,6 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include <mutex>
 
 #include "psa_device.cuh"
 #include "psa_internal.h"
@@ -786,27 +785,24 @@ int launch_verify(const VerifyArgs& a) {
 // ---------------------------------------------------------------------------
 // Verify without a caller workspace: the partials live in a fixed file-scope
 // device array.  Host code cannot use the array's name as a device address,
-// so the address is looked up once per device with that device current.
+// so every call looks the address up in the context that is current for the
+// call.  The lookup allocates nothing and costs little; caching it per device
+// ordinal would hand a stale address to a caller that switched contexts on
+// the same device (a driver-API context of its own, or a context rebuilt
+// after cudaDeviceReset), and the kernels would then fault.
 
 namespace psa {
 namespace {
 
 static __device__ __align__(256) uint8_t g_verify_scratch[PSA_VERIFY_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
-
 int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_verify_scratch) != cudaSuccess || !p) return PSA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_verify_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();
+    return PSA_ERR_CUDA;
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return PSA_OK;
 }
 

@@ -61,6 +61,10 @@ def _check(got, ref, what):
     (128, 2, 64, 2, 1, 128, 2),    # two packed groups, MQA
     (5, 7, 3, 2, 2, 128, 1),       # rows and keys far below one tile
     (300, 2, 41, 2, 2, 128, 1),    # several KV blocks, partial diagonal tiles
+    # long units: a prefix key block collects 1024 + 4 * 256 query rows of
+    # each of its two query heads, far more ring slots and tiles than above
+    (1024, 4, 256, 4, 2, 128, 1),
+    (512, 4, 128, 4, 2, 128, 2),   # two packed groups with GQA 2:1
 ])
 def test_backward_parity_flat(P, N, S, Hq, Hkv, d, groups):
     wl = W.PrefillWorkload("t", P=P, N=N, S=S, Hq=Hq, Hkv=Hkv, d=d, groups=groups)
@@ -105,3 +109,31 @@ def test_backward_full_size_grpo():
     assert (sv - want).norm() <= REL_FRO * want.norm()
     sk = dk.double().sum(0)
     assert sk.norm() <= 0.05 * dk.double().norm()
+
+
+def test_backward_full_size_grpo_heads_elementwise():
+    """The GRPO group at full size (T = 6144, 16 heads, d = 128), through the
+    same call as above, with every element of dq, dk and dv of two whole
+    heads checked against the oracle.  With 16 query heads over 16 KV heads
+    a head's gradients depend on that head's Q, K, V and dO only, so the
+    oracle runs on the head slice; every prefix key block's unit streams
+    all 2048 + 8 * 512 query rows that see it."""
+    wl = W.GRPO
+    q, k, v = wl.make("cpu")
+    gen = torch.Generator().manual_seed(301)
+    dout = (torch.randn((wl.T, wl.Hq, wl.d), generator=gen) * 0.5).to(torch.bfloat16)
+    qg, kg, vg, dog = (t.cuda() for t in (q, k, v, dout))
+    sched = psa.plan_prefill(wl.segments(), wl.cu_seqlens(), wl.d, "cuda")
+    o, lse = psa.prefill(qg, kg, vg, sched, wl.scale)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dk, dv = psa.prefill_bwd(qg, kg, vg, o, lse, dog,
+                                 psa.plan_prefill_bwd(wl.segments(), wl.cu_seqlens(), wl.d),
+                                 wl.scale, status=status)
+    torch.cuda.synchronize()
+    assert psa.read_status(status) == 0
+    assert wl.Hq == wl.Hkv
+    for h in (0, wl.Hq - 1):
+        sl = lambda t: t[:, h:h + 1].contiguous()  # noqa: E731
+        rq, rk, rv = oracle.prefill_bwd(sl(q), sl(k), sl(v), sl(dout), wl.segments(), wl.scale)
+        _check((dq[:, h:h + 1], dk[:, h:h + 1], dv[:, h:h + 1]), (rq, rk, rv),
+               f"GRPO head {h}")

@@ -616,3 +616,21 @@ def test_pair_counts_closed_form():
     assert W.GRPO.visible_pairs_per_head() == 11_537_408
     assert W.LARGE.visible_pairs_per_head() == 352_346_112
     assert W.SPARSE.pairs() == 31_458_304
+
+
+def test_sparse_oracle_refuses_indices_outside_the_latent():
+    """An index list entry must name a latent row or be the -1 pad: the
+    checker refuses anything else instead of reading past its buffer."""
+    wl = W.SparseLatentWorkload("t", T=20, H=2, dl=16, topk=8, seed=4)
+    q, lat, idx = wl.make()
+    oracle.sparse_latent(q, lat, idx, wl.scale)          # valid lists pass
+    for bad_val in (lat.shape[0], 10_000, -2):
+        bad = idx.clone()
+        bad[13, 2] = bad_val
+        with pytest.raises(ValueError):
+            oracle.sparse_latent(q, lat, bad, wl.scale)
+        # a row sample that skips the bad row is still served
+        o, _ = oracle.sparse_latent(q, lat, bad, wl.scale, rows=[0, 12, 19])
+        assert np.isfinite(o).all()
+    with pytest.raises(ValueError):
+        oracle.sparse_latent(q, lat, idx, wl.scale, rows=[20])

@@ -71,6 +71,8 @@ def test_sparse_out_of_range_index_is_skipped_and_reported():
     assert st == psa.PSA_ERR_INVALID_ARG
     ref_idx = bad.clone()
     ref_idx[140, 3] = -1          # the kernel skips it; the oracle is told so
+    with pytest.raises(ValueError):  # the oracle itself refuses the bad entry
+        oracle.sparse_latent(q, lat, bad, wl.scale, rows=[140])
     ro, rl = oracle.sparse_latent(q, lat, ref_idx, wl.scale)
     assert_parity(o, lse, ro, rl, "out of range skipped")
 

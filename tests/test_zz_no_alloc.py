@@ -10,8 +10,11 @@ fresh process and after the other tests (which leave the array holding the
 previous call's data -- nothing in it needs to start at zero)."""
 import ctypes
 
+import numpy as np
 import pytest
 import torch
+
+import oracle
 
 import shared_prefix_attention_b200 as psa
 from shared_prefix_attention_b200 import workloads as W
@@ -48,7 +51,9 @@ def _noalloc_call(wl, ts, indptr, status):
 def test_noalloc_matches_workspace_entry_on_two_calls():
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     # two calls in a row with different shapes and data: the second reuses
-    # the array the first one filled
+    # the array the first one filled.  Both entries run the same kernels with
+    # the same split count on the same inputs, so their results are
+    # bit-identical; a stale split row left in the array would break that.
     for seed, lens in ((21, [700, 64, 1500]), (22, [33, 2048])):
         wl, ts, indptr = _inputs(seed, lens)
         o_na, l_na = _noalloc_call(wl, ts, indptr, status)
@@ -56,9 +61,28 @@ def test_noalloc_matches_workspace_entry_on_two_calls():
                                 nsplit=wl.nsplit)
         torch.cuda.synchronize()
         assert psa.read_status(status) == 0
-        e = errors(o_na, l_na, o_ws.double().cpu().numpy(), l_ws.double().cpu().numpy())
+        assert torch.equal(o_na, o_ws)
+        assert torch.equal(l_na, l_ws)
+        # and pinned to the fp64 oracle directly
+        q, kd, vd, kc, vc = (t.cpu() for t in ts)
+        ro, rl = oracle.verify(q, kd, vd, kc, vc, np.array(wl.kv_indptr(), dtype=np.int64),
+                               wl.Ld, wl.scale)
+        e = errors(o_na, l_na, ro, rl)
         assert e["o_max_abs"] <= O_MAX_ABS and e["o_rel_fro"] <= O_REL_FRO, e
         assert e["lse_max_abs"] <= LSE_MAX_ABS, e
+
+
+def test_noalloc_python_wrapper_matches_workspace_entry():
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    wl, ts, indptr = _inputs(24, [300, 1024, 5])
+    o_na, l_na = psa.verify_noalloc(*ts, indptr, max(wl.lens()), wl.scale, wl.Ld,
+                                    nsplit=wl.nsplit, status=status)
+    o_ws, l_ws = psa.verify(*ts, indptr, max(wl.lens()), wl.scale, wl.Ld, nsplit=wl.nsplit)
+    torch.cuda.synchronize()
+    assert psa.read_status(status) == 0
+    assert torch.equal(o_na, o_ws) and torch.equal(l_na, l_ws)
+    with pytest.raises(ValueError):
+        psa.verify_noalloc(ts[0][:-1], *ts[1:], indptr, max(wl.lens()), wl.scale, wl.Ld)
 
 
 def test_noalloc_rejects_calls_beyond_the_scratch():
