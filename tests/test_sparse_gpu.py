@@ -67,12 +67,14 @@ def test_sparse_out_of_range_index_is_skipped_and_reported():
     q, lat, idx = wl.make("cpu")
     bad = idx.clone()
     bad[140, 3] = 10_000          # beyond the latent rows
-    o, lse, _, _, st = _run(q, lat, bad, wl.scale)
-    assert st == psa.PSA_ERR_INVALID_ARG
-    ref_idx = bad.clone()
-    ref_idx[140, 3] = -1          # the kernel skips it; the oracle is told so
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = psa.sparse_latent(q.cuda(), lat.cuda(), bad.cuda(), wl.scale, status=status)
+    torch.cuda.synchronize()
+    assert psa.read_status(status) == psa.PSA_ERR_INVALID_ARG
     with pytest.raises(ValueError):  # the oracle itself refuses the bad entry
         oracle.sparse_latent(q, lat, bad, wl.scale, rows=[140])
+    ref_idx = bad.clone()
+    ref_idx[140, 3] = -1          # the kernel skips it; the oracle is told so
     ro, rl = oracle.sparse_latent(q, lat, ref_idx, wl.scale)
     assert_parity(o, lse, ro, rl, "out of range skipped")
 
