@@ -50,7 +50,11 @@ typedef enum psa_status {
     PSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than *_workspace_size */
     PSA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
     PSA_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up (via dev_status) */
-    PSA_ERR_CAPACITY = 6      /* a host output array is too small; *nout holds the need */
+    PSA_ERR_CAPACITY = 6,     /* a host output array is too small; *nout holds the need */
+    PSA_ERR_BOUNDS = 7        /* debug build (libpsa_debug.so) only, via dev_status: a
+                                 device-side bounds check found an index taken from caller
+                                 data (a schedule entry, a prefix or mask offset) outside
+                                 its buffer; the access was skipped, the results are void */
 } psa_status;
 
 typedef enum psa_dtype {

@@ -14,6 +14,10 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpsa.so")
+# The same library built with device-side bounds checks (PSA_DEBUG): an index
+# taken from caller data outside its buffer is reported as PSA_ERR_BOUNDS
+# through the status word instead of being followed.
+DEBUG_LIB_PATH = os.path.join(_HERE, "libpsa_debug.so")
 
 PSA_OK = 0
 PSA_ERR_INVALID_ARG = 1
@@ -22,6 +26,7 @@ PSA_ERR_WORKSPACE = 3
 PSA_ERR_CUDA = 4
 PSA_ERR_TIMEOUT = 5
 PSA_ERR_CAPACITY = 6
+PSA_ERR_BOUNDS = 7
 PSA_BF16 = 0
 PSA_F32 = 1
 
@@ -72,12 +77,43 @@ _lib = None
 def lib():
     """The loaded libpsa (raises if it has not been built)."""
     global _lib
-    if _lib is not None:
+    if _lib is None:
+        _lib = load(LIB_PATH)
+    return _lib
+
+
+class use_library:
+    """Context manager: the binding's calls go to the library at ``path``
+    (e.g. DEBUG_LIB_PATH) inside the block, and back to the previous one
+    after it."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.saved = _lib
+        _lib = load(self.path)
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
+
+
+_loaded: dict = {}
+
+
+def load(path: str):
+    """Load a build of libpsa and declare its C signatures (cached per path;
+    raises if the file is missing)."""
+    if path in _loaded:
+        return _loaded[path]
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
                            "`python -m shared_prefix_attention_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     P, I32, I64, SZ, F = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
                           ctypes.c_float)
     sig = {
@@ -121,7 +157,7 @@ def lib():
         fn = getattr(L, name)
         fn.argtypes = args
         fn.restype = res
-    _lib = L
+    _loaded[path] = L
     return L
 
 

@@ -92,6 +92,8 @@ extern "C" const char* psa_status_string(int status) {
       return "device-side wait timed out";
     case PSA_ERR_CAPACITY:
       return "output capacity too small";
+    case PSA_ERR_BOUNDS:
+      return "device bounds check failed (debug build)";
     default:
       return "unknown status";
   }

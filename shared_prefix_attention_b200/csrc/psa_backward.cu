@@ -37,6 +37,7 @@
 
 #include <type_traits>
 
+#include "psa_debug.cuh"
 #include "psa_device.cuh"
 #include "psa_internal.h"
 
@@ -66,8 +67,9 @@ __device__ __forceinline__ bool sched_ok(const int32_t* sch, int64_t len) {
 // orientation (keys are rows in the transposed spec, whose causal rectangles
 // carry causal == 2: row sees col iff col - k0 >= row - q0).
 __device__ __forceinline__ uint64_t rect_mask(const int32_t* rects, int rb, int rc, int row,
-                                              int c0) {
+                                              int c0, int32_t n_rect, int32_t* status) {
   uint64_t m = 0;
+  if (!psa_in_bounds(rb >= 0 && rc >= 0 && int64_t(rb) + rc <= n_rect, status)) return 0;
   for (int i = 0; i < rc; ++i) {
     const int32_t* r = rects + 5 * (rb + i);
     const int q0 = __ldg(r), q1 = __ldg(r + 1), k0 = __ldg(r + 2), k1 = __ldg(r + 3);
@@ -180,11 +182,17 @@ __device__ __forceinline__ int snake_unit(int r) {
 // The unit's schedule item and head (dq: query head; dkdv: KV head) and its
 // number of streamed tiles (dkdv: every query head of the group).
 template <int MODE>
-__device__ __forceinline__ int unit_tiles(const BwdParams& p, const int4* items, int u, int4& it,
-                                          int& head) {
+__device__ __forceinline__ int unit_tiles(const BwdParams& p, const int4* items, int32_t n_kv,
+                                          int u, int4& it, int& head) {
   const int H = MODE == kDq ? p.Hq : p.Hkv;
   it = __ldg(items + u / H);
   head = u % H;
+  // a block outside the schedule or the tokens becomes an empty one for
+  // every role (debug build)
+  if (!psa_in_bounds(it.x >= 0 && it.y >= 0 && it.y <= BLK && int64_t(it.x) + it.y <= p.T &&
+                         it.z >= 0 && it.w >= 0 && int64_t(it.z) + it.w <= n_kv,
+                     p.status))
+    it = make_int4(0, 0, 0, 0);
   return MODE == kDq ? it.w : it.w * p.G;
 }
 
@@ -206,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) report_status(p.status, PSA_ERR_INVALID_ARG);
     return;
   }
-  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2);
+  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2), n_rect = __ldg(sch + 3);
   const int4* items = reinterpret_cast<const int4*>(sch + 8);
   const int32_t* tiles = sch + 8 + 4 * n_items;  // the column tiles of each block
   const int32_t* rects = tiles + 8 * n_kv;
@@ -261,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u >= units) break;
         int4 it;
         int head;
-        const int nt = unit_tiles<MODE>(p, items, u, it, head);
+        const int nt = unit_tiles<MODE>(p, items, n_kv, u, it, head);
         if (nt == 0) continue;
         // block operands X1, X2 (rows it.x .. it.x + 127 of this head)
         if (!mbar_wait(B.blk_empty, (ub & 1) ^ 1, &abort_flag, p.status)) break;
@@ -372,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u >= units) break;
         int4 it;
         int head;
-        const int nt = unit_tiles<MODE>(p, items, u, it, head);
+        const int nt = unit_tiles<MODE>(p, items, n_kv, u, it, head);
         if (nt == 0) continue;
         if (!mbar_wait(B.blk_full, ub & 1, &abort_flag, p.status)) break;
         // S runs NBUF - 1 tiles ahead of the accumulating products: the
@@ -410,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (u >= units) break;
       int4 it;
       int head;
-      const int nt = unit_tiles<MODE>(p, items, u, it, head);
+      const int nt = unit_tiles<MODE>(p, items, n_kv, u, it, head);
       const int grow = it.x + row;                 // this thread's row (query or key)
       const bool rvalid = row < it.y;
       // epilogue targets: dq writes dQ [T, Hq, D]; dkdv writes dV (wg 0) and dK (wg 1)
@@ -445,7 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (flags & (4 << half))
             vis = clen >= 64 ? ~0ull : ((1ull << clen) - 1ull);
           else
-            vis = rect_mask(rects, __ldg(e + 2 + 2 * half), __ldg(e + 3 + 2 * half), grow, c0);
+            vis = rect_mask(rects, __ldg(e + 2 + 2 * half), __ldg(e + 3 + 2 * half), grow, c0,
+                            n_rect, p.status);
         }
         const float* lse_col = nullptr;  // negated, as stored
         const float* dlt_col = nullptr;

@@ -32,6 +32,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "psa_debug.cuh"
 #include "psa_device.cuh"
 #include "psa_internal.h"
 #include "psa_tmem_wide.cuh"
@@ -132,14 +133,23 @@ __device__ __forceinline__ KvEntry load_kv(const int32_t* kvs, int idx, int x) {
   return e;
 }
 
+// A schedule block as the kernels use it: its rows inside [0, T) and its
+// tile entries inside the schedule's tile list (checked in the debug build).
+__device__ __forceinline__ bool item_in_bounds(const int4& it, int32_t n_kv, int32_t T) {
+  return it.x >= 0 && it.y >= 0 && it.y <= BLOCK_M && int64_t(it.x) + it.y <= T && it.z >= 0 &&
+         it.w >= 0 && int64_t(it.z) + it.w <= n_kv;
+}
+
 // Visible keys of row q inside KV tile e for half x, as a 128-bit mask.
 __device__ __forceinline__ void row_visibility(const KvEntry& e, int x, int q,
-                                               const int32_t* rects, uint32_t (&vis)[4]) {
+                                               const int32_t* rects, int32_t n_rect,
+                                               int32_t* status, uint32_t (&vis)[4]) {
   vis[0] = vis[1] = vis[2] = vis[3] = 0u;
   if (e.flags & (4 << x)) {
     set_bits(vis, 0, e.klen);
     return;
   }
+  if (!psa_in_bounds(e.rb >= 0 && e.rc >= 0 && int64_t(e.rb) + e.rc <= n_rect, status)) return;
   for (int ri = 0; ri < e.rc; ++ri) {
     const int32_t* rc = rects + 5 * (e.rb + ri);
     const int rq0 = __ldg(rc), rq1 = __ldg(rc + 1), rk0 = __ldg(rc + 2), rk1 = __ldg(rc + 3),
@@ -173,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) report_status(p.status, PSA_ERR_INVALID_ARG);
     return;
   }
-  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2);
+  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2), n_rect = __ldg(sch + 3);
   const int4* items = reinterpret_cast<const int4*>(sch + 8);
   const int32_t* kvs = sch + 8 + 4 * n_items;
   const int32_t* rects = kvs + 8 * n_kv;
@@ -252,6 +262,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(B.sch_empty + slot_s, sph ^ 1, &abort_flag, p.status)) break;
           u = atomicAdd(p.counter, 1);
           if (u < units) it = __ldg(items + u / p.Hq);
+          // a block outside the schedule or the tokens becomes an empty one
+          // for every role (debug build)
+          if (!psa_in_bounds(item_in_bounds(it, n_kv, p.T), p.status)) it = make_int4(0, 0, 0, 0);
           sch_item[slot_s] = it;
           sch_unit[slot_s] = u;
           mbar_arrive(B.sch_full + slot_s);
@@ -448,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         const bool need_mask = !(e.flags & (4 << x)) || e.klen < BN;
         uint32_t vis[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-        if (need_mask) row_visibility(e, x, q, rects, vis);
+        if (need_mask) row_visibility(e, x, q, rects, n_rect, p.status, vis);
 
         // the whole S row in one TMEM load
         uint32_t sr[BN];
@@ -584,13 +597,13 @@ template <int D>
 __global__ void __launch_bounds__(256) prefill_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
     float* __restrict__ o, float* __restrict__ lse, const int32_t* __restrict__ sch,
-    int64_t sched_len, int32_t Hq, int32_t G, float scale_log2, int32_t* status) {
+    int64_t sched_len, int32_t T, int32_t Hq, int32_t G, float scale_log2, int32_t* status) {
   constexpr int E = D / 32;
   if (!schedule_ok(sch, sched_len)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) report_status(status, PSA_ERR_INVALID_ARG);
     return;
   }
-  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2);
+  const int32_t n_items = __ldg(sch + 1), n_kv = __ldg(sch + 2), n_rect = __ldg(sch + 3);
   const int4* items = reinterpret_cast<const int4*>(sch + 8);
   const int32_t* kvs = sch + 8 + 4 * n_items;
   const int32_t* rects = kvs + 8 * n_kv;
@@ -604,6 +617,7 @@ __global__ void __launch_bounds__(256) prefill_f32_kernel(
     const int rem = int(u % (int64_t(BLOCK_M) * Hq));
     const int r = rem / Hq, h = rem % Hq;
     const int4 it = __ldg(items + item);
+    if (!psa_in_bounds(item_in_bounds(it, n_kv, T), lane == 0 ? status : nullptr)) continue;
     if (r >= it.y) continue;
     const int x = r / BM;
     const int qi = it.x + r, kvh = h / G;
@@ -618,7 +632,7 @@ __global__ void __launch_bounds__(256) prefill_f32_kernel(
       const KvEntry ent = load_kv(kvs, it.z + j, x);
       if (!(ent.flags & (1 << x))) continue;
       uint32_t vis[4];
-      row_visibility(ent, x, qi, rects, vis);
+      row_visibility(ent, x, qi, rects, n_rect, status, vis);
       for (int kk = 0; kk < ent.klen; ++kk) {
         if (!((vis[kk >> 5] >> (kk & 31)) & 1u)) continue;
         const int key = ent.k0 + kk;
@@ -655,7 +669,7 @@ int launch_prefill_f32_d(const PrefillArgs& a) {
   prefill_f32_kernel<D><<<grid, 256, 0, a.stream>>>(
       static_cast<const float*>(a.q), static_cast<const float*>(a.k),
       static_cast<const float*>(a.v), static_cast<float*>(a.o), a.lse, a.sched, a.sched_len,
-      a.Hq, a.Hq / a.Hkv, a.scale * kLog2e, a.status);
+      a.T, a.Hq, a.Hq / a.Hkv, a.scale * kLog2e, a.status);
   return cudaGetLastError() == cudaSuccess ? PSA_OK : PSA_ERR_CUDA;
 }
 

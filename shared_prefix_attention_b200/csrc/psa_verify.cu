@@ -27,6 +27,7 @@
 #include <cuda_runtime.h>
 
 
+#include "psa_debug.cuh"
 #include "psa_device.cuh"
 #include "psa_internal.h"
 
@@ -123,7 +124,13 @@ __device__ __forceinline__ void split_range(const Stage1Params& p, int b, int s,
   const int32_t a = __ldg(p.indptr + b), e = __ldg(p.indptr + b + 1);
   int32_t L = e - a;
   // a paged prefix must lie inside the page table, whose length is indptr[B]
-  if (L < 0 || a < 0 || (p.kv_indices && e > __ldg(p.indptr + p.B))) L = 0;
+  const bool in_table = !p.kv_indices || e <= __ldg(p.indptr + p.B);
+  if (L < 0 || a < 0 || !in_table) L = 0;
+  // debug build: an offset outside the page table or (contiguous) the cache
+  // is reported and the request's prefix left out
+  if (!psa_in_bounds(e >= a && a >= 0 && in_table && (p.kv_indices || int64_t(e) <= p.ntok),
+                     p.status))
+    L = 0;
   int32_t c = (L + p.nsplit - 1) / p.nsplit;
   c = (c + kTileKeys - 1) / kTileKeys * kTileKeys;
   t0 = a + min(L, s * c);
@@ -559,11 +566,18 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
   };
   // the draft block: drafts 0..j, or the tree mask's row (the same for every head)
   const uint8_t* mrow = nullptr;
-  if (p.dmask)
-    mrow = p.dmask + (p.mask_indptr ? size_t(__ldg(p.mask_indptr + b)) : size_t(q0) * Lb) +
-           size_t(j) * Lb;
+  bool mask_ok = true;
+  if (p.dmask) {
+    const int64_t moff = p.mask_indptr ? int64_t(__ldg(p.mask_indptr + b)) : int64_t(q0) * Lb;
+    // debug build: request b's Lb x Lb block must lie inside the mask, whose
+    // length is mask_indptr[B]; otherwise no draft is seen
+    mask_ok = psa_in_bounds(!p.mask_indptr || (moff >= 0 && moff + int64_t(Lb) * Lb <=
+                                                                 __ldg(p.mask_indptr + p.B)),
+                            lane == 0 ? p.status : nullptr);
+    mrow = p.dmask + size_t(moff) + size_t(j) * Lb;
+  }
   auto sees = [&](int i) { return mrow ? __ldg(mrow + i) != 0 : i <= j; };
-  const int nd = mrow ? Lb : j + 1;
+  const int nd = !mask_ok ? 0 : mrow ? Lb : j + 1;
   float M = -INFINITY;
   for (int i = 0; i < nd; ++i)
     if (sees(i)) M = fmaxf(M, draft_logit(i));

@@ -29,6 +29,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "psa_debug.cuh"
 #include "psa_device.cuh"
 #include "psa_internal.h"
 
@@ -109,7 +110,13 @@ __device__ __forceinline__ void split_range8(const P8Params& p, int b, int s, in
   const int32_t a = __ldg(p.indptr + b), e = __ldg(p.indptr + b + 1);
   int32_t L = e - a;
   // a paged prefix must lie inside the page table, whose length is indptr[B]
-  if (L < 0 || a < 0 || (p.kv_indices && e > __ldg(p.indptr + p.B))) L = 0;
+  const bool in_table = !p.kv_indices || e <= __ldg(p.indptr + p.B);
+  if (L < 0 || a < 0 || !in_table) L = 0;
+  // debug build: an offset outside the page table or (contiguous) the cache
+  // is reported and the request's prefix left out
+  if (!psa_in_bounds(e >= a && a >= 0 && in_table && (p.kv_indices || int64_t(e) <= p.ntok),
+                     p.status))
+    L = 0;
   int32_t c = (L + p.nsplit - 1) / p.nsplit;
   c = (c + kKeys - 1) / kKeys * kKeys;
   t0 = a + min(L, s * c);
