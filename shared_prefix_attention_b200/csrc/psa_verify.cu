@@ -578,11 +578,25 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
   }
   auto sees = [&](int i) { return mrow ? __ldg(mrow + i) != 0 : i <= j; };
   const int nd = !mask_ok ? 0 : mrow ? Lb : j + 1;
-  float M = -INFINITY;
-  for (int i = 0; i < nd; ++i)
-    if (sees(i)) M = fmaxf(M, draft_logit(i));
-  for (int s = lane; s < p.nsplit; s += 32)
-    M = fmaxf(M, p.part_lse[(size_t(s) * BL + row) * p.Hq + qh]);
+  // The draft logits, computed once: lane i keeps draft i's (nd <= 16).
+  float M = -INFINITY, dlog = -INFINITY;
+  for (int i = 0; i < nd; ++i) {
+    if (!sees(i)) continue;
+    const float l = draft_logit(i);
+    if (lane == i) dlog = l;
+    M = fmaxf(M, l);
+  }
+  // The splits' LSEs, all loaded up front: split s sits in lane s % 32 of
+  // slot s / 32 (nsplit <= 256), so the combine below waits on no load to
+  // learn a weight.
+  constexpr int kSlots = 8;
+  float lsv[kSlots];
+#pragma unroll
+  for (int k = 0; k < kSlots; ++k) {
+    const int s = k * 32 + lane;
+    lsv[k] = s < p.nsplit ? p.part_lse[(size_t(s) * BL + row) * p.Hq + qh] : -INFINITY;
+    M = fmaxf(M, lsv[k]);
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   if (M == -INFINITY) {
@@ -597,24 +611,45 @@ __global__ void __launch_bounds__(256) verify_stage2_kernel(Stage2Params p) {
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
-  for (int s = 0; s < p.nsplit; ++s) {
-    const size_t prow = (size_t(s) * BL + row) * p.Hq + qh;
-    const float ls = p.part_lse[prow];
-    const float w = fast_exp2(ls - M);  // empty split: exp2(-inf) = 0
-    if (w == 0.f) continue;
-    const float* op = p.part_o + prow * D + lane * E;
+  float wsum = 0.f;  // this lane's splits; summed over the warp below
+  // Partial O rows, four splits per step: the weights come from the
+  // registers above by shuffle and the four loads are in flight together.
+  // An empty split (LSE -inf, weight 0) is not read.
 #pragma unroll
-    for (int e = 0; e < E; e += 2) {
-      const float2 v = *reinterpret_cast<const float2*>(op + e);
-      acc[e] += w * v.x;
-      acc[e + 1] += w * v.y;
+  for (int k = 0; k < kSlots; ++k) {
+    if (k * 32 >= p.nsplit) break;
+    const float wk = fast_exp2(lsv[k] - M);  // empty or absent split: exp2(-inf) = 0
+    wsum += wk;
+    const int nj = min(32, p.nsplit - k * 32);
+    for (int j0 = 0; j0 < nj; j0 += 4) {
+      float w[4];
+      float v[4][E];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int jj = j0 + u;
+        w[u] = __shfl_sync(0xffffffffu, wk, jj & 31);
+        if (jj >= nj) w[u] = 0.f;
+        const size_t prow = (size_t(k * 32 + jj) * BL + row) * p.Hq + qh;
+        const float* op = p.part_o + prow * D + lane * E;
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+          float2 x = make_float2(0.f, 0.f);
+          if (w[u] != 0.f) x = *reinterpret_cast<const float2*>(op + e);
+          v[u][e] = x.x;
+          v[u][e + 1] = x.y;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] += w[u] * v[u][e];
     }
-    wsum += w;
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
   for (int i = 0; i < nd; ++i) {
     if (!sees(i)) continue;
-    const float w = fast_exp2(draft_logit(i) - M);
+    const float w = fast_exp2(__shfl_sync(0xffffffffu, dlog, i) - M);
     const __nv_bfloat16* vp = p.vd + (size_t(q0 + i) * p.Hkv + kvh) * D + lane * E;
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] += w * __bfloat162float(vp[e]);
