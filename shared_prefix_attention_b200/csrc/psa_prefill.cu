@@ -8,7 +8,9 @@
 // sm_100a design.  One CTA per SM, persistent over units (Q block of 256
 // rows, query head).  The host schedule lists the blocks longest-first and
 // the producer hands units out through a global counter, so long suffix
-// blocks start first and short prefix blocks fill the tail.  A block is two
+// blocks start first and short prefix blocks fill the tail (per KV head when
+// each KV head has units for two waves, so the CTAs in flight share its K/V
+// in L2).  A block is two
 // 128-row halves A and B that share every K/V tile load:
 //   warps 0, 2   TMA producers (Q and K; V): the Q block, then the K and V
 //                tiles of the block's visible KV tiles only (invisible tiles
@@ -105,6 +107,24 @@ __device__ __forceinline__ void regs_dec() {
 }
 __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+}
+
+// Unit u -> (schedule block, query head).  When every KV head has at least
+// two waves of units, the order is KV-head-major (blocks longest-first within
+// a KV head, its G query heads adjacent), so the CTAs in flight all stream
+// the same KV head's K/V tiles and L2 serves the re-reads; otherwise it is
+// block-major with the query heads adjacent.
+__device__ __forceinline__ void unit_block_head(int u, int n_items, int Hq, int G, int& item,
+                                                int& h) {
+  if (int64_t(n_items) * G >= 2 * int64_t(gridDim.x)) {
+    const int per_kv = n_items * G;
+    const int kvh = u / per_kv, rem = u - kvh * per_kv;
+    item = rem / G;
+    h = kvh * G + (rem - item * G);
+  } else {
+    item = u / Hq;
+    h = u - item * Hq;
+  }
 }
 
 // Header check shared by both prefill kernels (uniform across threads).
@@ -261,7 +281,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (kprod) {
           if (!mbar_wait(B.sch_empty + slot_s, sph ^ 1, &abort_flag, p.status)) break;
           u = atomicAdd(p.counter, 1);
-          if (u < units) it = __ldg(items + u / p.Hq);
+          if (u < units) {
+            int item, hh;
+            unit_block_head(u, n_items, p.Hq, p.G, item, hh);
+            it = __ldg(items + item);
+          }
           // a block outside the schedule or the tokens becomes an empty one
           // for every role (debug build)
           if (!psa_in_bounds(item_in_bounds(it, n_kv, p.T), p.status)) it = make_int4(0, 0, 0, 0);
@@ -275,7 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(B.sch_empty + slot_s);
         }
         if (u >= units) break;
-        const int h = u % p.Hq, kvh = h / p.G;
+        int item_u, h;
+        unit_block_head(u, n_items, p.Hq, p.G, item_u, h);
+        const int kvh = h / p.G;
         if (it.w == 0) continue;
         if (kprod) {
           if (!mbar_wait(B.q_empty, (uc & 1) ^ 1, &abort_flag, p.status)) break;
@@ -439,7 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(B.sch_empty + slot_s);
       if (u >= units) break;
-      const int h = u % p.Hq;
+      int item_u, h;
+      unit_block_head(u, n_items, p.Hq, p.G, item_u, h);
       const int q = it.x + x * BM + r;
       const bool valid = x * BM + r < it.y;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.o) + (size_t(q) * p.Hq + h) * D;
