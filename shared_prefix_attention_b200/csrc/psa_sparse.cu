@@ -74,7 +74,7 @@ constexpr uint32_t RED_BYTES = 2 * 4 * HMAX * 4;             // max and sum: [4 
 constexpr uint32_t OFF_HEAD = OFF_RED + RED_BYTES;           // per-head state
 constexpr uint32_t HEAD_BYTES = 4 * HMAX * 4;                // m, l, alpha, 1/l
 constexpr uint32_t OFF_BAR = OFF_HEAD + HEAD_BYTES;
-constexpr uint32_t NBAR = 2 * NPART + 2 + 5;
+constexpr uint32_t NBAR = 2 * NPART + 2 + 6;
 constexpr uint32_t SMEM = 1024 + OFF_BAR + NBAR * 8 + 64;
 
 struct Params {
@@ -119,20 +119,6 @@ __device__ __forceinline__ bool mbar_wait_hot(uint64_t* bar, uint32_t parity,
     }
   }
 }
-
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// A softmax-group barrier that every member skips once the CTA has aborted
-// (a member that gave up on a bounded wait never reaches the barrier); the
-// `break` leaves the enclosing loop.
-#define GROUP_SYNC(id)                 \
-  if (*(volatile int*)&abort_flag) {   \
-    ok = false;                        \
-    break;                             \
-  } else                               \
-    named_bar_sync((id), kSoftmaxThreads)
 
 // Reduces v[0..31] across the 32 lanes of the warp (max or sum); afterwards
 // lane L holds the result for entry L.  Each step keeps the half of the
@@ -223,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ uint32_t tmem_base_slot;
   __shared__ int abort_flag;
   __shared__ int q_ntiles;
+  __shared__ int over_tile;  // 1 + the last tile whose logits outgrew a running max
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -235,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pv_done = p_full + 1;            // MMA commit
   uint64_t* o_full = pv_done + 1;            // MMA commit
   uint64_t* o_free = o_full + 1;             // 8 softmax warps
+  uint64_t* grp = o_free + 1;                // the softmax group's rendezvous (8 warps)
   float* red_max = reinterpret_cast<float*>(smem + OFF_RED);  // [4 quadrants][64]
   float* red_sum = red_max + 4 * HMAX;                         // [4 quadrants][64]
   float* h_m = reinterpret_cast<float*>(smem + OFF_HEAD);  // running max (log2 domain)
@@ -256,6 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
     mbar_init(o_free, kSoftmaxThreads / 32);
+    mbar_init(grp, kSoftmaxThreads / 32);
+    over_tile = 0;
     fence_barrier_init();
   }
   if (threadIdx.x >= 32 * kSoftmaxWarp0 && threadIdx.x < 32 * kSoftmaxWarp0 + HMAX)
@@ -439,6 +429,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tile_glob = 0;
     uint32_t oq = 0;  // queries with at least one tile
     bool ok = true;
+    // The group's rendezvous: an 8-warp mbarrier with the bounded wait, so
+    // a member that gave up cannot leave the others waiting.
+    uint32_t gphase = 0;
+    auto group_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(grp);
+      const bool got = mbar_wait_hot(grp, gphase & 1, &abort_flag, p.status);
+      ++gphase;
+      return got;
+    };
     for (int qi = 0; ok; ++qi) {
       const int t = query_of(qi);
       if (t < 0) break;
@@ -478,23 +478,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < HW; ++h) over = fmaxf(over, v[h] - m[h]);
         }
-        if (*(volatile int*)&abort_flag) {
+        // the group's OR of "some logit outgrew its head's running max":
+        // a warp that saw one marks this tile, then everyone meets
+        if (__any_sync(0xffffffffu, over > kRescaleLog2) && lane == 0)
+          atomicMax(&over_tile, int(tile_glob) + 1);
+        if (!group_sync()) {
           ok = false;
           break;
         }
-        uint32_t any_over;
-        asm volatile(
-            "{\n\t.reg .pred pi, po;\n\t"
-            "setp.gt.f32 pi, %1, %2;\n\t"
-            "bar.red.or.pred po, 2, 256, pi;\n\t"
-            "selp.u32 %0, 1, 0, po;\n\t}"
-            : "=r"(any_over)
-            : "f"(over), "f"(kRescaleLog2)
-            : "memory");
+        const bool any_over = *(volatile int*)&over_tile == int(tile_glob) + 1;
         if (any_over) {
           // cross-key max per head: across lanes, then across quadrants
           red_max[quad * HMAX + hb + lane] = warp_transpose_reduce32<true>(v, lane);
-          GROUP_SYNC(2);
+          if (!group_sync()) {
+            ok = false;
+            break;
+          }
           if (tid < HMAX) {
             const float mt = fmaxf(fmaxf(red_max[tid], red_max[HMAX + tid]),
                                    fmaxf(red_max[2 * HMAX + tid], red_max[3 * HMAX + tid]));
@@ -509,7 +508,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool any = __any_sync(0xffffffffu, alpha != 1.f && j > 0);
             if (lane == 0) h_flagw[tid >> 5] = any ? 1 : 0;
           }
-          GROUP_SYNC(2);
+          if (!group_sync()) {
+            ok = false;
+            break;
+          }
           {
             float a[HW];
             load_heads32(h_alpha + hb, a);
@@ -577,14 +579,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // per-head sums: the partial sums of all keys meet once per query
       red_sum[quad * HMAX + hb + lane] = warp_transpose_reduce32<false>(lpart, lane);
-      GROUP_SYNC(2);
+      if (!group_sync()) {
+        ok = false;
+        break;
+      }
       if (tid < HMAX) {
         const float l = (red_sum[tid] + red_sum[HMAX + tid]) +
                         (red_sum[2 * HMAX + tid] + red_sum[3 * HMAX + tid]);
         h_l[tid] = l;
         h_inv[tid] = l > 0.f ? 1.f / l : 0.f;
       }
-      GROUP_SYNC(2);  // h_l, h_inv final
+      if (!group_sync()) break;  // h_l, h_inv final
       if (ntiles > 0) {
         if (!mbar_wait_hot(o_full, oq & 1, &abort_flag, p.status)) break;
         tc_fence_after();
@@ -608,7 +613,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < HW; ++h)
           stage[(hb + h) * 128 + r] = __float2bfloat16(__uint_as_float(ov[h]) * inv[h]);
-        GROUP_SYNC(2);
+        if (!group_sync()) {
+          ok = false;
+          break;
+        }
 #pragma unroll
         for (int k = 0; k < (HMAX * 16) / kSoftmaxThreads; ++k) {
           const int c = k * kSoftmaxThreads + tid;  // 16-byte chunk: head c / 16, piece c % 16
@@ -617,7 +625,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(p.o + (size_t(t) * p.H + h) * DL + mb * 128 + piece * 8) =
                 *reinterpret_cast<const uint4*>(stage + h * 128 + piece * 8);
         }
-        GROUP_SYNC(2);
+        if (!group_sync()) {
+          ok = false;
+          break;
+        }
       }
       if (!ok) break;
       tc_fence_before();
@@ -631,7 +642,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.lse[size_t(t) * p.H + tid] = l > 0.f ? (h_m[tid] + __log2f(l)) * kLn2 : -INFINITY;
       }
       if (tid < HMAX) h_m[tid] = -INFINITY;  // fresh running max for the next query
-      GROUP_SYNC(2);
+      if (!group_sync()) {
+        ok = false;
+        break;
+      }
     }
   }
 
