@@ -588,17 +588,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_ld();
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow);
+          // the row as 32-byte stores when the output is 32-byte aligned (half
+          // the store instructions of 16-byte ones; each thread's row is its
+          // own, so a warp store touches 32 rows)
+          if ((reinterpret_cast<uintptr_t>(p.o) & 31u) == 0) {
 #pragma unroll
-          for (int k = 0; k < D / 8; ++k)
-            dst[k] = make_uint4(
-                pack_bf16(__uint_as_float(orr[8 * k]) * inv, __uint_as_float(orr[8 * k + 1]) * inv),
-                pack_bf16(__uint_as_float(orr[8 * k + 2]) * inv,
-                          __uint_as_float(orr[8 * k + 3]) * inv),
-                pack_bf16(__uint_as_float(orr[8 * k + 4]) * inv,
-                          __uint_as_float(orr[8 * k + 5]) * inv),
-                pack_bf16(__uint_as_float(orr[8 * k + 6]) * inv,
-                          __uint_as_float(orr[8 * k + 7]) * inv));
+            for (int k = 0; k < D / 16; ++k) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                w[i] = pack_bf16(__uint_as_float(orr[16 * k + 2 * i]) * inv,
+                                 __uint_as_float(orr[16 * k + 2 * i + 1]) * inv);
+              asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                               orow + 16 * k),
+                           "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]),
+                           "r"(w[6]), "r"(w[7])
+                           : "memory");
+            }
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+            for (int k = 0; k < D / 8; ++k)
+              dst[k] = make_uint4(
+                  pack_bf16(__uint_as_float(orr[8 * k]) * inv, __uint_as_float(orr[8 * k + 1]) * inv),
+                  pack_bf16(__uint_as_float(orr[8 * k + 2]) * inv,
+                            __uint_as_float(orr[8 * k + 3]) * inv),
+                  pack_bf16(__uint_as_float(orr[8 * k + 4]) * inv,
+                            __uint_as_float(orr[8 * k + 5]) * inv),
+                  pack_bf16(__uint_as_float(orr[8 * k + 6]) * inv,
+                            __uint_as_float(orr[8 * k + 7]) * inv));
+          }
         }
       }
       tc_fence_before();

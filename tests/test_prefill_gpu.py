@@ -129,3 +129,24 @@ def test_prefill_repeatable_and_independent_of_output_contents():
     o2, l2 = psa.prefill(q, k, v, sched, wl.scale)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_prefill_output_only_16_byte_aligned():
+    """An output that starts 16 bytes past a 32-byte boundary (allowed: the
+    entry asks for 16-byte alignment) takes the epilogue's 16-byte stores;
+    the result is the same bytes as an aligned output's, and matches the
+    oracle."""
+    wl = W.PrefillWorkload("t", P=300, N=3, S=170, Hq=8, Hkv=2, d=128)
+    q, k, v = _inputs(wl.T, 8, 2, 128, 13)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    sched = psa.plan_prefill(wl.segments(), wl.cu_seqlens(), 128)
+    buf = torch.zeros(qd.numel() + 16, dtype=qd.dtype, device="cuda")
+    assert buf.data_ptr() % 32 == 0
+    o_off = buf[8:8 + qd.numel()].view(qd.shape)  # 16 bytes past the boundary
+    o_off, l_off = psa.prefill(qd, kd, vd, sched, wl.scale, out=o_off)
+    o_al, l_al = psa.prefill(qd, kd, vd, sched, wl.scale)
+    torch.cuda.synchronize()
+    assert o_al.data_ptr() % 32 == 0
+    assert torch.equal(o_off, o_al) and torch.equal(l_off, l_al)
+    ro, rl = oracle.prefill(q, k, v, wl.segments(), wl.scale)
+    assert_parity(o_off, l_off, ro, rl, "16-byte-aligned output")
