@@ -432,7 +432,9 @@ int32_t psa_verify_shared_auto_splits(int32_t B, int32_t Ld, int32_t Hq, int32_t
  *   lse              device [B*Ld, Hq] fp32      (written; nullable)
  * Draft j of request b sees prefix tokens 0..L-1 and drafts 0..j of b; the
  * result equals psa_verify_fwd on a cache holding B copies of the prefix.
- * d in {64, 128}; Hq / Hkv must divide 128.  nsplit: 1..256, or 0 for
+ * d in {64, 128}; Hq / Hkv must divide 128; 1 <= Ld <= 16 (the combine
+ * holds a row's draft block in one warp's registers; PSA_ERR_UNSUPPORTED
+ * above).  nsplit: 1..256, or 0 for
  * psa_verify_shared_auto_splits; the prefix is cut into nsplit chunks of
  * ceil(L / nsplit) keys rounded up to 128 (trailing chunks may be empty).
  * workspace: device, >= psa_verify_workspace_size(B, Ld, Hq, d, nsplit)

@@ -307,6 +307,8 @@ static int verify_shared_common(const void* q_draft, const void* k_draft, const 
       prefix_len > (int64_t(1) << 30) || !(scale > 0.f))
     return PSA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return PSA_ERR_UNSUPPORTED;
+  // the combine holds a row's draft block in one warp's registers
+  if (Ld > 16) return PSA_ERR_UNSUPPORTED;
   const int32_t G = Hq / Hkv;
   if (G > 128 || 128 % G != 0) return PSA_ERR_UNSUPPORTED;  // 128-row halves of whole tokens
   if (int64_t(B) * Ld > INT32_MAX / Hq) return PSA_ERR_INVALID_ARG;

@@ -432,6 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // nothing in this block sees (or is seen by) anything: zero gradient
         if (rvalid) {
           __nv_bfloat16* dst = out + (size_t(grow) * Hout + head) * D + ocol0;
+      const bool out_al32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
           for (int c = 0; c < OCOLS; c += 8)
             *reinterpret_cast<uint4*>(dst + c) = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -543,20 +544,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(B.acc_full, ub & 1, &abort_flag, p.status)) break;
       tc_fence_after();
       __nv_bfloat16* dst = out + (size_t(grow) * Hout + head) * D + ocol0;
+      const bool out_al32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
 #pragma unroll
       for (int c = 0; c < OCOLS; c += 32) {
         uint32_t a[32];
         tmem_ld32(tacc + c, a);
         tmem_wait_ld();
         if (rvalid) {
+          if (out_al32) {
+            // 32-byte stores (a thread's row is its own, so a warp store
+            // touches 32 rows; fewer, wider stores halve the instructions)
 #pragma unroll
-          for (int v = 0; v < 32; v += 8) {
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(a[v]) * oscale, __uint_as_float(a[v + 1]) * oscale);
-            w.y = pack_bf16(__uint_as_float(a[v + 2]) * oscale, __uint_as_float(a[v + 3]) * oscale);
-            w.z = pack_bf16(__uint_as_float(a[v + 4]) * oscale, __uint_as_float(a[v + 5]) * oscale);
-            w.w = pack_bf16(__uint_as_float(a[v + 6]) * oscale, __uint_as_float(a[v + 7]) * oscale);
-            *reinterpret_cast<uint4*>(dst + c + v) = w;
+            for (int v = 0; v < 32; v += 16) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                w[i] = pack_bf16(__uint_as_float(a[v + 2 * i]) * oscale,
+                                 __uint_as_float(a[v + 2 * i + 1]) * oscale);
+              asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(
+                               dst + c + v),
+                           "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]),
+                           "r"(w[6]), "r"(w[7])
+                           : "memory");
+            }
+          } else {
+#pragma unroll
+            for (int v = 0; v < 32; v += 8) {
+              uint4 w;
+              w.x = pack_bf16(__uint_as_float(a[v]) * oscale, __uint_as_float(a[v + 1]) * oscale);
+              w.y = pack_bf16(__uint_as_float(a[v + 2]) * oscale, __uint_as_float(a[v + 3]) * oscale);
+              w.z = pack_bf16(__uint_as_float(a[v + 4]) * oscale, __uint_as_float(a[v + 5]) * oscale);
+              w.w = pack_bf16(__uint_as_float(a[v + 6]) * oscale, __uint_as_float(a[v + 7]) * oscale);
+              *reinterpret_cast<uint4*>(dst + c + v) = w;
+            }
           }
         }
       }

@@ -94,6 +94,7 @@ def _shared_call(**kw):
 def test_verify_shared_host_validation():
     assert _shared_call(d=256) == psa.PSA_ERR_UNSUPPORTED             # head dim
     assert _shared_call(Hq=24, Hkv=1) == psa.PSA_ERR_UNSUPPORTED      # 24 rows per token
+    assert _shared_call(Ld=17) == psa.PSA_ERR_UNSUPPORTED             # draft block too big
     assert _shared_call(Hq=6, Hkv=4) == psa.PSA_ERR_INVALID_ARG       # Hq % Hkv
     assert _shared_call(scale=0.0) == psa.PSA_ERR_INVALID_ARG
     assert _shared_call(L=-1) == psa.PSA_ERR_INVALID_ARG

@@ -137,3 +137,30 @@ def test_backward_full_size_grpo_heads_elementwise():
         rq, rk, rv = oracle.prefill_bwd(sl(q), sl(k), sl(v), sl(dout), wl.segments(), wl.scale)
         _check((dq[:, h:h + 1], dk[:, h:h + 1], dv[:, h:h + 1]), (rq, rk, rv),
                f"GRPO head {h}")
+
+
+def test_backward_outputs_only_16_byte_aligned():
+    """dq / dk / dv that start 16 bytes past a 32-byte boundary (allowed: the
+    entry asks for 16-byte alignment) take the epilogue's 16-byte stores; the
+    gradients are the same bytes as with aligned outputs."""
+    segs, cu = psa.spec_flat(100, 3, 37), [0, 100 + 3 * 37]
+    T, Hq, Hkv, d = cu[1], 4, 2, 64
+    gen = torch.Generator().manual_seed(101)
+    draw = lambda shape: (torch.randn(shape, generator=gen) * 0.5).to(torch.bfloat16).cuda()
+    q, k, v, dout = draw((T, Hq, d)), draw((T, Hkv, d)), draw((T, Hkv, d)), draw((T, Hq, d))
+    scale = 1.0 / np.sqrt(d)
+    o, lse = psa.prefill(q, k, v, psa.plan_prefill(segs, cu, d, "cuda"), scale)
+    sch = psa.plan_prefill_bwd(segs, cu, d)
+
+    def offset_like(t):
+        buf = torch.zeros(t.numel() + 16, dtype=t.dtype, device="cuda")
+        assert buf.data_ptr() % 32 == 0
+        return buf[8:8 + t.numel()].view(t.shape)  # 16 bytes past the boundary
+
+    got = psa.prefill_bwd(q, k, v, o, lse, dout, sch, scale, dq=offset_like(q),
+                          dk=offset_like(k), dv=offset_like(v))
+    ref = psa.prefill_bwd(q, k, v, o, lse, dout, sch, scale)
+    torch.cuda.synchronize()
+    for g, r in zip(got, ref):
+        assert r.data_ptr() % 32 == 0 and g.data_ptr() % 32 == 16
+        assert torch.equal(g, r)
