@@ -46,6 +46,7 @@ def _run(wl, rows=None):
     (7, 3, 8, 2, 128, 513, 0),      # 84 rows, one key past a tile boundary
     (40, 4, 32, 8, 128, 1024, 2),   # 640 rows: three row blocks, last one half full
     (4, 4, 32, 1, 128, 384, 1),     # G = 32 (MQA), one split
+    (3, 16, 8, 2, 128, 650, 2),     # the longest draft block the entry takes
 ])
 def test_verify_shared_parity(B, Ld, Hq, Hkv, d, L, nsplit):
     o, lse, ro, rl = _run(_wl(B, Ld, Hq, Hkv, d, L, nsplit))
