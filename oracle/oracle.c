@@ -310,12 +310,20 @@ static void *bwd_worker(void *p) {
                     const float *krow = c->k + ((size_t)ks[i] * c->Hkv + kvh) * d;
                     const float *vrow = c->v + ((size_t)ks[i] * c->Hkv + kvh) * d;
                     double dp = dot(dorow, vrow, d);
+#if ORACLE_MUTANT == 8
+                    double dsc = z[i] * dp;     /* planted: the softmax Jacobian loses D */
+#else
                     double dsc = z[i] * (dp - D);
+#endif
                     double *dkrow = c->dk + ((size_t)ks[i] * c->Hkv + kvh) * d;
                     double *dvrow = c->dv + ((size_t)ks[i] * c->Hkv + kvh) * d;
                     for (int e = 0; e < d; ++e) {
                         dqrow[e] += c->scale * dsc * (double)krow[e];
+#if ORACLE_MUTANT == 9
+                        dkrow[e] += dsc * (double)qrow[e]; /* planted: dk loses the scale */
+#else
                         dkrow[e] += c->scale * dsc * (double)qrow[e];
+#endif
                         dvrow[e] += z[i] * (double)dorow[e];
                     }
                 }
@@ -470,7 +478,11 @@ static void verify_row(void *p, int r, double *z, const float **vr, double *o) {
     if (c->dmask)
         mrow = c->dmask + (c->mask_indptr ? c->mask_indptr[b] : q0 * Lb) + (int64_t)j * Lb;
     int64_t p0 = c->indptr ? c->indptr[b] : 0;
+#if ORACLE_MUTANT == 13
+    int64_t p1 = c->indptr ? c->indptr[b + 1] : c->shared_len - 1; /* planted: shared prefix short by one */
+#else
     int64_t p1 = c->indptr ? c->indptr[b + 1] : c->shared_len;
+#endif
     for (int h = 0; h < c->Hq; ++h) {
         int kvh = kv_head_of(h, c->Hq, c->Hkv);
         const float *qrow = c->qd + ((size_t)row * c->Hq + h) * c->d;
@@ -639,7 +651,11 @@ int oracle_verify_shared_tree(const float *qd, const float *kd, const float *vd,
 static double decode_e4m3(uint8_t b) {
     int sgn = b >> 7, e = (b >> 3) & 15, m = b & 7;
     if (e == 15 && m == 7) return NAN;
+#if ORACLE_MUTANT == 10
+    double v = e == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 8); /* planted: bias 8 */
+#else
     double v = e == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+#endif
     return sgn ? -v : v;
 }
 
@@ -693,7 +709,11 @@ static void verify8_row(void *p, int r, double *z, const float **vr, double *o) 
             double w = exp(z[n++] - m) / l;
             int64_t slot = c->kv_indices ? c->kv_indices[t] : t;
             const uint8_t *vrow = c->vc + ((size_t)slot * c->Hkv + kvh) * c->d;
+#if ORACLE_MUTANT == 11
+            for (int e = 0; e < c->d; ++e) o[e] += w * decode_e4m3(vrow[e]); /* planted: no v_scale */
+#else
             for (int e = 0; e < c->d; ++e) o[e] += w * c->vscale * decode_e4m3(vrow[e]);
+#endif
         }
         for (int i = 0; i <= j; ++i) {
             double w = exp(z[n++] - m) / l;
@@ -763,7 +783,11 @@ static void sparse_row(void *p, int r, double *z, const float **vr, double *o) {
         int n = 0;
         for (int i = 0; i < c->topk; ++i) {
             int32_t kj = list[i];
+#if ORACLE_MUTANT == 12
+            if (kj <= 0) continue;       /* planted: latent row 0 is taken for a pad */
+#else
             if (kj < 0) continue;        /* -1 pads a short list */
+#endif
             const float *lrow = c->lat + (size_t)kj * c->dl; /* K = V = latent */
             z[n] = apply_scale(dot(qrow, lrow, c->dl), c->scale);
             vr[n] = lrow;

@@ -583,8 +583,11 @@ def test_oracle_pin(pin):
 # pin above must catch: 1 drops the scale, 2 makes causality strict,
 # 3 interleaves GQA heads, 4 hides the prefix from suffixes, 5 drops the
 # row maximum from the LSE, 6 makes the draft block non-causal, 7 ignores
-# the verify's page table.
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7])
+# the verify's page table, 8 drops D = rowsum(dO * O) from dS, 9 drops the
+# scale from dk, 10 decodes e4m3 with exponent bias 8, 11 drops v_scale from
+# the fp8 cache's values, 12 takes latent row 0 for a pad, 13 shortens the
+# shared prefix by one token.
+@pytest.mark.parametrize("mutant", list(range(1, 14)))
 def test_planted_mistake_is_caught(mutant, tmp_path):
     path = oracle.build(mutant=mutant, out=str(tmp_path / f"liboracle_m{mutant}.so"))
     lib = oracle.load(path)
